@@ -1,0 +1,521 @@
+#!/usr/bin/env python
+"""Benchmark of the heterogeneous-batch LoRA branch (segmented shrink/expand) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+A step applies the LoRA delta of one batch to every projection the workload names
+(mlora_apply per projection, inputs resident in HBM).  The timed region replays a
+CUDA graph holding exactly K steps that cycle through enough independent buffer
+sets (pool, X, Y) to exceed twice the L2 cache, bracketed by CUDA events on the
+launching stream.  Metric: LoRA delta tokens/s (adapter rows per second), plus
+achieved HBM GB/s of the kernel against the measured copy peak.
+
+Default workload: the Llama-3-8B q_proj decode batch (d 4096, 64 rank-16 slots,
+256 rows, Zipf(1.1) adapters, 10% base-only).  --config selects the others:
+1 tiny, 2 qproj_decode, 3 qkv_prefill, 4 mixed_mlp, 5 block70b.
+
+Under torchrun each rank runs its own batch of the same shape (independent
+problems, no collective on the data path); value = all ranks' tokens / the
+slowest rank's time.  --impl reference times the fp64 CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+
+METRIC = "LoRA delta tokens/s and achieved HBM GB/s (% roofline), decode & prefill"
+UNIT = "delta tokens/s"
+DEFAULT_CONFIG = 2
+L2_FALLBACK = 126 * 2**20
+
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
+# --------------------------------------------------------------------------- workload facts
+
+def workload_facts(W) -> dict:
+    """Algorithmic bytes and flops of one step (every projection once)."""
+    adapter = W.row_slot >= 0
+    n_l = int(adapter.sum())
+    distinct = W.referenced_slots
+    r_rows = W.slot_rank[W.row_slot[adapter]].astype(np.int64)
+    total_bytes = 0
+    flops = 0
+    per_proj = []
+    for name, d_in, d_out in W.proj_shapes:
+        w_bytes = int(sum(int(W.slot_rank[s]) * (d_in + d_out) * 2 for s in distinct))
+        x_bytes = n_l * d_in * 2
+        y_bytes = n_l * d_out * 2 * 2
+        b = w_bytes + x_bytes + y_bytes
+        per_proj.append({"name": name, "d_in": d_in, "d_out": d_out, "bytes": b,
+                         "weight_bytes": w_bytes})
+        total_bytes += b
+        flops += int(2 * r_rows.sum() * (d_in + d_out))
+    return {"adapter_rows": n_l, "distinct_adapters": int(distinct.size),
+            "bytes": total_bytes, "flops": flops, "per_projection": per_proj}
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "segmented_rank_gemm_02_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on these sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d.get(workload)
+        if e and e.get("src_hash") == kernel_source_hash():
+            return e.get("dram_bytes_per_step")
+    except Exception:
+        pass
+    return None
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML on a background thread."""
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.period = period_s
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        p = self.nvml
+        while not self._stop.is_set():
+            try:
+                mhz = p.nvmlDeviceGetClockInfo(self.h, p.NVML_CLOCK_SM)
+                try:
+                    reasons = p.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    reasons = p.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, int(reasons)))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.ok:
+            self._t.join(timeout=2)
+
+    def summary(self, t0: float, t1: float) -> dict:
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:   # very short region: nearest samples around it
+            inside = sorted(self.samples, key=lambda s: abs(s[0] - 0.5 * (t0 + t1)))[:3]
+        mhz = [s[1] for s in inside]
+        bits = 0
+        for s in inside:
+            bits |= s[2]
+        names = sorted(n for b, n in REASON_BITS.items() if bits & b and n != "gpu_idle")
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(inside)}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def cpu_oracle_rate(W, seconds: float, steps: int = 0):
+    """Time the fp64 oracle on a bounded sample of the workload (tokens/s)."""
+    import oracle
+    projs = [W.projection(j) for j in range(len(W.proj_shapes))]
+    adapter_rows = np.nonzero(W.row_slot >= 0)[0]
+    # per-row cost estimate on a small sample
+    probe = adapter_rows[: min(16, adapter_rows.size)]
+    t = time.perf_counter()
+    for p in projs:
+        oracle.reference(W, p, rows=probe)
+    per_row = (time.perf_counter() - t) / max(1, probe.size)
+    budget = seconds / max(1, steps) if steps else seconds
+    n_rows = int(max(1, min(adapter_rows.size, budget / max(per_row, 1e-9))))
+    rows = adapter_rows[:n_rows]
+    done = 0
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        for p in projs:
+            oracle.reference(W, p, rows=rows)
+        done += rows.size
+        reps += 1
+        el = time.perf_counter() - t0
+        if steps:
+            if reps >= steps:
+                break
+        elif el >= seconds * 0.5:
+            break
+    el = time.perf_counter() - t0
+    sample = (f"first {rows.size} of {adapter_rows.size} adapter rows of {W.name}, all "
+              f"{len(projs)} projection(s), {reps} pass(es)")
+    return done / el, el, sample, oracle.max_threads()
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def run_ours(args, rank: int, world: int, device_index: int):
+    import torch
+    import oracle
+    import segmented_rank_gemm_02_b200 as mlora
+    import workloads as wl
+    from segmented_rank_gemm_02_b200 import staging
+
+    torch.cuda.set_device(device_index)
+    dev = torch.device("cuda", device_index)
+    W = wl.make(args.config)
+    facts = workload_facts(W)
+    projs = [W.projection(j) for j in range(len(W.proj_shapes))]
+    meta = mlora.build_segments(W.row_slot)
+    n_proj = len(projs)
+
+    # device copies of the adapters, used to fill every pool of the ring
+    dA = [{s: mlora.as_bf16_tensor(p.A[s], dev) for s in p.A} for p in projs]
+    dB = [{s: mlora.as_bf16_tensor(p.B[s], dev) for s in p.B} for p in projs]
+    X0 = [mlora.as_bf16_tensor(p.X, dev) for p in projs]
+    Y0 = [mlora.as_bf16_tensor(p.Y0, dev) for p in projs]
+
+    def new_set():
+        out = []
+        for j, p in enumerate(projs):
+            pool = mlora.Pool(p.d_in, p.d_out, W.n_slots, W.r_max)
+            for s in sorted(p.A):
+                pool.load_slot(s, int(W.slot_rank[s]), float(W.slot_alpha[s]), dA[j][s], dB[j][s])
+            m = dict(meta)
+            m["ranks"] = np.array([0 if s < 0 else W.slot_rank[s] for s in meta["slots"]], np.int32)
+            segs = mlora.DeviceSegments(m, W.n_rows, dev)
+            out.append({"pool": pool, "segs": segs, "X": X0[j].clone(), "Y": Y0[j].clone()})
+        return out
+
+    rb = next(b for b in (8, 16, 32, 64) if b >= W.r_max)
+    pool_bytes = sum(W.n_slots * 2 * (((rb * (p.d_in + p.d_out) + 127) // 128) * 128)
+                     for p in projs)
+    act_bytes = sum(W.n_rows * (p.d_in + p.d_out) * 2 for p in projs)
+    set_bytes = pool_bytes + act_bytes
+    try:
+        l2 = int(torch.cuda.get_device_properties(dev).L2_cache_size)
+    except Exception:
+        l2 = L2_FALLBACK
+    n_sets = max(1, math.ceil(2 * l2 / set_bytes))
+    sets = [new_set() for _ in range(n_sets)]
+    torch.cuda.synchronize()
+
+    # parity on sampled rows of a fresh set (outside any timed region)
+    rows = np.unique(np.concatenate([meta["token_indices"][meta["offsets"][:-1]],
+                                     np.nonzero(W.row_slot >= 0)[0][:8]]))
+    rows = rows[W.row_slot[rows] >= 0][:48]
+    worst = 0.0
+    for j, p in enumerate(projs):
+        e = sets[0][j]
+        mlora.apply(e["pool"], e["segs"], e["X"], e["Y"])
+        assert e["pool"].check() == 0
+        got = oracle.bf16_to_f64(mlora.bf16_bits(e["Y"][torch.as_tensor(rows, device=dev)]))
+        ref = oracle.reference(W, p, rows=rows)
+        worst = max(worst, float(np.max(np.abs(got - ref) / (1e-2 * (1 + np.abs(ref))))))
+        e["Y"].copy_(Y0[j])
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(k):
+        for j in range(n_proj):
+            e = sets[k % n_sets][j]
+            mlora.apply(e["pool"], e["segs"], e["X"], e["Y"], stream=stream)
+
+    # warm-up steps (eager), then capture exactly K steps into one graph
+    with torch.cuda.stream(stream):
+        for k in range(args.warmup):
+            step(k)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for k in range(args.steps):
+            step(k)
+    with torch.cuda.stream(stream):
+        graph.replay()   # first replay uploads the graph; not timed
+    stream.synchronize()
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    def timed():
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            graph.replay()
+            end.record(stream)
+        torch.cuda.synchronize()
+        t1 = time.perf_counter()
+        if dist:
+            dist.barrier()
+        return start.elapsed_time(end), t0, t1
+
+    with ClockSampler(device_index) as clk:
+        ms, t0, t1 = timed()
+    clocks = clk.summary(t0, t1)
+    if set(clocks.get("reasons", [])) & BAD_REASONS:
+        with ClockSampler(device_index) as clk:
+            ms, t0, t1 = timed()
+        clocks = clk.summary(t0, t1)
+        clocks["remeasured"] = True
+
+    ms_max = ms
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    del graph
+
+    # end to end through the public API with host buffers: host grouping, H2D of the
+    # metadata, X and Y0 from pinned memory, mlora_apply, D2H of Y
+    e2e = run_e2e(args, W, projs, meta, sets[0], dev, stream)
+
+    tokens = facts["adapter_rows"]
+    steps = args.steps
+    sec = ms_max / 1e3
+    value = tokens * steps * world / sec
+    per_launch_s = (ms / 1e3) / steps
+    peaks = measured_peaks()
+    achieved = facts["bytes"] / per_launch_s / 1e9
+    traffic = recorded_traffic(W.name)
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": W.name, "projections": [p[0] for p in W.proj_shapes],
+            "shapes": [[p[1], p[2]] for p in W.proj_shapes], "rows": W.n_rows,
+            "adapter_rows": tokens, "slots": W.n_slots,
+            "distinct_adapters": facts["distinct_adapters"],
+            "ranks": sorted(set(int(r) for r in W.slot_rank[W.referenced_slots])),
+            "global_batch": tokens * world, "parallelism": f"replicas x{world} (independent batches)",
+            "l2": f"rotating {n_sets} buffer set(s) of {set_bytes / 2**20:.0f} MiB "
+                  f"({n_sets * set_bytes / 2**20:.0f} MiB > 2x {l2 / 2**20:.0f} MiB L2)",
+            "timing": "one CUDA graph of exactly K steps, CUDA events on its stream",
+        },
+        "roofline": {
+            "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+            "peak_source": peaks["source"], "algorithmic_bytes_per_step": facts["bytes"],
+            "flops_per_step": facts["flops"],
+            "tensor_frac": facts["flops"] / per_launch_s / 1e12 / peaks["bf16_tflops"],
+            "kernel": "lora_tile_kernel (fused apply)",
+        },
+        "e2e": e2e,
+        "gpu_launches": steps * n_proj,
+        "clocks": clocks,
+        "parity": {"rows_checked": int(rows.size), "max_err_over_tolerance": worst},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, el, sample, cores = cpu_oracle_rate(W, args.cpu_seconds)
+        result["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                  "sample": sample, "seconds": el}
+    for s in sets:
+        for e in s:
+            e["pool"].close()
+    return result
+
+
+def run_e2e(args, W, projs, meta0, entries, dev, stream):
+    import torch
+    import segmented_rank_gemm_02_b200 as mlora
+
+    row_slot = np.ascontiguousarray(W.row_slot, np.int32)
+    S_max = W.n_rows
+    n = W.n_rows
+    # pinned host staging, double-buffered: [offsets S+1 | slots S | ranks S | token_indices n]
+    meta_host = [torch.empty(3 * S_max + 1 + n, dtype=torch.int32).pin_memory() for _ in range(2)]
+    meta_ready = [None, None]   # event after the H2D copy that last read each buffer
+    meta_dev = torch.empty_like(meta_host[0], device=dev)
+    Xh = [torch.from_numpy(p.X.view(np.int16)).view(torch.bfloat16).pin_memory() for p in projs]
+    Y0h = [torch.from_numpy(p.Y0.view(np.int16)).view(torch.bfloat16).pin_memory() for p in projs]
+    Yout = [torch.empty_like(y).pin_memory() for y in Y0h]
+    pool0 = entries[0]["pool"]
+
+    counter = [0]
+
+    def one_step():
+        b = counter[0] & 1
+        counter[0] += 1
+        if meta_ready[b] is not None:
+            meta_ready[b].synchronize()                  # the DMA has read this buffer
+        m = mlora.build_segments(row_slot, pool0)        # host grouping (C, via the ABI)
+        S = int(m["slots"].size)
+        mh = meta_host[b].numpy()
+        mh[:S + 1] = m["offsets"]
+        mh[S_max + 1:S_max + 1 + S] = m["slots"]
+        mh[2 * S_max + 1:2 * S_max + 1 + S] = m["ranks"]
+        mh[3 * S_max + 1:] = m["token_indices"]
+        meta_dev.copy_(meta_host[b], non_blocking=True)
+        ev = torch.cuda.Event()
+        ev.record(stream)
+        meta_ready[b] = ev
+        segs = mlora.SegmentsStruct(S, n, n, int(m["max_segment_rows"]),
+                                    meta_dev.data_ptr(), meta_dev.data_ptr() + 4 * (S_max + 1),
+                                    meta_dev.data_ptr() + 4 * (2 * S_max + 1), None,
+                                    meta_dev.data_ptr() + 4 * (3 * S_max + 1))
+        holder = type("S", (), {})()
+        holder.struct = segs
+        for j, e in enumerate(entries):
+            e["X"].copy_(Xh[j], non_blocking=True)
+            e["Y"].copy_(Y0h[j], non_blocking=True)
+            mlora.apply(e["pool"], holder, e["X"], e["Y"], stream=stream)
+            Yout[j].copy_(e["Y"], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, min(args.warmup, 10))):
+            one_step()
+    torch.cuda.synchronize()
+    t = time.perf_counter()
+    with torch.cuda.stream(stream):
+        one_step()
+    torch.cuda.synchronize()
+    est = time.perf_counter() - t
+    steps = int(max(3, min(args.steps, args.e2e_seconds / max(est, 1e-6))))
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(steps):
+            one_step()
+        end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    tokens = int((W.row_slot >= 0).sum())
+    h2d = meta_host[0].numel() * 4 + sum(x.numel() * 2 + y.numel() * 2 for x, y in zip(Xh, Y0h))
+    d2h = sum(y.numel() * 2 for y in Yout)
+    return {"value": tokens * steps / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": ms / steps,
+            "includes": "host grouping (mlora_build_segments), H2D metadata+X+Y0 from pinned "
+                        "memory, mlora_apply, D2H Y"}
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank: int, world: int):
+    import workloads as wl
+    W = wl.make(args.config)
+    facts = workload_facts(W)
+    budget = float(args.cpu_seconds) if args.cpu_seconds else 60.0
+    # warm-up passes are bounded samples too (not timed)
+    if args.warmup:
+        cpu_oracle_rate(W, budget * 0.05, steps=1)
+    rate, el, sample, cores = cpu_oracle_rate(W, budget, steps=max(1, args.steps))
+    return {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el * 1e3 / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": W.name, "adapter_rows": facts["adapter_rows"],
+                   "projections": [p[0] for p in W.proj_shapes]},
+        "cpu_baseline": {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--e2e-seconds", type=float, default=5.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return 0
+
+    pg = False
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+        pg = True
+    try:
+        result = run_ours(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(result), flush=True)
+    finally:
+        if pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

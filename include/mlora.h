@@ -1,0 +1,193 @@
+/*
+ * mlora.h -- C ABI of the heterogeneous-batch LoRA branch for B200 (sm_100a).
+ *
+ * The operation (page "Multi-LoRA Serving: adapter batching", charlestar.github.io,
+ * sections "LoRA on one Linear layer", "The math of a mixed batch" and
+ * "What metadata a segmented kernel needs"):
+ *
+ *   A linear layer Y = X W^T (W in R^{d_out x d_in}) gains, per adapter a, the
+ *   low-rank branch  s_a (X A_a^T) B_a^T  with A_a in R^{r x d_in},
+ *   B_a in R^{d_out x r} and s_a = alpha_a / r_a.  The caller computes the shared
+ *   base output Y0 = X W^T for every row; this library adds each row's own
+ *   adapter delta in place:
+ *
+ *       H[p, j]  = sum_k X[t, k] A_a[j, k]            (shrink, fp32 accumulation)
+ *       Y[t, o]  = bf16( Y0[t, o] + s_g sum_j H[p, j] B_a[o, j] )   (expand, scatter)
+ *
+ *   where the rows are grouped into segments g (slot a = adapter_slots[g];
+ *   slot -1 = base model only) and grouped position p of segment g maps to the
+ *   original row t = token_indices[p].  Rows of base segments, rows in no
+ *   segment and rows of rejected segments are never written (bit-identical Y0).
+ *
+ * Adapters live in a pre-allocated pool of fixed-stride slots indexed by slot
+ * number (page "LoRA/QLoRA multi-tenant serving", ybb.press, section 1.1, unified
+ * size alignment).  Ranks up to 64 are stored and computed at their own rank
+ * bucket (8, 16, 32 or 64; page "Multi-LoRA Serving: adapter batching", section
+ * "How LoRA ranks affect the kernel"), never padded to the pool's maximum.
+ *
+ * Conventions for every entry point:
+ *   - bf16 tensors are IEEE bfloat16 bit patterns (2 bytes per element),
+ *     row-major with an element row stride (ld*).
+ *   - "device" pointers are CUDA device pointers of the device current when the
+ *     pool was created; calls must be made with that device current.
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Kernels are launched asynchronously on it; the caller keeps every buffer
+ *     alive until the stream has passed the call.
+ *   - Errors the host can see (null or misaligned pointers, bad sizes, slot or
+ *     rank out of range) return at once with nothing launched.  Errors only the
+ *     device can see (bad metadata contents) make the kernels skip the offending
+ *     segment or row -- never trap -- and set bits in the pool's device status
+ *     word, which mlora_pool_check reports.
+ *   - Limits: d_in and d_out multiples of 8 (16-byte rows); rank 1..64;
+ *     X, Y 16-byte aligned with ld* a multiple of 8; H 16-byte aligned with
+ *     ldh a multiple of 4.
+ */
+#ifndef MLORA_H
+#define MLORA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MLORA_OK = 0,
+    MLORA_ERR_INVALID_ARG = 1,     /* null/misaligned pointer, size or index out of range */
+    MLORA_ERR_UNSUPPORTED = 2,     /* shape outside the supported limits, no sm_100 device */
+    MLORA_ERR_OUT_OF_MEMORY = 3,   /* device allocation failed */
+    MLORA_ERR_BAD_METADATA = 4,    /* mlora_pool_check: the device flagged bad metadata */
+    MLORA_ERR_CUDA = 5             /* a CUDA runtime call failed */
+} mlora_status;
+
+/* Device status bits reported by mlora_pool_check. */
+#define MLORA_FLAG_BAD_OFFSETS  1u   /* offsets decreasing, negative or beyond n_tokens */
+#define MLORA_FLAG_BAD_SLOT     2u   /* adapter slot < -1 or >= n_slots */
+#define MLORA_FLAG_BAD_RANK     4u   /* ranks[g] differs from the rank loaded in the slot */
+#define MLORA_FLAG_BAD_ROW      8u   /* token_indices entry outside [0, n_rows) */
+#define MLORA_FLAG_SLOT_EMPTY  16u   /* segment refers to a slot with nothing loaded */
+#define MLORA_FLAG_TIMEOUT     32u   /* an internal wait gave up (results of that tile invalid) */
+
+/* Opaque adapter pool.  Owns its device slot buffer, slot table and status word. */
+typedef struct mlora_pool mlora_pool;
+
+/*
+ * Segment metadata for one call (page "Multi-LoRA Serving: adapter batching",
+ * section "What metadata a segmented kernel needs": segment_offsets,
+ * adapter_slots, token_indices, ranks, scales).  All arrays are DEVICE memory,
+ * owned by the caller, read-only to the library.
+ */
+typedef struct {
+    int32_t n_segments;              /* S >= 0 */
+    int32_t n_rows;                  /* rows of X and Y; token_indices values must be < n_rows */
+    int32_t n_tokens;                /* grouped positions: length of token_indices
+                                        (== segment_offsets[S] for well-formed metadata);
+                                        rows of H in mlora_shrink / mlora_expand */
+    int32_t max_segment_rows;        /* host hint: an upper bound on the length of any
+                                        adapter segment, or 0 if unknown.  Only steers
+                                        kernel choice; a wrong hint never changes results. */
+    const int32_t *segment_offsets;  /* [S+1], non-decreasing, offsets[0] >= 0 */
+    const int32_t *adapter_slots;    /* [S], -1 = base model only, else 0..n_slots-1 */
+    const int32_t *ranks;            /* [S] or NULL; if given, must equal the slot's rank
+                                        (entries of base segments are ignored) */
+    const float *scales;             /* [S] or NULL (then each slot's alpha / rank) */
+    const int32_t *token_indices;    /* [n_tokens] grouped position -> original row, no
+                                        duplicates; NULL = identity (p -> row p) */
+} mlora_segments;
+
+/*
+ * Create a pool of n_slots adapter slots for one projection (d_in -> d_out) with
+ * ranks up to r_max (1..64).  Allocates n_slots * bucket(r_max) * (d_in + d_out)
+ * bf16 elements of device memory on the current device; all slots start empty.
+ * Returns MLORA_ERR_OUT_OF_MEMORY if the allocation fails.
+ */
+mlora_status mlora_pool_create(int32_t d_in, int32_t d_out, int32_t n_slots, int32_t r_max,
+                               mlora_pool **out);
+
+/* Free the pool (synchronises the device first).  NULL is accepted. */
+mlora_status mlora_pool_destroy(mlora_pool *pool);
+
+/*
+ * Load an adapter into a slot: A is bf16 [rank, d_in] row-major, B is bf16
+ * [d_out, rank] row-major (the PEFT layout of lora_A / lora_B), both in host
+ * memory (src_is_device = 0) or device memory (1).  The slot is repacked into
+ * the pool's internal layout and zero-filled up to its rank bucket.  The copy is
+ * stream-ordered on `stream`; host sources may be reused when the call returns.
+ * On any error the slot keeps its previous contents and rank.
+ */
+mlora_status mlora_pool_load_slot(mlora_pool *pool, int32_t slot, int32_t rank, float alpha,
+                                  const void *A, const void *B, int32_t src_is_device,
+                                  void *stream);
+
+/* Mark a slot empty (stream-ordered).  Segments that use it are then rejected. */
+mlora_status mlora_pool_clear_slot(mlora_pool *pool, int32_t slot, void *stream);
+
+/* Host-side view of a slot: rank (0 if empty), alpha, and the parameter count
+ * r (d_in + d_out) (page "Multi-LoRA Serving: adapter batching", section "LoRA on
+ * one Linear layer").  Any output pointer may be NULL. */
+mlora_status mlora_pool_slot_info(const mlora_pool *pool, int32_t slot, int32_t *rank,
+                                  float *alpha, int64_t *params);
+
+/* Pool geometry.  Any output pointer may be NULL. */
+mlora_status mlora_pool_shape(const mlora_pool *pool, int32_t *d_in, int32_t *d_out,
+                              int32_t *n_slots, int32_t *r_max);
+
+/*
+ * Synchronise `stream`, read and clear the pool's device status word.  Returns
+ * MLORA_ERR_BAD_METADATA if any MLORA_FLAG_* bit was set since the last check
+ * (the bits are stored to *flags if flags is not NULL), else MLORA_OK.
+ */
+mlora_status mlora_pool_check(mlora_pool *pool, void *stream, uint32_t *flags);
+
+/*
+ * Shrink alone: H[p, 0:r] = X[t_p, :] A_a^T for every grouped position p of every
+ * adapter segment, fp32, grouped order (row stride ldh >= r).  X is device bf16
+ * [n_rows, d_in] (row stride ldx); H is device fp32 [n_tokens, ldh].  Entries of
+ * base or rejected segments and columns >= r are not written.
+ */
+mlora_status mlora_shrink(mlora_pool *pool, const mlora_segments *segs, const void *X,
+                          int64_t ldx, float *H, int64_t ldh, void *stream);
+
+/*
+ * Expand alone: Y[t_p, :] = bf16(Y[t_p, :] + s_g H[p, 0:r] B_a^T) for every grouped
+ * position p of every adapter segment.  H is device fp32 [n_tokens, ldh] in
+ * grouped order; Y is device bf16 [n_rows, d_out] (row stride ldy), updated in
+ * place.
+ */
+mlora_status mlora_expand(mlora_pool *pool, const mlora_segments *segs, const float *H,
+                          int64_t ldh, void *Y, int64_t ldy, void *stream);
+
+/*
+ * Fused shrink + expand: Y[t, :] = bf16(Y0[t, :] + s_g (X[t, :] A_a^T) B_a^T) in
+ * place on the caller's base output Y (= Y0 = X W^T on entry).  The rank-r
+ * intermediate stays on chip.  X: device bf16 [n_rows, d_in]; Y: device bf16
+ * [n_rows, d_out].
+ */
+mlora_status mlora_apply(mlora_pool *pool, const mlora_segments *segs, const void *X,
+                         int64_t ldx, void *Y, int64_t ldy, void *stream);
+
+/*
+ * Host helper: group rows by slot (row_slots[t] = slot of row t, -1 = base).
+ * Segments come in the order their slot first appears; rows keep their original
+ * order inside a segment.  Outputs are HOST arrays the caller sizes:
+ * offsets[n_rows + 1], slots[n_rows], token_indices[n_rows].  *n_segments gets S,
+ * *max_segment_rows (may be NULL) the longest adapter segment.  If pool and
+ * ranks are both non-NULL, ranks[n_rows] gets each segment's slot rank (0 for
+ * base).  Slots are not range-checked here (the device checks them).
+ */
+mlora_status mlora_build_segments(const int32_t *row_slots, int32_t n_rows,
+                                  int32_t *offsets, int32_t *slots, int32_t *token_indices,
+                                  int32_t *n_segments, int32_t *max_segment_rows,
+                                  const mlora_pool *pool, int32_t *ranks);
+
+/* Static description of a status code. */
+const char *mlora_status_string(mlora_status status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int32_t mlora_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLORA_H */

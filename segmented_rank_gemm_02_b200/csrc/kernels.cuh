@@ -1,0 +1,75 @@
+// kernels.cuh -- interface between the host library and the sm_100a kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace mlora {
+
+enum TileMode : int { MODE_APPLY = 0, MODE_SHRINK = 1, MODE_EXPAND = 2 };
+
+// Rows of one work tile of the segmented kernel (one m16 MMA tile).
+constexpr int kTileRows = 16;
+
+// Device status bits (same values as the MLORA_FLAG_* macros of the public header).
+constexpr unsigned kFlagBadOffsets = 1u;
+constexpr unsigned kFlagBadSlot = 2u;
+constexpr unsigned kFlagBadRank = 4u;
+constexpr unsigned kFlagBadRow = 8u;
+constexpr unsigned kFlagSlotEmpty = 16u;
+constexpr unsigned kFlagTimeout = 32u;
+
+// Smallest rank bucket (8, 16, 32, 64) holding rank r; 0 if r is out of range.
+__host__ __device__ constexpr int rank_bucket(int r)
+{
+    return r <= 0 ? 0 : r <= 8 ? 8 : r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : 0;
+}
+
+// Everything one launch of the segmented tile kernel needs.  Passed by value.
+struct TileParams {
+    // adapter pool: slot a's A block starts at pool + a * slot_stride and holds
+    // [d_in/8][R][8] bf16 (R = bucket of the slot's rank); its B block starts
+    // b_offset elements later and holds [R/8][d_out][8] bf16.
+    const __nv_bfloat16 *pool;
+    int64_t slot_stride;
+    int64_t b_offset;
+    const int32_t *slot_rank;   // [n_slots], 0 = empty
+    const float *slot_scale;    // [n_slots], alpha / rank
+    int32_t n_slots;
+    unsigned int *status;       // device status word (MLORA_FLAG_* bits)
+    int32_t d_in, d_out;
+    // segment metadata (device)
+    int32_t n_segments, n_rows, n_tokens;
+    const int32_t *offsets;
+    const int32_t *slots;
+    const int32_t *ranks;       // may be null
+    const float *scales;        // may be null
+    const int32_t *token_indices;  // may be null (identity)
+    // tensors
+    const __nv_bfloat16 *X;
+    int64_t ldx;
+    __nv_bfloat16 *Y;
+    int64_t ldy;
+    float *H;
+    int64_t ldh;
+    // decomposition: CTA c of a cluster owns d_in columns [c*k_slice, (c+1)*k_slice)
+    // for the shrink and d_out columns [c*n_slice, (c+1)*n_slice) for the expand.
+    int32_t k_slice, n_slice;
+};
+
+// Launch `n_clusters` clusters of `cluster` CTAs of the tile kernel for the pool's
+// largest rank bucket `rmax_bucket` (8/16/32/64) in mode `mode`.
+cudaError_t launch_tile_kernel(int mode, int rmax_bucket, const TileParams &p, int cluster,
+                               int n_clusters, cudaStream_t stream);
+
+// Set per-kernel attributes (dynamic shared memory) on the current device.
+cudaError_t prepare_tile_kernels();
+
+// Repack one adapter from the PEFT layout into a pool slot and publish its rank/scale.
+cudaError_t launch_repack_slot(__nv_bfloat16 *slot_base, int64_t b_offset, int R, int rank,
+                               int d_in, int d_out, const __nv_bfloat16 *A_src,
+                               const __nv_bfloat16 *B_src, int32_t *slot_rank_entry,
+                               float *slot_scale_entry, float scale, cudaStream_t stream);
+
+}  // namespace mlora

@@ -1,0 +1,429 @@
+// mlora.cu -- host side of the C ABI declared in include/mlora.h.
+//
+// The adapter pool (page "LoRA/QLoRA multi-tenant serving", ybb.press, section 1.1:
+// one pre-allocated buffer, fixed per-adapter size, O(1) slot addressing) and the
+// argument checks, kernel choice and launches of mlora_shrink / mlora_expand /
+// mlora_apply.  The grouping helper mlora_build_segments follows the metadata
+// layout of page "Multi-LoRA Serving: adapter batching", section "What metadata a
+// segmented kernel needs".
+#include "mlora.h"
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <unordered_map>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "kernels.cuh"
+
+struct mlora_pool {
+    int device;
+    int32_t d_in, d_out, n_slots, r_max, r_bucket_max;
+    int64_t slot_stride;   // elements per slot
+    int64_t b_offset;      // elements from a slot's start to its B block
+    __nv_bfloat16 *buf;
+    int32_t *d_rank;
+    float *d_scale;
+    unsigned int *d_status;
+    std::vector<int32_t> h_rank;
+    std::vector<float> h_alpha;
+};
+
+namespace {
+
+using mlora::rank_bucket;
+
+// Runs the body with the pool's device current, restoring the caller's device.
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev)
+    {
+        if (cudaGetDevice(&prev) != cudaSuccess) {
+            ok = false;
+            return;
+        }
+        if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+    }
+    ~DeviceGuard()
+    {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+std::mutex g_prep_mutex;
+bool g_prepared[128] = {};
+
+mlora_status prepare_device(int dev)
+{
+    std::lock_guard<std::mutex> lock(g_prep_mutex);
+    if (dev < 0 || dev >= 128) return MLORA_ERR_INVALID_ARG;
+    if (g_prepared[dev]) return MLORA_OK;
+    if (mlora::prepare_tile_kernels() != cudaSuccess) return MLORA_ERR_CUDA;
+    g_prepared[dev] = true;
+    return MLORA_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// Cluster size: enough CTAs per tile to spread one adapter's A and B over ~1K
+// columns each, at most 8 (the portable cluster size), and every CTA must own at
+// least one 16-column group of d_in and one 8-column group of d_out.
+int choose_cluster(int d_in, int d_out)
+{
+    int c = (int)std::min<int64_t>(8, std::max<int64_t>(1, (int64_t)(d_in + d_out + 1023) / 1024));
+    while (c > 1 && (round_up((d_in + c - 1) / c, 16) * (c - 1) >= d_in ||
+                     round_up((d_out + c - 1) / c, 8) * (c - 1) >= d_out))
+        --c;
+    return c;
+}
+
+mlora_status check_segments(const mlora_pool *pool, const mlora_segments *s)
+{
+    if (pool == nullptr || s == nullptr) return MLORA_ERR_INVALID_ARG;
+    if (s->n_segments < 0 || s->n_rows < 0 || s->n_tokens < 0) return MLORA_ERR_INVALID_ARG;
+    if (s->n_segments > 0 && (s->segment_offsets == nullptr || s->adapter_slots == nullptr))
+        return MLORA_ERR_INVALID_ARG;
+    return MLORA_OK;
+}
+
+mlora::TileParams base_params(const mlora_pool *pool, const mlora_segments *s)
+{
+    mlora::TileParams p{};
+    p.pool = pool->buf;
+    p.slot_stride = pool->slot_stride;
+    p.b_offset = pool->b_offset;
+    p.slot_rank = pool->d_rank;
+    p.slot_scale = pool->d_scale;
+    p.n_slots = pool->n_slots;
+    p.status = pool->d_status;
+    p.d_in = pool->d_in;
+    p.d_out = pool->d_out;
+    p.n_segments = s->n_segments;
+    p.n_rows = s->n_rows;
+    p.n_tokens = s->n_tokens;
+    p.offsets = s->segment_offsets;
+    p.slots = s->adapter_slots;
+    p.ranks = s->ranks;
+    p.scales = s->scales;
+    p.token_indices = s->token_indices;
+    return p;
+}
+
+mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::TileParams &p,
+                    void *stream)
+{
+    const int c = choose_cluster(pool->d_in, pool->d_out);
+    p.k_slice = (int32_t)round_up((pool->d_in + c - 1) / c, 16);
+    p.n_slice = (int32_t)round_up((pool->d_out + c - 1) / c, 8);
+    // Upper bound on the number of 16-row tiles of well-formed metadata.
+    const int64_t tiles = (int64_t)s->n_segments + (int64_t)s->n_tokens / mlora::kTileRows + 1;
+    if (tiles * c > 0x7fffffff) return MLORA_ERR_UNSUPPORTED;
+    mlora_status st = prepare_device(pool->device);
+    if (st != MLORA_OK) return st;
+    cudaError_t e = mlora::launch_tile_kernel(mode, pool->r_bucket_max, p, c, (int)tiles,
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MLORA_OK : MLORA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *mlora_status_string(mlora_status status)
+{
+    switch (status) {
+    case MLORA_OK: return "ok";
+    case MLORA_ERR_INVALID_ARG: return "invalid argument";
+    case MLORA_ERR_UNSUPPORTED: return "unsupported shape or device";
+    case MLORA_ERR_OUT_OF_MEMORY: return "out of device memory";
+    case MLORA_ERR_BAD_METADATA: return "device flagged bad segment metadata";
+    case MLORA_ERR_CUDA: return "CUDA runtime error";
+    }
+    return "unknown status";
+}
+
+int32_t mlora_version(void) { return 100; }
+
+mlora_status mlora_pool_create(int32_t d_in, int32_t d_out, int32_t n_slots, int32_t r_max,
+                               mlora_pool **out)
+{
+    if (out == nullptr) return MLORA_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (d_in <= 0 || d_out <= 0 || n_slots <= 0 || r_max <= 0) return MLORA_ERR_INVALID_ARG;
+    if (d_in % 8 != 0 || d_out % 8 != 0 || r_max > 64) return MLORA_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLORA_ERR_CUDA;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MLORA_ERR_CUDA;
+    if (prop.major != 10 || prop.minor != 0) return MLORA_ERR_UNSUPPORTED;   // built for sm_100a
+
+    const int rb = rank_bucket(r_max);
+    const int64_t stride = round_up((int64_t)rb * (d_in + d_out), 128);   // 256-byte slots
+    const double bytes = (double)stride * 2.0 * n_slots;
+    if (bytes > 9.0e18) return MLORA_ERR_OUT_OF_MEMORY;
+
+    mlora_pool *pool = new (std::nothrow) mlora_pool();
+    if (pool == nullptr) return MLORA_ERR_OUT_OF_MEMORY;
+    pool->device = dev;
+    pool->d_in = d_in;
+    pool->d_out = d_out;
+    pool->n_slots = n_slots;
+    pool->r_max = r_max;
+    pool->r_bucket_max = rb;
+    pool->slot_stride = stride;
+    pool->b_offset = (int64_t)rb * d_in;
+    pool->buf = nullptr;
+    pool->d_rank = nullptr;
+    pool->d_scale = nullptr;
+    pool->d_status = nullptr;
+    pool->h_rank.assign(n_slots, 0);
+    pool->h_alpha.assign(n_slots, 0.f);
+
+    mlora_status st = MLORA_OK;
+    if (cudaMalloc(&pool->buf, (size_t)stride * 2 * n_slots) != cudaSuccess ||
+        cudaMalloc(&pool->d_rank, sizeof(int32_t) * n_slots) != cudaSuccess ||
+        cudaMalloc(&pool->d_scale, sizeof(float) * n_slots) != cudaSuccess ||
+        cudaMalloc(&pool->d_status, sizeof(unsigned int)) != cudaSuccess) {
+        st = MLORA_ERR_OUT_OF_MEMORY;
+    } else if (cudaMemset(pool->d_rank, 0, sizeof(int32_t) * n_slots) != cudaSuccess ||
+               cudaMemset(pool->d_scale, 0, sizeof(float) * n_slots) != cudaSuccess ||
+               cudaMemset(pool->d_status, 0, sizeof(unsigned int)) != cudaSuccess ||
+               cudaDeviceSynchronize() != cudaSuccess) {
+        st = MLORA_ERR_CUDA;
+    } else {
+        st = prepare_device(dev);
+    }
+    if (st != MLORA_OK) {
+        cudaGetLastError();   // clear a sticky allocation error
+        mlora_pool_destroy(pool);
+        return st;
+    }
+    *out = pool;
+    return MLORA_OK;
+}
+
+mlora_status mlora_pool_destroy(mlora_pool *pool)
+{
+    if (pool == nullptr) return MLORA_OK;
+    DeviceGuard guard(pool->device);
+    cudaDeviceSynchronize();
+    if (pool->buf) cudaFree(pool->buf);
+    if (pool->d_rank) cudaFree(pool->d_rank);
+    if (pool->d_scale) cudaFree(pool->d_scale);
+    if (pool->d_status) cudaFree(pool->d_status);
+    delete pool;
+    return MLORA_OK;
+}
+
+mlora_status mlora_pool_shape(const mlora_pool *pool, int32_t *d_in, int32_t *d_out,
+                              int32_t *n_slots, int32_t *r_max)
+{
+    if (pool == nullptr) return MLORA_ERR_INVALID_ARG;
+    if (d_in) *d_in = pool->d_in;
+    if (d_out) *d_out = pool->d_out;
+    if (n_slots) *n_slots = pool->n_slots;
+    if (r_max) *r_max = pool->r_max;
+    return MLORA_OK;
+}
+
+mlora_status mlora_pool_load_slot(mlora_pool *pool, int32_t slot, int32_t rank, float alpha,
+                                  const void *A, const void *B, int32_t src_is_device,
+                                  void *stream)
+{
+    if (pool == nullptr || A == nullptr || B == nullptr) return MLORA_ERR_INVALID_ARG;
+    if (slot < 0 || slot >= pool->n_slots) return MLORA_ERR_INVALID_ARG;
+    if (rank < 1 || rank > pool->r_max) return MLORA_ERR_INVALID_ARG;
+    if (!std::isfinite(alpha)) return MLORA_ERR_INVALID_ARG;
+    if (src_is_device && ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B)) & 1u))
+        return MLORA_ERR_INVALID_ARG;
+    DeviceGuard guard(pool->device);
+    if (!guard.ok) return MLORA_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int R = rank_bucket(rank);
+    const size_t a_elems = (size_t)rank * pool->d_in;
+    const size_t b_elems = (size_t)pool->d_out * rank;
+    const __nv_bfloat16 *a_src = static_cast<const __nv_bfloat16 *>(A);
+    const __nv_bfloat16 *b_src = static_cast<const __nv_bfloat16 *>(B);
+    __nv_bfloat16 *staging = nullptr;
+    if (!src_is_device) {
+        // Copy into stream-ordered staging first: a failed copy leaves the slot untouched.
+        if (cudaMallocAsync(&staging, (a_elems + b_elems) * 2, st) != cudaSuccess) {
+            cudaGetLastError();
+            return MLORA_ERR_OUT_OF_MEMORY;
+        }
+        if (cudaMemcpyAsync(staging, A, a_elems * 2, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+            cudaMemcpyAsync(staging + a_elems, B, b_elems * 2, cudaMemcpyHostToDevice, st) !=
+                cudaSuccess) {
+            cudaGetLastError();
+            cudaFreeAsync(staging, st);
+            return MLORA_ERR_CUDA;
+        }
+        a_src = staging;
+        b_src = staging + a_elems;
+    }
+    const float scale = alpha / (float)rank;
+    cudaError_t e = mlora::launch_repack_slot(pool->buf + (int64_t)slot * pool->slot_stride,
+                                              pool->b_offset, R, rank, pool->d_in, pool->d_out,
+                                              a_src, b_src, pool->d_rank + slot,
+                                              pool->d_scale + slot, scale, st);
+    if (staging) cudaFreeAsync(staging, st);
+    if (e != cudaSuccess) return MLORA_ERR_CUDA;
+    pool->h_rank[slot] = rank;
+    pool->h_alpha[slot] = alpha;
+    return MLORA_OK;
+}
+
+mlora_status mlora_pool_clear_slot(mlora_pool *pool, int32_t slot, void *stream)
+{
+    if (pool == nullptr || slot < 0 || slot >= pool->n_slots) return MLORA_ERR_INVALID_ARG;
+    DeviceGuard guard(pool->device);
+    if (!guard.ok) return MLORA_ERR_CUDA;
+    if (cudaMemsetAsync(pool->d_rank + slot, 0, sizeof(int32_t),
+                        static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return MLORA_ERR_CUDA;
+    pool->h_rank[slot] = 0;
+    pool->h_alpha[slot] = 0.f;
+    return MLORA_OK;
+}
+
+mlora_status mlora_pool_slot_info(const mlora_pool *pool, int32_t slot, int32_t *rank,
+                                  float *alpha, int64_t *params)
+{
+    if (pool == nullptr || slot < 0 || slot >= pool->n_slots) return MLORA_ERR_INVALID_ARG;
+    const int32_t r = pool->h_rank[slot];
+    if (rank) *rank = r;
+    if (alpha) *alpha = pool->h_alpha[slot];
+    if (params) *params = (int64_t)r * ((int64_t)pool->d_in + pool->d_out);
+    return MLORA_OK;
+}
+
+mlora_status mlora_pool_check(mlora_pool *pool, void *stream, uint32_t *flags)
+{
+    if (pool == nullptr) return MLORA_ERR_INVALID_ARG;
+    DeviceGuard guard(pool->device);
+    if (!guard.ok) return MLORA_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned int h = 0;
+    if (cudaMemcpyAsync(&h, pool->d_status, sizeof h, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemsetAsync(pool->d_status, 0, sizeof(unsigned int), st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return MLORA_ERR_CUDA;
+    if (flags) *flags = h;
+    return h ? MLORA_ERR_BAD_METADATA : MLORA_OK;
+}
+
+mlora_status mlora_apply(mlora_pool *pool, const mlora_segments *segs, const void *X, int64_t ldx,
+                         void *Y, int64_t ldy, void *stream)
+{
+    mlora_status st = check_segments(pool, segs);
+    if (st != MLORA_OK) return st;
+    if (segs->n_segments == 0 || segs->n_tokens == 0) return MLORA_OK;
+    if (X == nullptr || Y == nullptr || !aligned16(X) || !aligned16(Y)) return MLORA_ERR_INVALID_ARG;
+    if (ldx < pool->d_in || ldx % 8 != 0 || ldy < pool->d_out || ldy % 8 != 0)
+        return MLORA_ERR_INVALID_ARG;
+    DeviceGuard guard(pool->device);
+    if (!guard.ok) return MLORA_ERR_CUDA;
+    mlora::TileParams p = base_params(pool, segs);
+    p.X = static_cast<const __nv_bfloat16 *>(X);
+    p.ldx = ldx;
+    p.Y = static_cast<__nv_bfloat16 *>(Y);
+    p.ldy = ldy;
+    return launch(pool, segs, mlora::MODE_APPLY, p, stream);
+}
+
+mlora_status mlora_shrink(mlora_pool *pool, const mlora_segments *segs, const void *X,
+                          int64_t ldx, float *H, int64_t ldh, void *stream)
+{
+    mlora_status st = check_segments(pool, segs);
+    if (st != MLORA_OK) return st;
+    if (segs->n_segments == 0 || segs->n_tokens == 0) return MLORA_OK;
+    if (X == nullptr || H == nullptr || !aligned16(X) || !aligned16(H)) return MLORA_ERR_INVALID_ARG;
+    if (ldx < pool->d_in || ldx % 8 != 0 || ldh < pool->r_max || ldh % 4 != 0)
+        return MLORA_ERR_INVALID_ARG;
+    DeviceGuard guard(pool->device);
+    if (!guard.ok) return MLORA_ERR_CUDA;
+    mlora::TileParams p = base_params(pool, segs);
+    p.X = static_cast<const __nv_bfloat16 *>(X);
+    p.ldx = ldx;
+    p.H = H;
+    p.ldh = ldh;
+    return launch(pool, segs, mlora::MODE_SHRINK, p, stream);
+}
+
+mlora_status mlora_expand(mlora_pool *pool, const mlora_segments *segs, const float *H,
+                          int64_t ldh, void *Y, int64_t ldy, void *stream)
+{
+    mlora_status st = check_segments(pool, segs);
+    if (st != MLORA_OK) return st;
+    if (segs->n_segments == 0 || segs->n_tokens == 0) return MLORA_OK;
+    if (H == nullptr || Y == nullptr || !aligned16(H) || !aligned16(Y)) return MLORA_ERR_INVALID_ARG;
+    if (ldh < pool->r_max || ldh % 4 != 0 || ldy < pool->d_out || ldy % 8 != 0)
+        return MLORA_ERR_INVALID_ARG;
+    DeviceGuard guard(pool->device);
+    if (!guard.ok) return MLORA_ERR_CUDA;
+    mlora::TileParams p = base_params(pool, segs);
+    p.H = const_cast<float *>(H);
+    p.ldh = ldh;
+    p.Y = static_cast<__nv_bfloat16 *>(Y);
+    p.ldy = ldy;
+    return launch(pool, segs, mlora::MODE_EXPAND, p, stream);
+}
+
+mlora_status mlora_build_segments(const int32_t *row_slots, int32_t n_rows, int32_t *offsets,
+                                  int32_t *slots, int32_t *token_indices, int32_t *n_segments,
+                                  int32_t *max_segment_rows, const mlora_pool *pool,
+                                  int32_t *ranks)
+{
+    if (n_rows < 0 || offsets == nullptr || n_segments == nullptr) return MLORA_ERR_INVALID_ARG;
+    if (n_rows > 0 && (row_slots == nullptr || slots == nullptr || token_indices == nullptr))
+        return MLORA_ERR_INVALID_ARG;
+    // Pass 1: segment id of each row in order of first appearance, and counts.
+    std::unordered_map<int32_t, int32_t> seg_of;
+    seg_of.reserve((size_t)std::min<int32_t>(n_rows, 1 << 16) + 1);
+    std::vector<int32_t> counts;
+    std::vector<int32_t> row_seg((size_t)n_rows);
+    for (int32_t t = 0; t < n_rows; ++t) {
+        auto it = seg_of.find(row_slots[t]);
+        int32_t g;
+        if (it == seg_of.end()) {
+            g = (int32_t)counts.size();
+            seg_of.emplace(row_slots[t], g);
+            slots[g] = row_slots[t];
+            counts.push_back(0);
+        } else {
+            g = it->second;
+        }
+        row_seg[t] = g;
+        ++counts[g];
+    }
+    const int32_t S = (int32_t)counts.size();
+    // Pass 2: offsets; pass 3: stable scatter of rows to grouped positions.
+    offsets[0] = 0;
+    int32_t longest = 0;
+    for (int32_t g = 0; g < S; ++g) {
+        offsets[g + 1] = offsets[g] + counts[g];
+        if (slots[g] >= 0) longest = std::max(longest, counts[g]);
+    }
+    std::vector<int32_t> cursor(offsets, offsets + S);
+    for (int32_t t = 0; t < n_rows; ++t) token_indices[cursor[row_seg[t]]++] = t;
+    *n_segments = S;
+    if (max_segment_rows) *max_segment_rows = longest;
+    if (pool != nullptr && ranks != nullptr) {
+        for (int32_t g = 0; g < S; ++g) {
+            const int32_t a = slots[g];
+            ranks[g] = (a >= 0 && a < pool->n_slots) ? pool->h_rank[a] : 0;
+        }
+    }
+    return MLORA_OK;
+}
+
+}  // extern "C"

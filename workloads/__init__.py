@@ -232,7 +232,7 @@ def make_small(config: int) -> Workload:
 
 def random_case(seed: int, n_rows: int, d_in: int, d_out: int, n_slots: int,
                 ranks, base_frac: float = 0.1, alpha: Optional[float] = None,
-                shuffle: bool = True) -> Workload:
+                shuffle: bool = True, r_max: Optional[int] = None) -> Workload:
     """A small random workload for edge-case sweeps (ranks drawn from ``ranks``)."""
     rng = np.random.default_rng(seed)
     slot_rank = rng.choice(np.asarray(ranks, np.int32), size=n_slots).astype(np.int32)
@@ -241,5 +241,7 @@ def random_case(seed: int, n_rows: int, d_in: int, d_out: int, n_slots: int,
         row_slot = np.sort(row_slot).astype(np.int32)
     row_slot = _base_mask(rng, row_slot, base_frac)
     alphas = (2.0 * slot_rank if alpha is None else np.full(n_slots, alpha)).astype(np.float64)
-    return Workload(f"random{seed}", seed, n_slots, int(max(RANK_BUCKETS[-1], slot_rank.max())),
-                    slot_rank, alphas, row_slot, [("proj", d_in, d_out)], "mixed")
+    if r_max is None:
+        r_max = next(b for b in RANK_BUCKETS if b >= int(slot_rank.max()))
+    return Workload(f"random{seed}", seed, n_slots, int(r_max), slot_rank, alphas, row_slot,
+                    [("proj", d_in, d_out)], "mixed")
