@@ -9,8 +9,9 @@ namespace mlora {
 
 enum TileMode : int { MODE_APPLY = 0, MODE_SHRINK = 1, MODE_EXPAND = 2 };
 
-// Rows of one work tile of the segmented kernel (one m16 MMA tile).
-constexpr int kTileRows = 16;
+// Grouped positions in one work tile of the segmented (decode-family) kernel: the
+// top half of one m16 MMA tile.
+constexpr int kTileRows = 8;
 
 // Device status bits (same values as the MLORA_FLAG_* macros of the public header).
 constexpr unsigned kFlagBadOffsets = 1u;
@@ -56,12 +57,15 @@ struct TileParams {
     // decomposition: CTA c of a cluster owns d_in columns [c*k_slice, (c+1)*k_slice)
     // for the shrink and d_out columns [c*n_slice, (c+1)*n_slice) for the expand.
     int32_t k_slice, n_slice;
+    // segments with at least this many grouped positions are left to another kernel
+    int32_t long_rows;
 };
 
-// Launch `n_clusters` clusters of `cluster` CTAs of the tile kernel for the pool's
-// largest rank bucket `rmax_bucket` (8/16/32/64) in mode `mode`.
+// Launch the tile kernel for the pool's largest rank bucket `rmax_bucket`
+// (8/16/32/64) in mode `mode`, with clusters of `cluster` CTAs: as many clusters as
+// can be resident at once, but no more than `max_tiles` (each loops over tiles).
 cudaError_t launch_tile_kernel(int mode, int rmax_bucket, const TileParams &p, int cluster,
-                               int n_clusters, cudaStream_t stream);
+                               int64_t max_tiles, cudaStream_t stream);
 
 // Set per-kernel attributes (dynamic shared memory) on the current device.
 cudaError_t prepare_tile_kernels();

@@ -1,0 +1,544 @@
+// lora_decode.cu -- segmented LoRA shrink / expand / fused apply for sm_100a,
+// the decode-shaped family: many short segments, a few rows per adapter.
+//
+// The computation (page "Multi-LoRA Serving: adapter batching", section "What
+// metadata a segmented kernel needs"): for each adapter segment g with slot a
+// and each grouped position p of it, with t = token_indices[p],
+//     H[p, :] = X[t, :] A_a^T                       (shrink, rank r)
+//     Y[t, :] = bf16(Y[t, :] + s_g H[p, :] B_a^T)   (expand + scatter)
+//
+// Work decomposition.  A work tile is (segment, up to 8 consecutive grouped
+// positions).  A thread-block cluster of C CTAs owns a tile: CTA c covers its
+// slice of d_in in the shrink (split-K) and its slice of d_out in the expand.
+// The C partial H tiles (8 x R fp32) are summed through distributed shared
+// memory, so in the fused mode H never leaves the chip.  The grid holds as many
+// clusters as can be resident at once; each loops over tiles.
+//
+// Split-K GEMV with register operands.  Decode tiles are too small for staged
+// copies to pay off, so every thread loads its mma.sync operands straight from
+// global memory with 128-bit loads:
+//   * shrink: per 32-column block of d_in, thread (g, t) of a warp loads 8
+//     consecutive bf16 of X row g and of adapter row n at columns 8t..8t+7; the
+//     two k16 mma steps of the block consume them in that order.  The sum over k
+//     does not care which columns share a step, as long as X and A agree.
+//   * expand: four n8 mma tiles cover 32 output columns; the B row a lane feeds
+//     is chosen so that thread (g, t) ends up owning columns 8t..8t+7 of row g,
+//     so Y0 is read and Y written as one 16-byte vector per thread and row.  The
+//     rank index inside each k16 step is permuted the same way for H and B.
+// The rows 8..15 of every m16 tile are zero (a tile has 8 rows).
+//
+// Rank buckets.  A kernel is compiled for the pool's largest bucket RMAX and runs
+// every tile with code specialised for its own slot's bucket R <= RMAX, so a
+// rank-8 adapter moves and multiplies rank-8 data even in a rank-64 pool.
+//
+// Precision.  fp32 accumulation throughout.  For the expand, H is split into bf16
+// hi + lo parts and both are multiplied on the tensor cores, so H enters the
+// product with about 2^-17 relative error instead of bf16's 2^-9.
+//
+// Invalid metadata never traps: bad segments and rows are skipped and flagged in
+// the status word; every CTA of a cluster reaches the same decisions, so cluster
+// barriers always match.  The kernel has no spin-waits.
+#include <climits>
+#include <mutex>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace mlora {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int TM = kTileRows;   // 8
+constexpr int kMaxCluster = 8;
+
+template <int RMAX>
+struct DecodeCfg {
+    static constexpr int WPART_FLOATS = kWarps * TM * RMAX;   // per-warp partial H
+    static constexpr int HPART_FLOATS = TM * RMAX;            // this CTA's partial H
+    static constexpr int HPITCH = RMAX + 4;
+    static constexpr int HFULL_FLOATS = TM * HPITCH;          // full H (after the cluster sum)
+    static constexpr int SMEM = 4 * (WPART_FLOATS + HPART_FLOATS + HFULL_FLOATS);
+    static constexpr int MIN_BLOCKS = RMAX <= 16 ? 4 : 2;
+};
+
+// Per-R work sizes: k32 blocks per shrink batch, 32-column groups per expand batch.
+template <int R>
+struct RankCfg {
+    static constexpr int NT = R / 8;                         // n8 tiles of the shrink
+    static constexpr int SB = R <= 8 ? 4 : R <= 16 ? 2 : 1;  // k32 blocks per batch
+    static constexpr int KS = R <= 8 ? 1 : R / 16;           // expand k steps
+    static constexpr int EB = R <= 8 ? 2 : 1;                // column groups per batch
+};
+
+struct SharedCtl {
+    int scan[kWarps];
+    int rows[TM];       // original row of each tile position, -1 = absent or invalid
+    int tile[5];        // segment, first position, end position, slot, rank from metadata
+    float seg_scale;
+    int slot_rank;
+    float slot_scale;
+};
+
+struct Tile {
+    int seg, p0, nvalid, slot, rank;
+    float scale;
+    bool ok;
+};
+
+__device__ __forceinline__ void report(const TileParams &p, unsigned flag)
+{
+    atomicOr(p.status, flag);
+}
+
+__device__ __forceinline__ uint4 ldg_nc(const void *p)
+{
+    return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+__device__ __forceinline__ uint2 ldg_nc2(const void *p)
+{
+    return __ldg(reinterpret_cast<const uint2 *>(p));
+}
+
+// Block-wide scan of per-segment tile counts.  Returns the number of tiles; if
+// tile `want` exists, its segment and first position are left in ctl.tile.
+__device__ int scan_tiles(const TileParams &p, int want, SharedCtl &ctl, bool reporter)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) ctl.tile[0] = -1;
+    __syncthreads();
+    int running = 0;
+    for (int base = 0; base < p.n_segments; base += kThreads) {
+        const int g = base + tid;
+        int cnt = 0, p0 = 0, p1 = 0, a = -1, rk = -1;
+        float sc = 0.f;
+        if (g < p.n_segments) {
+            a = p.slots[g];
+            p0 = p.offsets[g];
+            p1 = p.offsets[g + 1];
+            if (p.ranks) rk = p.ranks[g];
+            if (p.scales) sc = p.scales[g];
+            if (a != -1) {
+                if (a < -1 || a >= p.n_slots) {
+                    if (reporter) report(p, kFlagBadSlot);
+                } else if (p0 < 0 || p1 < p0 || p1 > p.n_tokens) {
+                    if (reporter) report(p, kFlagBadOffsets);
+                } else if (p1 - p0 < p.long_rows) {
+                    cnt = (p1 - p0 + TM - 1) / TM;
+                }
+            }
+        }
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) ctl.scan[warp] = incl;
+        __syncthreads();
+        int before = 0, total = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const int v = ctl.scan[w];
+            before += (w < warp) ? v : 0;
+            total += v;
+        }
+        incl += before;
+        const int lo = running + incl - cnt;
+        if (cnt > 0 && want >= lo && want < running + incl) {
+            ctl.tile[0] = g;
+            ctl.tile[1] = p0 + (want - lo) * TM;
+            ctl.tile[2] = p1;
+            ctl.tile[3] = a;
+            ctl.tile[4] = rk;
+            ctl.seg_scale = sc;
+        }
+        running += total;
+        __syncthreads();   // ctl.scan is rewritten by the next chunk
+    }
+    return running;
+}
+
+// One tile, specialised for rank bucket R.
+template <int RMAX, int MODE, int R>
+__device__ void run_tile(const TileParams &p, const Tile &tl, int row_g, SharedCtl &ctl,
+                         float *smem_f, uint32_t crank, uint32_t csize)
+{
+    using RC = RankCfg<R>;
+    using DC = DecodeCfg<RMAX>;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    float *wpart = smem_f;
+    float *hpart = wpart + DC::WPART_FLOATS;
+    float *hfull = hpart + DC::HPART_FLOATS;
+    const __nv_bfloat16 *slotA = p.pool + (int64_t)tl.slot * p.slot_stride;
+    const __nv_bfloat16 *slotB = slotA + p.b_offset;
+    const bool row_ok = row_g >= 0;   // row g of the tile is present
+
+    // ---------------- shrink: this CTA's d_in slice, 32 columns per block
+    if constexpr (MODE != MODE_EXPAND) {
+        const int k_begin = min(p.d_in, (int)crank * p.k_slice);
+        const int k_end = min(p.d_in, k_begin + p.k_slice);
+        const int nblk = (k_end - k_begin + 31) / 32;
+        const __nv_bfloat16 *xrow = p.X + (int64_t)(row_ok ? row_g : 0) * p.ldx;
+        float acc[RC::NT][4];
+#pragma unroll
+        for (int n = 0; n < RC::NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+        for (int b0 = warp; b0 < nblk; b0 += kWarps * RC::SB) {
+            uint4 xv[RC::SB], av[RC::SB][RC::NT];
+#pragma unroll
+            for (int s = 0; s < RC::SB; ++s) {
+                const int b = b0 + s * kWarps;
+                const int k = k_begin + b * 32 + 8 * t;   // this thread's 8 columns
+                const bool kin = b < nblk && k < k_end;
+                xv[s] = (kin && row_ok) ? ldg_nc(xrow + k) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int n = 0; n < RC::NT; ++n)
+                    av[s][n] = kin ? ldg_nc(slotA + ((int64_t)(k / 8) * R + n * 8 + g) * 8)
+                                   : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int s = 0; s < RC::SB; ++s)
+#pragma unroll
+                for (int n = 0; n < RC::NT; ++n) {
+                    mma_16816(acc[n], xv[s].x, 0u, xv[s].y, 0u, av[s][n].x, av[s][n].y);
+                    mma_16816(acc[n], xv[s].z, 0u, xv[s].w, 0u, av[s][n].z, av[s][n].w);
+                }
+        }
+        // per-warp partials -> CTA partial (fixed order over warps)
+#pragma unroll
+        for (int n = 0; n < RC::NT; ++n) {
+            wpart[(warp * TM + g) * R + n * 8 + 2 * t] = acc[n][0];
+            wpart[(warp * TM + g) * R + n * 8 + 2 * t + 1] = acc[n][1];
+        }
+        __syncthreads();
+        for (int e = tid; e < TM * R; e += kThreads) {
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) sum += wpart[w * TM * R + e];
+            hpart[e] = sum;
+        }
+        // the cluster's partials, summed in CTA order through distributed shared memory
+        cluster_arrive_release();
+        cluster_wait_acquire();
+        const uint32_t hpart_s = smem_addr(hpart);
+        for (int e = tid; e < TM * R; e += kThreads) {
+            const int i = e / R, j = e % R;
+            if (MODE == MODE_SHRINK &&
+                ((uint32_t)i % csize != crank || i >= tl.nvalid || j >= tl.rank || !tl.ok ||
+                 ctl.rows[i] < 0))
+                continue;
+            float v[kMaxCluster];
+#pragma unroll
+            for (int c = 0; c < kMaxCluster; ++c)
+                v[c] = (c < (int)csize) ? ld_dsmem_f32(map_to_rank(hpart_s + 4u * e, c)) : 0.f;
+            float sum = 0.f;
+#pragma unroll
+            for (int c = 0; c < kMaxCluster; ++c) sum += v[c];
+            if constexpr (MODE == MODE_APPLY) {
+                hfull[i * DC::HPITCH + j] = sum;
+            } else {
+                p.H[(int64_t)(tl.p0 + i) * p.ldh + j] = sum;
+            }
+        }
+        cluster_arrive_relaxed();   // paired with the wait at the end of the tile
+    } else {
+        for (int e = tid; e < TM * R; e += kThreads) {
+            const int i = e / R, j = e % R;
+            float v = 0.f;
+            if (i < tl.nvalid && j < tl.rank) v = p.H[(int64_t)(tl.p0 + i) * p.ldh + j];
+            hfull[i * DC::HPITCH + j] = v;
+        }
+    }
+
+    // ---------------- expand: this CTA's d_out slice, 32 columns per group
+    if constexpr (MODE != MODE_SHRINK) {
+        __syncthreads();
+        // H row g as bf16 hi + lo fragments; step s covers rank 16s + 4t .. 16s + 4t + 3
+        // (rank 8: 2t, 2t + 1)
+        uint32_t ah[RC::KS][2], al[RC::KS][2];
+#pragma unroll
+        for (int s = 0; s < RC::KS; ++s) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int col = (R == 8) ? 2 * t : 16 * s + 4 * t + 2 * q;
+                const float x0 = hfull[g * DC::HPITCH + col];
+                const float x1 = hfull[g * DC::HPITCH + col + 1];
+                float h0, l0, h1, l1;
+                split_bf16(x0, h0, l0);
+                split_bf16(x1, h1, l1);
+                ah[s][q] = pack_bf16x2(h0, h1);
+                al[s][q] = pack_bf16x2(l0, l1);
+            }
+        }
+        const int n_begin = min(p.d_out, (int)crank * p.n_slice);
+        const int n_end = min(p.d_out, n_begin + p.n_slice);
+        const int ngrp = (n_end - n_begin + 31) / 32;
+        const bool store = tl.ok && row_ok;
+        __nv_bfloat16 *yrow = p.Y + (int64_t)(row_ok ? row_g : 0) * p.ldy;
+        // B row fed by lane (g, t) in n8 tile i of a group: 8 (g / 2) + 2 i + (g % 2)
+        const int brow = 8 * (g >> 1) + (g & 1);
+        for (int q0 = warp; q0 < ngrp; q0 += kWarps * RC::EB) {
+            uint2 bv[RC::EB][4][RC::KS];
+            uint4 yv[RC::EB];
+#pragma unroll
+            for (int e = 0; e < RC::EB; ++e) {
+                const int base = n_begin + (q0 + e * kWarps) * 32;
+                const bool gin = q0 + e * kWarps < ngrp;
+                const int bcol = base + brow;                  // + 2 i
+                const bool bin = gin && base + 8 * (g >> 1) < n_end;
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int s = 0; s < RC::KS; ++s) {
+                        if constexpr (R == 8) {
+                            const uint32_t v = bin ? __ldg(reinterpret_cast<const uint32_t *>(
+                                                         slotB + (int64_t)(bcol + 2 * i) * 8 + 2 * t))
+                                                   : 0u;
+                            bv[e][i][s] = make_uint2(v, 0u);
+                        } else {
+                            bv[e][i][s] = bin ? ldg_nc2(slotB + ((int64_t)(2 * s + (t >> 1)) * p.d_out +
+                                                                  bcol + 2 * i) * 8 + (t & 1) * 4)
+                                              : make_uint2(0u, 0u);
+                        }
+                    }
+                const bool cin = gin && base + 8 * t < n_end;
+                yv[e] = (cin && row_ok) ? *reinterpret_cast<const uint4 *>(yrow + base + 8 * t)
+                                        : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int e = 0; e < RC::EB; ++e) {
+                const int base = n_begin + (q0 + e * kWarps) * 32;
+                const bool cin = (q0 + e * kWarps < ngrp) && base + 8 * t < n_end;
+                float d[4][4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    d[i][0] = d[i][1] = d[i][2] = d[i][3] = 0.f;
+#pragma unroll
+                    for (int s = 0; s < RC::KS; ++s) {
+                        if constexpr (R == 8) {
+                            mma_1688(d[i], ah[0][0], 0u, bv[e][i][0].x);
+                            mma_1688(d[i], al[0][0], 0u, bv[e][i][0].x);
+                        } else {
+                            mma_16816(d[i], ah[s][0], 0u, ah[s][1], 0u, bv[e][i][s].x, bv[e][i][s].y);
+                            mma_16816(d[i], al[s][0], 0u, al[s][1], 0u, bv[e][i][s].x, bv[e][i][s].y);
+                        }
+                    }
+                }
+                // thread (g, t) holds row g, columns base + 8t + 2i + {0, 1}
+                const __nv_bfloat162 *y0 = reinterpret_cast<const __nv_bfloat162 *>(&yv[e]);
+                uint4 out;
+                uint32_t *o = reinterpret_cast<uint32_t *>(&out);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __bfloat1622float2(y0[i]);
+                    o[i] = pack_bf16x2(fmaf(tl.scale, d[i][0], f.x), fmaf(tl.scale, d[i][1], f.y));
+                }
+                if (store && cin) *reinterpret_cast<uint4 *>(yrow + base + 8 * t) = out;
+            }
+        }
+    }
+    if constexpr (MODE != MODE_EXPAND) cluster_wait_acquire();
+}
+
+template <int RMAX, int MODE>
+__global__ void __launch_bounds__(kThreads, DecodeCfg<RMAX>::MIN_BLOCKS)
+    lora_decode_kernel(const __grid_constant__ TileParams p)
+{
+    extern __shared__ __align__(16) float smem_f[];
+    __shared__ SharedCtl ctl;
+    const int tid = threadIdx.x;
+    const uint32_t crank = cluster_rank();
+    const uint32_t csize = cluster_size();
+    const int n_clusters = (int)(gridDim.x / csize);
+    const bool reporter = blockIdx.x == 0;
+    const int g = (tid & 31) >> 2;
+
+    int tile = (int)cluster_index();
+    int total = scan_tiles(p, tile, ctl, reporter);
+    for (; tile < total; tile += n_clusters) {
+        if (tile != (int)cluster_index()) scan_tiles(p, tile, ctl, false);
+        // every CTA of the cluster reads the same metadata and reaches the same tile
+        Tile tl;
+        tl.seg = ctl.tile[0];
+        tl.p0 = ctl.tile[1];
+        tl.nvalid = min(TM, ctl.tile[2] - tl.p0);
+        tl.slot = ctl.tile[3];
+        const int r_meta = ctl.tile[4];
+        // rows of this tile (each lane needs row g), slot rank and scale
+        int row_g = -1;
+        if (g < tl.nvalid) {
+            row_g = p.token_indices ? p.token_indices[tl.p0 + g] : tl.p0 + g;
+            if (row_g < 0 || row_g >= p.n_rows) {
+                if (crank == 0 && (tid & 3) == 0 && tid < 32) report(p, kFlagBadRow);
+                row_g = -1;
+            }
+        }
+        if (tid < 32 && (tid & 3) == 0) ctl.rows[g] = row_g;
+        if (tid == 0) {
+            ctl.slot_rank = p.slot_rank[tl.slot];
+            ctl.slot_scale = p.slot_scale[tl.slot];
+        }
+        __syncthreads();
+        const int r = ctl.slot_rank;
+        tl.ok = r > 0 && (p.ranks == nullptr || r_meta == r) && rank_bucket(r) <= RMAX;
+        if (tid == 0 && crank == 0 && !tl.ok) report(p, r <= 0 ? kFlagSlotEmpty : kFlagBadRank);
+        tl.rank = tl.ok ? r : 0;   // a rejected tile reads and writes no H
+        tl.scale = p.scales ? ctl.seg_scale : ctl.slot_scale;
+        const int R = tl.ok ? rank_bucket(r) : 8;
+        if (R == 8) {
+            run_tile<RMAX, MODE, 8>(p, tl, row_g, ctl, smem_f, crank, csize);
+        } else if (R == 16) {
+            if constexpr (RMAX >= 16) run_tile<RMAX, MODE, 16>(p, tl, row_g, ctl, smem_f, crank, csize);
+        } else if (R == 32) {
+            if constexpr (RMAX >= 32) run_tile<RMAX, MODE, 32>(p, tl, row_g, ctl, smem_f, crank, csize);
+        } else {
+            if constexpr (RMAX >= 64) run_tile<RMAX, MODE, 64>(p, tl, row_g, ctl, smem_f, crank, csize);
+        }
+        __syncthreads();   // ctl and the H buffers are rewritten by the next tile
+    }
+}
+
+template <int RMAX, int MODE>
+cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, cudaStream_t stream)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = DecodeCfg<RMAX>::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+
+    // clusters resident at once for this kernel and cluster size (cached per device)
+    static std::mutex mu;
+    static int cached[64][kMaxCluster + 1] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    int active;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        active = cached[dev][cluster];
+        if (active == 0) {
+            cfg.gridDim = dim3((unsigned)cluster, 1, 1);
+            cudaError_t e =
+                cudaOccupancyMaxActiveClusters(&active, lora_decode_kernel<RMAX, MODE>, &cfg);
+            if (e != cudaSuccess) return e;
+            if (active <= 0) return cudaErrorInvalidConfiguration;
+            cached[dev][cluster] = active;
+        }
+    }
+    const int64_t n = max_tiles < active ? max_tiles : active;
+    cfg.gridDim = dim3((unsigned)(n * cluster), 1, 1);
+    return cudaLaunchKernelEx(&cfg, lora_decode_kernel<RMAX, MODE>, p);
+}
+
+template <int RMAX>
+cudaError_t launch_rmax(int mode, const TileParams &p, int cluster, int64_t max_tiles,
+                        cudaStream_t stream)
+{
+    switch (mode) {
+    case MODE_APPLY: return launch_one<RMAX, MODE_APPLY>(p, cluster, max_tiles, stream);
+    case MODE_SHRINK: return launch_one<RMAX, MODE_SHRINK>(p, cluster, max_tiles, stream);
+    case MODE_EXPAND: return launch_one<RMAX, MODE_EXPAND>(p, cluster, max_tiles, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int RMAX>
+cudaError_t set_attrs()
+{
+    cudaError_t e;
+    e = cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_APPLY>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX>::SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_SHRINK>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX>::SMEM);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_EXPAND>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX>::SMEM);
+}
+
+// Repack: A [rank, d_in] -> [d_in/8][R][8]; B [d_out, rank] -> [R/8][d_out][8]; zero
+// beyond rank.  One thread per 16-byte destination group, written in order.
+__global__ void repack_slot_kernel(__nv_bfloat16 *slot, int64_t b_offset, int R, int rank,
+                                   int d_in, int d_out, const __nv_bfloat16 *A,
+                                   const __nv_bfloat16 *B, int32_t *rank_entry,
+                                   float *scale_entry, float scale)
+{
+    const int na = R * (d_in / 8);    // 16-byte groups of the A block
+    const int nb = (R / 8) * d_out;   // 16-byte groups of the B block
+    const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < na + nb; e += gridDim.x * blockDim.x) {
+        __align__(16) __nv_bfloat16 v[8];
+        __nv_bfloat16 *dst;
+        if (e < na) {
+            const int kg = e / R, j = e - kg * R;          // group [kg][j][0..7]
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                v[c] = j < rank ? A[(int64_t)j * d_in + kg * 8 + c] : zero;
+            dst = slot + (int64_t)e * 8;
+        } else {
+            const int f = e - na;
+            const int jg = f / d_out, o = f - jg * d_out;   // group [jg][o][0..7]
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const int j = jg * 8 + c;
+                v[c] = j < rank ? B[(int64_t)o * rank + j] : zero;
+            }
+            dst = slot + b_offset + (int64_t)f * 8;
+        }
+        *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(v);
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *rank_entry = rank;
+        *scale_entry = scale;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_tile_kernel(int mode, int rmax_bucket, const TileParams &p, int cluster,
+                               int64_t max_tiles, cudaStream_t stream)
+{
+    if (cluster < 1 || cluster > kMaxCluster || max_tiles < 1) return cudaErrorInvalidValue;
+    switch (rmax_bucket) {
+    case 8: return launch_rmax<8>(mode, p, cluster, max_tiles, stream);
+    case 16: return launch_rmax<16>(mode, p, cluster, max_tiles, stream);
+    case 32: return launch_rmax<32>(mode, p, cluster, max_tiles, stream);
+    case 64: return launch_rmax<64>(mode, p, cluster, max_tiles, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t prepare_tile_kernels()
+{
+    cudaError_t e;
+    if ((e = set_attrs<8>()) != cudaSuccess) return e;
+    if ((e = set_attrs<16>()) != cudaSuccess) return e;
+    if ((e = set_attrs<32>()) != cudaSuccess) return e;
+    return set_attrs<64>();
+}
+
+cudaError_t launch_repack_slot(__nv_bfloat16 *slot_base, int64_t b_offset, int R, int rank,
+                               int d_in, int d_out, const __nv_bfloat16 *A_src,
+                               const __nv_bfloat16 *B_src, int32_t *slot_rank_entry,
+                               float *slot_scale_entry, float scale, cudaStream_t stream)
+{
+    const int64_t groups = (int64_t)R * (d_in / 8) + (int64_t)(R / 8) * d_out;
+    const int threads = 256;
+    const int64_t blocks64 = (groups + threads - 1) / threads;
+    const int blocks = (int)(blocks64 < 2048 ? blocks64 : 2048);
+    repack_slot_kernel<<<blocks, threads, 0, stream>>>(slot_base, b_offset, R, rank, d_in, d_out,
+                                                       A_src, B_src, slot_rank_entry,
+                                                       slot_scale_entry, scale);
+    return cudaGetLastError();
+}
+
+}  // namespace mlora

@@ -76,11 +76,11 @@ int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
 // Cluster size: enough CTAs per tile to spread one adapter's A and B over ~1K
 // columns each, at most 8 (the portable cluster size), and every CTA must own at
-// least one 16-column group of d_in and one 8-column group of d_out.
+// least one 32-column block of d_in and one 8-column group of d_out.
 int choose_cluster(int d_in, int d_out)
 {
     int c = (int)std::min<int64_t>(8, std::max<int64_t>(1, (int64_t)(d_in + d_out + 1023) / 1024));
-    while (c > 1 && (round_up((d_in + c - 1) / c, 16) * (c - 1) >= d_in ||
+    while (c > 1 && (round_up((d_in + c - 1) / c, 32) * (c - 1) >= d_in ||
                      round_up((d_out + c - 1) / c, 8) * (c - 1) >= d_out))
         --c;
     return c;
@@ -122,14 +122,14 @@ mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::
                     void *stream)
 {
     const int c = choose_cluster(pool->d_in, pool->d_out);
-    p.k_slice = (int32_t)round_up((pool->d_in + c - 1) / c, 16);
+    p.k_slice = (int32_t)round_up((pool->d_in + c - 1) / c, 32);
     p.n_slice = (int32_t)round_up((pool->d_out + c - 1) / c, 8);
-    // Upper bound on the number of 16-row tiles of well-formed metadata.
+    p.long_rows = 0x7fffffff;
+    // Upper bound on the number of work tiles of well-formed metadata.
     const int64_t tiles = (int64_t)s->n_segments + (int64_t)s->n_tokens / mlora::kTileRows + 1;
-    if (tiles * c > 0x7fffffff) return MLORA_ERR_UNSUPPORTED;
     mlora_status st = prepare_device(pool->device);
     if (st != MLORA_OK) return st;
-    cudaError_t e = mlora::launch_tile_kernel(mode, pool->r_bucket_max, p, c, (int)tiles,
+    cudaError_t e = mlora::launch_tile_kernel(mode, pool->r_bucket_max, p, c, tiles,
                                               static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MLORA_OK : MLORA_ERR_CUDA;
 }
