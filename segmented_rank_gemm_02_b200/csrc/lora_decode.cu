@@ -63,13 +63,25 @@ struct DecodeCfg {
     static constexpr int MIN_BLOCKS = RMAX <= 16 ? 4 : 2;
 };
 
-// Per-R work sizes: k32 blocks per shrink batch, 32-column groups per expand batch.
+// Per-R register operands: one k32 block of the shrink, one 32-column group of the
+// expand.  Every warp keeps two of each in flight.
 template <int R>
 struct RankCfg {
-    static constexpr int NT = R / 8;                         // n8 tiles of the shrink
-    static constexpr int SB = R <= 8 ? 4 : R <= 16 ? 2 : 1;  // k32 blocks per batch
-    static constexpr int KS = R <= 8 ? 1 : R / 16;           // expand k steps
-    static constexpr int EB = R <= 8 ? 2 : 1;                // column groups per batch
+    static constexpr int NT = R / 8;                  // n8 tiles of the shrink
+    static constexpr int KS = R <= 8 ? 1 : R / 16;    // k steps of the expand
+    static constexpr bool EARLY_EXPAND = R <= 32;     // first expand group loaded up front
+};
+
+template <int R>
+struct ShrinkOps {
+    uint4 x;                    // X row g, columns 8t..8t+7 of the block
+    uint4 a[RankCfg<R>::NT];    // adapter rows n*8+g, same columns
+};
+
+template <int R>
+struct ExpandOps {
+    uint2 b[4][RankCfg<R>::KS];  // B rows of the four n8 tiles, this lane's ranks
+    uint4 y;                     // Y0 row g, columns 8t..8t+7 of the group
 };
 
 struct SharedCtl {
@@ -82,9 +94,7 @@ struct SharedCtl {
 };
 
 struct Tile {
-    int seg, p0, nvalid, slot, rank;
-    float scale;
-    bool ok;
+    int seg, p0, nvalid, slot;
 };
 
 __device__ __forceinline__ void report(const TileParams &p, unsigned flag)
@@ -161,10 +171,117 @@ __device__ int scan_tiles(const TileParams &p, int want, SharedCtl &ctl, bool re
     return running;
 }
 
-// One tile, specialised for rank bucket R.
+// Geometry of this CTA's part of a tile.
+struct Slices {
+    int k_begin, k_end, nblk;   // d_in slice, 32-column blocks
+    int n_begin, n_end, ngrp;   // d_out slice, 32-column groups
+};
+
+template <int R>
+__device__ __forceinline__ void load_a(ShrinkOps<R> &o, const __nv_bfloat16 *slotA, const Slices &sl,
+                                       int blk, int g, int t)
+{
+    const int k = sl.k_begin + blk * 32 + 8 * t;   // this thread's 8 columns
+    const bool kin = blk < sl.nblk && k < sl.k_end;
+#pragma unroll
+    for (int n = 0; n < RankCfg<R>::NT; ++n)
+        o.a[n] = kin ? ldg_nc(slotA + ((int64_t)(k / 8) * R + n * 8 + g) * 8) : make_uint4(0, 0, 0, 0);
+}
+
+template <int R>
+__device__ __forceinline__ void load_x(ShrinkOps<R> &o, const __nv_bfloat16 *xrow, bool row_ok,
+                                       const Slices &sl, int blk, int t)
+{
+    const int k = sl.k_begin + blk * 32 + 8 * t;
+    o.x = (row_ok && blk < sl.nblk && k < sl.k_end) ? ldg_nc(xrow + k) : make_uint4(0, 0, 0, 0);
+}
+
+template <int R>
+__device__ __forceinline__ void mma_shrink(float (&acc)[RankCfg<R>::NT][4], const ShrinkOps<R> &o)
+{
+#pragma unroll
+    for (int n = 0; n < RankCfg<R>::NT; ++n) {
+        mma_16816(acc[n], o.x.x, 0u, o.x.y, 0u, o.a[n].x, o.a[n].y);
+        mma_16816(acc[n], o.x.z, 0u, o.x.w, 0u, o.a[n].z, o.a[n].w);
+    }
+}
+
+// B row fed by lane (g, t) in n8 tile i of a group: base + 8 (g / 2) + (g % 2) + 2 i, so
+// that thread (g, t) accumulates columns base + 8t .. base + 8t + 7 of row g.
+template <int R>
+__device__ __forceinline__ void load_b(ExpandOps<R> &o, const __nv_bfloat16 *slotB, int d_out,
+                                       const Slices &sl, int grp, int g, int t)
+{
+    const int base = sl.n_begin + grp * 32;
+    const bool bin = grp < sl.ngrp && base + 8 * (g >> 1) < sl.n_end;
+    const int brow = base + 8 * (g >> 1) + (g & 1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int s = 0; s < RankCfg<R>::KS; ++s) {
+            if constexpr (R == 8) {
+                const uint32_t v =
+                    bin ? __ldg(reinterpret_cast<const uint32_t *>(slotB + (int64_t)(brow + 2 * i) * 8 + 2 * t))
+                        : 0u;
+                o.b[i][s] = make_uint2(v, 0u);
+            } else {
+                o.b[i][s] = bin ? ldg_nc2(slotB + ((int64_t)(2 * s + (t >> 1)) * d_out + brow + 2 * i) * 8 +
+                                          (t & 1) * 4)
+                                : make_uint2(0u, 0u);
+            }
+        }
+}
+
+template <int R>
+__device__ __forceinline__ void load_y(ExpandOps<R> &o, const __nv_bfloat16 *yrow, bool row_ok,
+                                       const Slices &sl, int grp, int t)
+{
+    const int c = sl.n_begin + grp * 32 + 8 * t;
+    o.y = (row_ok && grp < sl.ngrp && c < sl.n_end) ? *reinterpret_cast<const uint4 *>(yrow + c)
+                                                     : make_uint4(0, 0, 0, 0);
+}
+
+// y = bf16(y0 + s (H B^T)) for one group; thread (g, t) stores row g, columns 8t..8t+7.
+template <int R>
+__device__ __forceinline__ void mma_expand_store(const ExpandOps<R> &o, const uint32_t (&ah)[RankCfg<R>::KS][2],
+                                                 const uint32_t (&al)[RankCfg<R>::KS][2], float scale,
+                                                 __nv_bfloat16 *yrow, bool store, const Slices &sl,
+                                                 int grp, int t)
+{
+    float d[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        d[i][0] = d[i][1] = d[i][2] = d[i][3] = 0.f;
+#pragma unroll
+        for (int s = 0; s < RankCfg<R>::KS; ++s) {
+            if constexpr (R == 8) {
+                mma_1688(d[i], ah[0][0], 0u, o.b[i][0].x);
+                mma_1688(d[i], al[0][0], 0u, o.b[i][0].x);
+            } else {
+                mma_16816(d[i], ah[s][0], 0u, ah[s][1], 0u, o.b[i][s].x, o.b[i][s].y);
+                mma_16816(d[i], al[s][0], 0u, al[s][1], 0u, o.b[i][s].x, o.b[i][s].y);
+            }
+        }
+    }
+    const int c = sl.n_begin + grp * 32 + 8 * t;
+    if (!store || grp >= sl.ngrp || c >= sl.n_end) return;
+    const __nv_bfloat162 *y0 = reinterpret_cast<const __nv_bfloat162 *>(&o.y);
+    uint4 out;
+    uint32_t *w = reinterpret_cast<uint32_t *>(&out);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(y0[i]);
+        w[i] = pack_bf16x2(fmaf(scale, d[i][0], f.x), fmaf(scale, d[i][1], f.y));
+    }
+    *reinterpret_cast<uint4 *>(yrow + c) = out;
+}
+
+// One tile, specialised for rank bucket R.  Loads are issued as early as their
+// addresses are known: adapter blocks right away, rows once their indices land,
+// the expand's operands before the cluster reduction.
 template <int RMAX, int MODE, int R>
-__device__ void run_tile(const TileParams &p, const Tile &tl, int row_g, SharedCtl &ctl,
-                         float *smem_f, uint32_t crank, uint32_t csize)
+__device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float seg_scale,
+                         SharedCtl &ctl, float *smem_f, uint32_t crank, uint32_t csize)
 {
     using RC = RankCfg<R>;
     using DC = DecodeCfg<RMAX>;
@@ -175,45 +292,105 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int row_g, SharedC
     float *hfull = hpart + DC::HPART_FLOATS;
     const __nv_bfloat16 *slotA = p.pool + (int64_t)tl.slot * p.slot_stride;
     const __nv_bfloat16 *slotB = slotA + p.b_offset;
-    const bool row_ok = row_g >= 0;   // row g of the tile is present
 
-    // ---------------- shrink: this CTA's d_in slice, 32 columns per block
+    Slices sl;
+    sl.k_begin = min(p.d_in, (int)crank * p.k_slice);
+    sl.k_end = min(p.d_in, sl.k_begin + p.k_slice);
+    sl.nblk = (MODE == MODE_EXPAND) ? 0 : (sl.k_end - sl.k_begin + 31) / 32;
+    sl.n_begin = min(p.d_out, (int)crank * p.n_slice);
+    sl.n_end = min(p.d_out, sl.n_begin + p.n_slice);
+    sl.ngrp = (MODE == MODE_SHRINK) ? 0 : (sl.n_end - sl.n_begin + 31) / 32;
+    // blocks w, w + 8, ... and groups w, w + 8, ... of this warp, as local indices 0, 1, ...
+    const int nb = sl.nblk > warp ? (sl.nblk - warp + kWarps - 1) / kWarps : 0;
+    const int ng = sl.ngrp > warp ? (sl.ngrp - warp + kWarps - 1) / kWarps : 0;
+
+    // ---- requests that need only the segment's slot
+    int row_g = -1;
+    if (g < tl.nvalid) row_g = p.token_indices ? __ldg(p.token_indices + tl.p0 + g) : tl.p0 + g;
+    int srank = 0;
+    float sscale = 0.f;
+    if (tid == 0) {
+        srank = p.slot_rank[tl.slot];
+        sscale = p.slot_scale[tl.slot];
+    }
+    ShrinkOps<R> s0, s1;
+    ExpandOps<R> e0, e1;
     if constexpr (MODE != MODE_EXPAND) {
-        const int k_begin = min(p.d_in, (int)crank * p.k_slice);
-        const int k_end = min(p.d_in, k_begin + p.k_slice);
-        const int nblk = (k_end - k_begin + 31) / 32;
-        const __nv_bfloat16 *xrow = p.X + (int64_t)(row_ok ? row_g : 0) * p.ldx;
+        load_a<R>(s0, slotA, sl, warp, g, t);
+        load_a<R>(s1, slotA, sl, warp + kWarps, g, t);
+    }
+    if constexpr (MODE != MODE_SHRINK && RC::EARLY_EXPAND) load_b<R>(e0, slotB, p.d_out, sl, warp, g, t);
+
+    // ---- requests that need the row
+    if (g < tl.nvalid && (row_g < 0 || row_g >= p.n_rows)) {
+        if (crank == 0 && warp == 0 && t == 0) report(p, kFlagBadRow);
+        row_g = -1;
+    }
+    const bool row_ok = row_g >= 0;
+    const __nv_bfloat16 *xrow = p.X + (int64_t)(row_ok ? row_g : 0) * p.ldx;
+    __nv_bfloat16 *yrow = p.Y + (int64_t)(row_ok ? row_g : 0) * p.ldy;
+    if constexpr (MODE != MODE_EXPAND) {
+        load_x<R>(s0, xrow, row_ok, sl, warp, t);
+        load_x<R>(s1, xrow, row_ok, sl, warp + kWarps, t);
+    }
+    if constexpr (MODE != MODE_SHRINK && RC::EARLY_EXPAND) load_y<R>(e0, yrow, row_ok, sl, warp, t);
+
+    // ---- shrink: this CTA's d_in slice, two blocks in flight per warp
+    if constexpr (MODE != MODE_EXPAND) {
         float acc[RC::NT][4];
 #pragma unroll
         for (int n = 0; n < RC::NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-        for (int b0 = warp; b0 < nblk; b0 += kWarps * RC::SB) {
-            uint4 xv[RC::SB], av[RC::SB][RC::NT];
-#pragma unroll
-            for (int s = 0; s < RC::SB; ++s) {
-                const int b = b0 + s * kWarps;
-                const int k = k_begin + b * 32 + 8 * t;   // this thread's 8 columns
-                const bool kin = b < nblk && k < k_end;
-                xv[s] = (kin && row_ok) ? ldg_nc(xrow + k) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-                for (int n = 0; n < RC::NT; ++n)
-                    av[s][n] = kin ? ldg_nc(slotA + ((int64_t)(k / 8) * R + n * 8 + g) * 8)
-                                   : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < nb; i += 2) {
+            mma_shrink<R>(acc, s0);
+            if (i + 2 < nb) {
+                const int b = warp + (i + 2) * kWarps;
+                load_a<R>(s0, slotA, sl, b, g, t);
+                load_x<R>(s0, xrow, row_ok, sl, b, t);
             }
-#pragma unroll
-            for (int s = 0; s < RC::SB; ++s)
-#pragma unroll
-                for (int n = 0; n < RC::NT; ++n) {
-                    mma_16816(acc[n], xv[s].x, 0u, xv[s].y, 0u, av[s][n].x, av[s][n].y);
-                    mma_16816(acc[n], xv[s].z, 0u, xv[s].w, 0u, av[s][n].z, av[s][n].w);
+            if (i + 1 < nb) {
+                mma_shrink<R>(acc, s1);
+                if (i + 3 < nb) {
+                    const int b = warp + (i + 3) * kWarps;
+                    load_a<R>(s1, slotA, sl, b, g, t);
+                    load_x<R>(s1, xrow, row_ok, sl, b, t);
                 }
+            }
         }
-        // per-warp partials -> CTA partial (fixed order over warps)
+        if constexpr (MODE != MODE_SHRINK) {
+            // the expand's first groups travel while the cluster sums H
+            if constexpr (!RC::EARLY_EXPAND) {
+                load_b<R>(e0, slotB, p.d_out, sl, warp, g, t);
+                load_y<R>(e0, yrow, row_ok, sl, warp, t);
+            }
+            load_b<R>(e1, slotB, p.d_out, sl, warp + kWarps, g, t);
+            load_y<R>(e1, yrow, row_ok, sl, warp + kWarps, t);
+        }
 #pragma unroll
         for (int n = 0; n < RC::NT; ++n) {
             wpart[(warp * TM + g) * R + n * 8 + 2 * t] = acc[n][0];
             wpart[(warp * TM + g) * R + n * 8 + 2 * t + 1] = acc[n][1];
         }
-        __syncthreads();
+    } else {
+        load_b<R>(e1, slotB, p.d_out, sl, warp + kWarps, g, t);
+        load_y<R>(e1, yrow, row_ok, sl, warp + kWarps, t);
+        if constexpr (!RC::EARLY_EXPAND) {
+            load_b<R>(e0, slotB, p.d_out, sl, warp, g, t);
+            load_y<R>(e0, yrow, row_ok, sl, warp, t);
+        }
+    }
+    if (tid == 0) {
+        ctl.slot_rank = srank;
+        ctl.slot_scale = sscale;
+    }
+    if (warp == 0 && t == 0) ctl.rows[g] = row_g;
+    __syncthreads();
+    const int r = ctl.slot_rank;
+    const bool ok = r > 0 && (p.ranks == nullptr || r_meta == r) && rank_bucket(r) == R;
+    if (tid == 0 && crank == 0 && !ok) report(p, r <= 0 ? kFlagSlotEmpty : kFlagBadRank);
+    const int rank = ok ? r : 0;   // a rejected tile reads and writes no H
+    const float scale = p.scales ? seg_scale : ctl.slot_scale;
+
+    if constexpr (MODE != MODE_EXPAND) {
         for (int e = tid; e < TM * R; e += kThreads) {
             float sum = 0.f;
 #pragma unroll
@@ -227,8 +404,7 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int row_g, SharedC
         for (int e = tid; e < TM * R; e += kThreads) {
             const int i = e / R, j = e % R;
             if (MODE == MODE_SHRINK &&
-                ((uint32_t)i % csize != crank || i >= tl.nvalid || j >= tl.rank || !tl.ok ||
-                 ctl.rows[i] < 0))
+                ((uint32_t)i % csize != crank || i >= tl.nvalid || j >= rank || ctl.rows[i] < 0))
                 continue;
             float v[kMaxCluster];
 #pragma unroll
@@ -248,95 +424,44 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int row_g, SharedC
         for (int e = tid; e < TM * R; e += kThreads) {
             const int i = e / R, j = e % R;
             float v = 0.f;
-            if (i < tl.nvalid && j < tl.rank) v = p.H[(int64_t)(tl.p0 + i) * p.ldh + j];
+            if (i < tl.nvalid && j < rank) v = p.H[(int64_t)(tl.p0 + i) * p.ldh + j];
             hfull[i * DC::HPITCH + j] = v;
         }
     }
 
-    // ---------------- expand: this CTA's d_out slice, 32 columns per group
+    // ---- expand: this CTA's d_out slice, two groups in flight per warp
     if constexpr (MODE != MODE_SHRINK) {
         __syncthreads();
         // H row g as bf16 hi + lo fragments; step s covers rank 16s + 4t .. 16s + 4t + 3
-        // (rank 8: 2t, 2t + 1)
+        // (rank bucket 8: 2t, 2t + 1)
         uint32_t ah[RC::KS][2], al[RC::KS][2];
 #pragma unroll
         for (int s = 0; s < RC::KS; ++s) {
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 const int col = (R == 8) ? 2 * t : 16 * s + 4 * t + 2 * q;
-                const float x0 = hfull[g * DC::HPITCH + col];
-                const float x1 = hfull[g * DC::HPITCH + col + 1];
                 float h0, l0, h1, l1;
-                split_bf16(x0, h0, l0);
-                split_bf16(x1, h1, l1);
+                split_bf16(hfull[g * DC::HPITCH + col], h0, l0);
+                split_bf16(hfull[g * DC::HPITCH + col + 1], h1, l1);
                 ah[s][q] = pack_bf16x2(h0, h1);
                 al[s][q] = pack_bf16x2(l0, l1);
             }
         }
-        const int n_begin = min(p.d_out, (int)crank * p.n_slice);
-        const int n_end = min(p.d_out, n_begin + p.n_slice);
-        const int ngrp = (n_end - n_begin + 31) / 32;
-        const bool store = tl.ok && row_ok;
-        __nv_bfloat16 *yrow = p.Y + (int64_t)(row_ok ? row_g : 0) * p.ldy;
-        // B row fed by lane (g, t) in n8 tile i of a group: 8 (g / 2) + 2 i + (g % 2)
-        const int brow = 8 * (g >> 1) + (g & 1);
-        for (int q0 = warp; q0 < ngrp; q0 += kWarps * RC::EB) {
-            uint2 bv[RC::EB][4][RC::KS];
-            uint4 yv[RC::EB];
-#pragma unroll
-            for (int e = 0; e < RC::EB; ++e) {
-                const int base = n_begin + (q0 + e * kWarps) * 32;
-                const bool gin = q0 + e * kWarps < ngrp;
-                const int bcol = base + brow;                  // + 2 i
-                const bool bin = gin && base + 8 * (g >> 1) < n_end;
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int s = 0; s < RC::KS; ++s) {
-                        if constexpr (R == 8) {
-                            const uint32_t v = bin ? __ldg(reinterpret_cast<const uint32_t *>(
-                                                         slotB + (int64_t)(bcol + 2 * i) * 8 + 2 * t))
-                                                   : 0u;
-                            bv[e][i][s] = make_uint2(v, 0u);
-                        } else {
-                            bv[e][i][s] = bin ? ldg_nc2(slotB + ((int64_t)(2 * s + (t >> 1)) * p.d_out +
-                                                                  bcol + 2 * i) * 8 + (t & 1) * 4)
-                                              : make_uint2(0u, 0u);
-                        }
-                    }
-                const bool cin = gin && base + 8 * t < n_end;
-                yv[e] = (cin && row_ok) ? *reinterpret_cast<const uint4 *>(yrow + base + 8 * t)
-                                        : make_uint4(0, 0, 0, 0);
+        const bool store = ok && row_ok;
+        for (int i = 0; i < ng; i += 2) {
+            mma_expand_store<R>(e0, ah, al, scale, yrow, store, sl, warp + i * kWarps, t);
+            if (i + 2 < ng) {
+                const int q = warp + (i + 2) * kWarps;
+                load_b<R>(e0, slotB, p.d_out, sl, q, g, t);
+                load_y<R>(e0, yrow, row_ok, sl, q, t);
             }
-#pragma unroll
-            for (int e = 0; e < RC::EB; ++e) {
-                const int base = n_begin + (q0 + e * kWarps) * 32;
-                const bool cin = (q0 + e * kWarps < ngrp) && base + 8 * t < n_end;
-                float d[4][4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    d[i][0] = d[i][1] = d[i][2] = d[i][3] = 0.f;
-#pragma unroll
-                    for (int s = 0; s < RC::KS; ++s) {
-                        if constexpr (R == 8) {
-                            mma_1688(d[i], ah[0][0], 0u, bv[e][i][0].x);
-                            mma_1688(d[i], al[0][0], 0u, bv[e][i][0].x);
-                        } else {
-                            mma_16816(d[i], ah[s][0], 0u, ah[s][1], 0u, bv[e][i][s].x, bv[e][i][s].y);
-                            mma_16816(d[i], al[s][0], 0u, al[s][1], 0u, bv[e][i][s].x, bv[e][i][s].y);
-                        }
-                    }
+            if (i + 1 < ng) {
+                mma_expand_store<R>(e1, ah, al, scale, yrow, store, sl, warp + (i + 1) * kWarps, t);
+                if (i + 3 < ng) {
+                    const int q = warp + (i + 3) * kWarps;
+                    load_b<R>(e1, slotB, p.d_out, sl, q, g, t);
+                    load_y<R>(e1, yrow, row_ok, sl, q, t);
                 }
-                // thread (g, t) holds row g, columns base + 8t + 2i + {0, 1}
-                const __nv_bfloat162 *y0 = reinterpret_cast<const __nv_bfloat162 *>(&yv[e]);
-                uint4 out;
-                uint32_t *o = reinterpret_cast<uint32_t *>(&out);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f = __bfloat1622float2(y0[i]);
-                    o[i] = pack_bf16x2(fmaf(tl.scale, d[i][0], f.x), fmaf(tl.scale, d[i][1], f.y));
-                }
-                if (store && cin) *reinterpret_cast<uint4 *>(yrow + base + 8 * t) = out;
             }
         }
     }
@@ -354,10 +479,9 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<RMAX>::MIN_BLOCKS)
     const uint32_t csize = cluster_size();
     const int n_clusters = (int)(gridDim.x / csize);
     const bool reporter = blockIdx.x == 0;
-    const int g = (tid & 31) >> 2;
 
     int tile = (int)cluster_index();
-    int total = scan_tiles(p, tile, ctl, reporter);
+    const int total = scan_tiles(p, tile, ctl, reporter);
     for (; tile < total; tile += n_clusters) {
         if (tile != (int)cluster_index()) scan_tiles(p, tile, ctl, false);
         // every CTA of the cluster reads the same metadata and reaches the same tile
@@ -367,35 +491,27 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<RMAX>::MIN_BLOCKS)
         tl.nvalid = min(TM, ctl.tile[2] - tl.p0);
         tl.slot = ctl.tile[3];
         const int r_meta = ctl.tile[4];
-        // rows of this tile (each lane needs row g), slot rank and scale
-        int row_g = -1;
-        if (g < tl.nvalid) {
-            row_g = p.token_indices ? p.token_indices[tl.p0 + g] : tl.p0 + g;
-            if (row_g < 0 || row_g >= p.n_rows) {
-                if (crank == 0 && (tid & 3) == 0 && tid < 32) report(p, kFlagBadRow);
-                row_g = -1;
-            }
+        const float seg_scale = ctl.seg_scale;
+        // rank bucket from the metadata when it is given and in range, else from the slot
+        int R = rank_bucket(r_meta);
+        if (p.ranks == nullptr || R == 0 || R > RMAX) {
+            __syncthreads();
+            if (tid == 0) ctl.slot_rank = p.slot_rank[tl.slot];
+            __syncthreads();
+            R = rank_bucket(ctl.slot_rank);
+            if (R == 0 || R > RMAX) R = 8;   // rejected inside; moves rank-8 bytes
         }
-        if (tid < 32 && (tid & 3) == 0) ctl.rows[g] = row_g;
-        if (tid == 0) {
-            ctl.slot_rank = p.slot_rank[tl.slot];
-            ctl.slot_scale = p.slot_scale[tl.slot];
-        }
-        __syncthreads();
-        const int r = ctl.slot_rank;
-        tl.ok = r > 0 && (p.ranks == nullptr || r_meta == r) && rank_bucket(r) <= RMAX;
-        if (tid == 0 && crank == 0 && !tl.ok) report(p, r <= 0 ? kFlagSlotEmpty : kFlagBadRank);
-        tl.rank = tl.ok ? r : 0;   // a rejected tile reads and writes no H
-        tl.scale = p.scales ? ctl.seg_scale : ctl.slot_scale;
-        const int R = tl.ok ? rank_bucket(r) : 8;
         if (R == 8) {
-            run_tile<RMAX, MODE, 8>(p, tl, row_g, ctl, smem_f, crank, csize);
+            run_tile<RMAX, MODE, 8>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize);
         } else if (R == 16) {
-            if constexpr (RMAX >= 16) run_tile<RMAX, MODE, 16>(p, tl, row_g, ctl, smem_f, crank, csize);
+            if constexpr (RMAX >= 16)
+                run_tile<RMAX, MODE, 16>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize);
         } else if (R == 32) {
-            if constexpr (RMAX >= 32) run_tile<RMAX, MODE, 32>(p, tl, row_g, ctl, smem_f, crank, csize);
+            if constexpr (RMAX >= 32)
+                run_tile<RMAX, MODE, 32>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize);
         } else {
-            if constexpr (RMAX >= 64) run_tile<RMAX, MODE, 64>(p, tl, row_g, ctl, smem_f, crank, csize);
+            if constexpr (RMAX >= 64)
+                run_tile<RMAX, MODE, 64>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize);
         }
         __syncthreads();   // ctl and the H buffers are rewritten by the next tile
     }
