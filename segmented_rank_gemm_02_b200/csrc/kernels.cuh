@@ -57,9 +57,30 @@ struct TileParams {
     // decomposition: CTA c of a cluster owns d_in columns [c*k_slice, (c+1)*k_slice)
     // for the shrink and d_out columns [c*n_slice, (c+1)*n_slice) for the expand.
     int32_t k_slice, n_slice;
-    // segments with at least this many grouped positions are left to another kernel
+    // segments with at least this many grouped positions go to the long-segment
+    // (tensor-memory) kernels; the others to the decode-shaped kernel
     int32_t long_rows;
+    // long-segment kernels: H of the long tiles, [n_tokens][ws_ld] fp32 (the pool's
+    // workspace in the fused apply, the caller's H in standalone shrink / expand)
+    float *ws;
+    int64_t ws_ld;
+    int32_t ksplit;            // CTAs per shrink cluster, each one part of d_in
+    int32_t k_part;            // d_in columns per part (multiple of 64)
+    int32_t n_unit;            // d_out columns per expand work unit (multiple of 128)
 };
+
+// Rows per tile of the long-segment kernels (one M=128 tensor-memory tile).
+constexpr int kLongTileRows = 128;
+// Long-segment kernels: number of d_out ranges of n_unit columns.
+__host__ __device__ inline int n_ranges(const TileParams &p) { return (p.d_out + p.n_unit - 1) / p.n_unit; }
+
+// Long-segment shrink (H of the long tiles into p.ws) and expand (reads p.ws; in
+// MODE_EXPAND it also reports the tiles' metadata problems); persistent grids.
+cudaError_t launch_long_shrink(int rmax_bucket, const TileParams &p, int64_t max_tiles,
+                               cudaStream_t stream);
+cudaError_t launch_long_expand(int rmax_bucket, int mode, const TileParams &p, int64_t max_units,
+                               cudaStream_t stream);
+cudaError_t prepare_long_kernels();
 
 // Launch the tile kernel for the pool's largest rank bucket `rmax_bucket`
 // (8/16/32/64) in mode `mode`, with clusters of `cluster` CTAs: as many clusters as

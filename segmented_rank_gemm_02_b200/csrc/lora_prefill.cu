@@ -1,0 +1,673 @@
+// lora_prefill.cu -- long segments (prefill-shaped): tcgen05 tensor-core tiles.
+//
+// The computation is the same as the decode family's (page "Multi-LoRA Serving:
+// adapter batching", sections "What metadata a segmented kernel needs" and
+// "Prefill and decode have different LoRA shapes": a prefill segment holds
+// hundreds to thousands of rows, so its two low-rank products are real matrix
+// multiplications).  A work tile is (segment, 128 consecutive grouped positions),
+// one M=128 tensor-memory tile.
+//
+// Shrink (long_shrink_kernel).  A thread-block cluster of `ksplit` CTAs owns a tile;
+// CTA c covers one part of d_in.  128 threads gather the tile's X rows (through
+// token_indices) and the adapter's A columns with 16-byte cp.async into a 4-stage
+// ring laid out as the tensor core's canonical K-major, no-swizzle operand layout
+// (8x8 core matrices of 128 contiguous bytes), two blocks ahead of the tensor core;
+// one thread issues tcgen05.mma (M=128, N=rank bucket, K=16 per instruction) into an
+// fp32 accumulator in tensor memory and commits each stage to an mbarrier that
+// frees it.  The epilogue reads the accumulator back with tcgen05.ld (one row per
+// thread); the cluster sums its partial tiles through distributed shared memory in
+// a fixed order and writes H (fp32) once.
+//
+// Expand (long_expand_kernel).  Work unit = (tile, range of d_out).  The tile's H is
+// written once to shared memory as bf16 hi + lo parts in the canonical layout; then
+// for each 128-column chunk -- double-buffered, the next chunk's B rows and Y0 rows
+// in flight while this one is multiplied and stored -- tcgen05.mma accumulates
+// H_hi B^T + H_lo B^T (M=128, N=128) in tensor memory, and the epilogue adds
+// s * acc to Y0, rounds to bf16 and stores each row with 16-byte stores.
+//
+// Rank buckets: kernels are compiled for the pool's largest bucket and dispatch each
+// tile to code for its own bucket (rank 8 runs as 16 with zero columns).
+// Every mbarrier wait is bounded; on expiry the kernel flags a timeout, stores
+// nothing more, waits again (bounded) for its tensor-core work and frees its
+// tensor memory before it leaves.
+#include <mutex>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace mlora {
+
+namespace {
+
+constexpr int PT = 128;               // threads per CTA = rows per tile
+constexpr int PM = kLongTileRows;     // 128
+constexpr int KB = 64;                // d_in columns per shrink block
+constexpr int NCH = 128;              // d_out columns per expand chunk
+constexpr int NS = 4;                 // shrink pipeline stages
+constexpr int PD = 2;                 // shrink prefetch distance (blocks ahead of the MMA)
+constexpr int kMaxSplit = 8;          // CTAs per shrink cluster
+constexpr uint64_t kWaitNs = 1000000000ull;
+
+__host__ __device__ constexpr int padded_rank(int r) { return r < 16 ? 16 : r; }
+
+template <int RMAX>
+struct LongCfg {
+    static constexpr int RK = padded_rank(RMAX);
+    static constexpr int X_STAGE = PM * KB * 2;         // 16 KB: [8 groups][16 row groups][8][8]
+    static constexpr int A_STAGE = KB * RK * 2;         // [8 groups][RK rows][8]
+    static constexpr int S_STAGE = X_STAGE + A_STAGE;
+    static constexpr int S_SMEM = NS * S_STAGE;
+    static constexpr int RED_PITCH = RK + 4;            // floats per row of a partial tile
+    static_assert(PM * RED_PITCH * 4 <= S_SMEM, "partial tile must fit in the ring");
+    static constexpr int S_TMEM = RK < 32 ? 32 : RK;
+    static constexpr int H_BYTES = PM * RK * 2;         // one of hi / lo: [RK/8][16][8][8]
+    static constexpr int B_BYTES = NCH * RK * 2;        // [RK/8][16 column groups][8][8]
+    static constexpr int YPITCH = NCH * 2 + 16;         // bytes per staged Y0 row
+    static constexpr int CHUNK_BYTES = B_BYTES + PM * YPITCH;
+    static constexpr int E_SMEM = 2 * H_BYTES + 2 * CHUNK_BYTES;
+    static constexpr int E_TMEM = NCH;
+};
+
+struct LongCtl {
+    uint64_t bar[NS];   // shrink: MMA completion per stage; expand: bar[0]
+    uint32_t tmem;
+    int scan[PT / 32];
+    int tile[5];        // segment, first position, end position, slot, rank from metadata
+    float seg_scale;
+    int slot_rank;
+    float slot_scale;
+    int rows[PM];
+    int fail;
+};
+
+__device__ __forceinline__ void report(const TileParams &p, unsigned flag) { atomicOr(p.status, flag); }
+
+// Block-wide scan of the long segments' tile counts; returns the number of tiles
+// and leaves tile `want` (if it exists) in ctl.tile.
+__device__ int scan_long(const TileParams &p, int want, LongCtl &ctl)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) ctl.tile[0] = -1;
+    __syncthreads();
+    int running = 0;
+    for (int base = 0; base < p.n_segments; base += PT) {
+        const int g = base + tid;
+        int cnt = 0, p0 = 0, p1 = 0, a = -1, rk = -1;
+        float sc = 0.f;
+        if (g < p.n_segments) {
+            a = p.slots[g];
+            p0 = p.offsets[g];
+            p1 = p.offsets[g + 1];
+            if (p.ranks) rk = p.ranks[g];
+            if (p.scales) sc = p.scales[g];
+            // malformed segments are reported by the decode-shaped kernel's scan
+            if (a >= 0 && a < p.n_slots && p0 >= 0 && p1 >= p0 && p1 <= p.n_tokens &&
+                p1 - p0 >= p.long_rows)
+                cnt = (p1 - p0 + PM - 1) / PM;
+        }
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) ctl.scan[warp] = incl;
+        __syncthreads();
+        int before = 0, total = 0;
+#pragma unroll
+        for (int w = 0; w < PT / 32; ++w) {
+            const int v = ctl.scan[w];
+            before += (w < warp) ? v : 0;
+            total += v;
+        }
+        incl += before;
+        const int lo = running + incl - cnt;
+        if (cnt > 0 && want >= lo && want < running + incl) {
+            ctl.tile[0] = g;
+            ctl.tile[1] = p0 + (want - lo) * PM;
+            ctl.tile[2] = p1;
+            ctl.tile[3] = a;
+            ctl.tile[4] = rk;
+            ctl.seg_scale = sc;
+        }
+        running += total;
+        __syncthreads();
+    }
+    return running;
+}
+
+// Rows of the current tile, the slot's rank and scale; returns the rank bucket to run
+// (0 if the tile must be skipped) and sets ok (results may be stored).
+__device__ int tile_setup(const TileParams &p, LongCtl &ctl, int nvalid, bool reporter, bool &ok,
+                          int &rank)
+{
+    const int tid = threadIdx.x;
+    const int p0 = ctl.tile[1], slot = ctl.tile[3], r_meta = ctl.tile[4];
+    int t = -1;
+    if (tid < nvalid) {
+        t = p.token_indices ? p.token_indices[p0 + tid] : p0 + tid;
+        if (t < 0 || t >= p.n_rows) {
+            if (reporter) report(p, kFlagBadRow);
+            t = -1;
+        }
+    }
+    ctl.rows[tid] = t;
+    if (tid == 0) {
+        ctl.slot_rank = p.slot_rank[slot];
+        ctl.slot_scale = p.slot_scale[slot];
+    }
+    __syncthreads();
+    const int r = ctl.slot_rank;
+    ok = r > 0 && (p.ranks == nullptr || r_meta == r) && rank_bucket(r) != 0;
+    if (reporter && tid == 0 && !ok) report(p, r <= 0 ? kFlagSlotEmpty : kFlagBadRank);
+    rank = ok ? r : 0;
+    return ok ? rank_bucket(r) : 0;
+}
+
+__device__ __forceinline__ bool wait_or_fail(const TileParams &p, LongCtl &ctl, uint64_t *bar,
+                                             uint32_t parity)
+{
+    if (ctl.fail) return false;
+    if (!mbar_wait_bounded(bar, parity, kWaitNs)) {
+        ctl.fail = 1;
+        report(p, kFlagTimeout);
+        return false;
+    }
+    return true;
+}
+
+// ------------------------------------------------------------------ shrink
+template <int RMAX, int R>
+__device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *smem, uint32_t tmem,
+                            uint32_t &gb, uint32_t crank, uint32_t csize, int nvalid, int rank,
+                            bool ok)
+{
+    using C = LongCfg<RMAX>;
+    constexpr int RK = padded_rank(R);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int p0 = ctl.tile[1], slot = ctl.tile[3];
+    const __nv_bfloat16 *slotA = p.pool + (int64_t)slot * p.slot_stride;
+    const int k0 = min(p.d_in, (int)crank * p.k_part);
+    const int k1 = min(p.d_in, k0 + p.k_part);
+    const int nkb = (k1 - k0 + KB - 1) / KB;
+    const int trow = ctl.rows[tid];
+    const __nv_bfloat16 *xrow = p.X + (int64_t)(trow >= 0 ? trow : 0) * p.ldx;
+    const uint32_t idesc = umma_idesc_bf16(PM, RK);
+
+    auto produce = [&](int b) {
+        const uint32_t G = gb + b;
+        const int s = G % NS;
+        if (G >= NS) wait_or_fail(p, ctl, &ctl.bar[s], ((G / NS) - 1) & 1u);
+        uint8_t *xs = smem + s * C::S_STAGE;
+        uint8_t *as = xs + C::X_STAGE;
+        const int kb0 = k0 + b * KB;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {   // this thread's row, eight 8-column groups
+            const int k = kb0 + 8 * j;
+            const bool v = trow >= 0 && k < k1;
+            cp_async16(xs + (j * (PM / 8) + tid / 8) * 128 + (tid % 8) * 16, v ? xrow + k : p.X, v);
+        }
+        for (int c = tid; c < 8 * RK; c += PT) {   // RK adapter rows (>= R are zero)
+            const int j = c / RK, n = c % RK;
+            const int k = kb0 + 8 * j;
+            const bool v = n < R && k < k1;
+            cp_async16(as + (j * RK + n) * 16, v ? slotA + ((int64_t)(k / 8) * R + n) * 8 : p.pool, v);
+        }
+    };
+    auto consume = [&](int b) {
+        const uint32_t G = gb + b;
+        const int s = G % NS;
+        cp_async_wait<PD>();
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0 && !ctl.fail) {
+            tc_fence_after();
+            const uint32_t xs = smem_addr(smem + s * C::S_STAGE);
+            const uint32_t as = xs + C::X_STAGE;
+#pragma unroll
+            for (int st = 0; st < KB / 16; ++st) {
+                const uint64_t ad = umma_desc_kmajor(xs + st * 2 * (PM / 8) * 128, (PM / 8) * 128, 128);
+                const uint64_t bd = umma_desc_kmajor(as + st * 2 * RK * 16, RK * 16, 128);
+                umma_bf16(tmem, ad, bd, idesc, (b > 0 || st > 0) ? 1u : 0u);
+            }
+            umma_commit(&ctl.bar[s]);
+        }
+    };
+
+    for (int b = 0; b < PD; ++b) {
+        if (b < nkb) produce(b);
+        cp_async_commit();
+    }
+    for (int b = 0; b < nkb; ++b) {
+        if (b + PD < nkb) produce(b + PD);
+        cp_async_commit();
+        consume(b);
+    }
+    gb += nkb;
+
+    // this CTA's partial tile: thread = row, read back from tensor memory
+    if (nkb > 0) {
+        const uint32_t G = gb - 1;
+        wait_or_fail(p, ctl, &ctl.bar[G % NS], (G / NS) & 1u);
+    }
+    tc_fence_after();
+    float h[RK];
+    if (nkb > 0) {
+        const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16);
+        if constexpr (RK == 16) {
+            uint32_t v0[8], v1[8];
+            tmem_ld8(taddr, v0);
+            tmem_ld8(taddr + 8, v1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                h[j] = __uint_as_float(v0[j]);
+                h[8 + j] = __uint_as_float(v1[j]);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < RK / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(taddr + 32 * c, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) h[32 * c + j] = __uint_as_float(v[j]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < RK; ++j) h[j] = 0.f;
+    }
+    // every block of this tile has been consumed, so the ring holds the partial tile
+    float *red = reinterpret_cast<float *>(smem);
+#pragma unroll
+    for (int j = 0; j < RK; j += 4)
+        *reinterpret_cast<float4 *>(red + tid * C::RED_PITCH + j) = make_float4(h[j], h[j + 1], h[j + 2], h[j + 3]);
+    tc_fence_before();
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    // rows r with r % csize == crank: sum the cluster's partials in CTA order, write H
+    if ((uint32_t)tid % csize == crank && ok && !ctl.fail && tid < nvalid && trow >= 0) {
+        float acc[RK];
+#pragma unroll
+        for (int j = 0; j < RK; ++j) acc[j] = 0.f;
+        const uint32_t row_addr = smem_addr(red + tid * C::RED_PITCH);
+        for (uint32_t c = 0; c < csize; ++c) {
+            const uint32_t base = map_to_rank(row_addr, c);
+#pragma unroll
+            for (int j = 0; j < RK; j += 4) {
+                const float4 v = ld_dsmem_f32x4(base + 4u * j);
+                acc[j] += v.x;
+                acc[j + 1] += v.y;
+                acc[j + 2] += v.z;
+                acc[j + 3] += v.w;
+            }
+        }
+        float *dst = p.ws + (int64_t)(p0 + tid) * p.ws_ld;
+#pragma unroll
+        for (int j = 0; j < RK; ++j)
+            if (j < rank) dst[j] = acc[j];
+    }
+    // peers are done reading this CTA's partial tile before the ring is refilled
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    __syncthreads();
+    tc_fence_after();
+}
+
+template <int RMAX>
+__global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__ TileParams p)
+{
+    using C = LongCfg<RMAX>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ LongCtl ctl;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const uint32_t crank = cluster_rank(), csize = cluster_size();
+    const int n_clusters = (int)(gridDim.x / csize);
+    if (warp == 0) {
+        tmem_alloc(&ctl.tmem, C::S_TMEM);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < NS; ++s) mbar_init(&ctl.bar[s], 1);
+        fence_mbar_init();
+        ctl.fail = 0;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl.tmem;
+    uint32_t gb = 0;
+    // every CTA of a cluster reads the same metadata and takes the same tiles
+    for (int tile = (int)cluster_index();; tile += n_clusters) {
+        const int ntiles = scan_long(p, tile, ctl);
+        if (tile >= ntiles) break;
+        const int nvalid = min(PM, ctl.tile[2] - ctl.tile[1]);
+        bool ok;
+        int rank;
+        const int R = tile_setup(p, ctl, nvalid, crank == 0, ok, rank);
+        if (R == 8) {
+            shrink_tile<RMAX, 8>(p, ctl, smem, tmem, gb, crank, csize, nvalid, rank, ok);
+        } else if (R == 16) {
+            shrink_tile<RMAX, 16>(p, ctl, smem, tmem, gb, crank, csize, nvalid, rank, ok);
+        } else if (R == 32) {
+            if constexpr (RMAX >= 32) shrink_tile<RMAX, 32>(p, ctl, smem, tmem, gb, crank, csize, nvalid, rank, ok);
+        } else if (R == 64) {
+            if constexpr (RMAX >= 64) shrink_tile<RMAX, 64>(p, ctl, smem, tmem, gb, crank, csize, nvalid, rank, ok);
+        }
+        __syncthreads();
+    }
+    // leave: no copies in flight, tensor-core work done, tensor memory freed
+    cp_async_wait<0>();
+    if (ctl.fail && tid == 0 && gb > 0) {
+        const uint32_t G = gb - 1;
+        mbar_wait_bounded(&ctl.bar[G % NS], (G / NS) & 1u, kWaitNs);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, C::S_TMEM);
+}
+
+// ------------------------------------------------------------------ expand
+template <int RMAX, int MODE, int R>
+__device__ void expand_unit(const TileParams &p, LongCtl &ctl, uint8_t *smem, uint32_t tmem,
+                            uint32_t &phase, int n_lo, int n_hi, int nvalid, int rank, bool ok,
+                            float scale)
+{
+    using C = LongCfg<RMAX>;
+    constexpr int RK = padded_rank(R);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int p0 = ctl.tile[1], slot = ctl.tile[3];
+    const __nv_bfloat16 *slotB = p.pool + (int64_t)slot * p.slot_stride + p.b_offset;
+    uint8_t *ahi = smem;
+    uint8_t *alo = smem + C::H_BYTES;
+    uint8_t *chunk0 = smem + 2 * C::H_BYTES;
+    const int trow = ctl.rows[tid];
+    const bool hrow = ok && tid < nvalid;
+    const bool store = hrow && trow >= 0 && !ctl.fail;
+    __nv_bfloat16 *yrow = p.Y + (int64_t)(trow >= 0 ? trow : 0) * p.ldy;
+
+    // this thread's H row as bf16 hi + lo, canonical K-major layout
+    const float *hsrc = p.ws + (int64_t)(p0 + (hrow ? tid : 0)) * p.ws_ld;
+    float h[RK];
+#pragma unroll
+    for (int j = 0; j < RK; ++j) h[j] = (hrow && j < rank) ? hsrc[j] : 0.f;
+#pragma unroll
+    for (int j = 0; j < RK / 8; ++j) {
+        uint4 hi, lo;
+        uint32_t *ph = reinterpret_cast<uint32_t *>(&hi);
+        uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float h0, l0, h1, l1;
+            split_bf16(h[8 * j + 2 * c], h0, l0);
+            split_bf16(h[8 * j + 2 * c + 1], h1, l1);
+            ph[c] = pack_bf16x2(h0, h1);
+            pl[c] = pack_bf16x2(l0, l1);
+        }
+        const int off = (j * (PM / 8) + tid / 8) * 128 + (tid % 8) * 16;
+        *reinterpret_cast<uint4 *>(ahi + off) = hi;
+        *reinterpret_cast<uint4 *>(alo + off) = lo;
+    }
+
+    auto issue = [&](int c0, uint8_t *buf) {
+        const int len = min(NCH, n_hi - c0);
+        uint8_t *bs = buf;
+        uint8_t *ys = buf + C::B_BYTES;
+#pragma unroll
+        for (int j = 0; j < RK / 8; ++j) {   // B rows of the chunk: column tid, RK/8 groups
+            const bool v = tid < len && 8 * j < R;
+            cp_async16(bs + (j * (NCH / 8) + tid / 8) * 128 + (tid % 8) * 16,
+                       v ? slotB + ((int64_t)j * p.d_out + c0 + tid) * 8 : p.pool, v);
+        }
+        if (store)
+            for (int q = 0; q < len / 8; ++q) cp_async16(ys + tid * C::YPITCH + 16 * q, yrow + c0 + 8 * q, true);
+    };
+
+    const uint32_t idesc = umma_idesc_bf16(PM, NCH);
+    const int nch = (n_hi - n_lo + NCH - 1) / NCH;
+    if (nch > 0) issue(n_lo, chunk0);
+    cp_async_commit();
+    for (int ci = 0; ci < nch; ++ci) {
+        const int c0 = n_lo + ci * NCH;
+        const int len = min(NCH, n_hi - c0);
+        uint8_t *buf = chunk0 + (ci & 1) * C::CHUNK_BYTES;
+        if (ci + 1 < nch) issue(c0 + NCH, chunk0 + ((ci + 1) & 1) * C::CHUNK_BYTES);
+        cp_async_commit();
+        cp_async_wait<1>();
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0 && !ctl.fail) {
+            tc_fence_after();
+            const uint32_t a_hi = smem_addr(ahi), a_lo = smem_addr(alo), b_s = smem_addr(buf);
+#pragma unroll
+            for (int st = 0; st < RK / 16; ++st) {
+                const uint32_t koff = st * 2 * (PM / 8) * 128;
+                const uint64_t bd = umma_desc_kmajor(b_s + st * 2 * (NCH / 8) * 128, (NCH / 8) * 128, 128);
+                umma_bf16(tmem, umma_desc_kmajor(a_hi + koff, (PM / 8) * 128, 128), bd, idesc,
+                          st > 0 ? 1u : 0u);
+                umma_bf16(tmem, umma_desc_kmajor(a_lo + koff, (PM / 8) * 128, 128), bd, idesc, 1u);
+            }
+            umma_commit(&ctl.bar[0]);
+        }
+        wait_or_fail(p, ctl, &ctl.bar[0], phase);
+        phase ^= 1u;
+        tc_fence_after();
+        // epilogue: thread = row; accumulator lanes 32*warp.. are this warp's rows
+        const uint8_t *ys = buf + C::B_BYTES;
+        const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16);
+        for (int cb = 0; cb < len; cb += 32) {
+            uint32_t v[32];
+            tmem_ld32(taddr + cb, v);
+            tmem_wait_ld();
+            if (store) {
+                const int ncol = min(32, len - cb);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (8 * q >= ncol) break;
+                    const uint4 y0 = *reinterpret_cast<const uint4 *>(ys + tid * C::YPITCH + (cb + 8 * q) * 2);
+                    const __nv_bfloat162 *y2 = reinterpret_cast<const __nv_bfloat162 *>(&y0);
+                    uint4 out;
+                    uint32_t *o = reinterpret_cast<uint32_t *>(&out);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(y2[e]);
+                        o[e] = pack_bf16x2(fmaf(scale, __uint_as_float(v[8 * q + 2 * e]), f.x),
+                                           fmaf(scale, __uint_as_float(v[8 * q + 2 * e + 1]), f.y));
+                    }
+                    *reinterpret_cast<uint4 *>(yrow + c0 + cb + 8 * q) = out;
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();   // this buffer and the accumulator are reused
+    }
+    cp_async_wait<0>();
+}
+
+template <int RMAX, int MODE>
+__global__ void __launch_bounds__(PT) long_expand_kernel(const __grid_constant__ TileParams p)
+{
+    using C = LongCfg<RMAX>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ LongCtl ctl;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if (warp == 0) {
+        tmem_alloc(&ctl.tmem, C::E_TMEM);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(&ctl.bar[0], 1);
+        fence_mbar_init();
+        ctl.fail = 0;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl.tmem;
+    uint32_t phase = 0;
+    const int nr = n_ranges(p);
+    for (int unit = blockIdx.x;; unit += gridDim.x) {
+        const int tile = unit / nr, range = unit % nr;
+        const int ntiles = scan_long(p, tile, ctl);
+        if (tile >= ntiles || ctl.fail) break;
+        const int nvalid = min(PM, ctl.tile[2] - ctl.tile[1]);
+        bool ok;
+        int rank;
+        // in the fused apply the shrink kernel reported this tile's metadata problems
+        const int R = tile_setup(p, ctl, nvalid, MODE == MODE_EXPAND && range == 0, ok, rank);
+        const float scale = p.scales ? ctl.seg_scale : ctl.slot_scale;
+        const int n_lo = range * p.n_unit, n_hi = min(p.d_out, n_lo + p.n_unit);
+        if (R == 8) {
+            expand_unit<RMAX, MODE, 8>(p, ctl, smem, tmem, phase, n_lo, n_hi, nvalid, rank, ok, scale);
+        } else if (R == 16) {
+            expand_unit<RMAX, MODE, 16>(p, ctl, smem, tmem, phase, n_lo, n_hi, nvalid, rank, ok, scale);
+        } else if (R == 32) {
+            if constexpr (RMAX >= 32)
+                expand_unit<RMAX, MODE, 32>(p, ctl, smem, tmem, phase, n_lo, n_hi, nvalid, rank, ok, scale);
+        } else if (R == 64) {
+            if constexpr (RMAX >= 64)
+                expand_unit<RMAX, MODE, 64>(p, ctl, smem, tmem, phase, n_lo, n_hi, nvalid, rank, ok, scale);
+        }
+        __syncthreads();
+    }
+    cp_async_wait<0>();
+    if (ctl.fail && tid == 0) mbar_wait_bounded(&ctl.bar[0], phase ^ 1u, kWaitNs);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, C::E_TMEM);
+}
+
+// ------------------------------------------------------------------ launches
+// CTAs of `kernel` resident per SM with `smem` bytes, limited by tensor memory.
+template <typename K>
+int resident_per_sm(K kernel, int smem, int tmem_cols)
+{
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, PT, smem) != cudaSuccess)
+        per_sm = 0;
+    if (per_sm <= 0) per_sm = 1;
+    return per_sm < 512 / tmem_cols ? per_sm : 512 / tmem_cols;
+}
+
+template <int RMAX>
+cudaError_t shrink_rmax(const TileParams &p, int64_t max_tiles, cudaStream_t stream)
+{
+    using C = LongCfg<RMAX>;
+    const int cluster = p.ksplit;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(PT, 1, 1);
+    cfg.dynamicSmemBytes = C::S_SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    static std::mutex mu;
+    static int cached[64][kMaxSplit + 1] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    int active;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        active = cached[dev][cluster];
+        if (active == 0) {
+            cfg.gridDim = dim3((unsigned)cluster, 1, 1);
+            cudaError_t e = cudaOccupancyMaxActiveClusters(&active, long_shrink_kernel<RMAX>, &cfg);
+            if (e != cudaSuccess) return e;
+            if (active <= 0) return cudaErrorInvalidConfiguration;
+            int sms = 0;
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            // tensor memory: at most 512 / S_TMEM CTAs per SM
+            const int cap = sms * (512 / C::S_TMEM) / cluster;
+            if (cap > 0 && active > cap) active = cap;
+            cached[dev][cluster] = active;
+        }
+    }
+    const int64_t n = max_tiles < active ? max_tiles : active;
+    if (n <= 0) return cudaSuccess;
+    cfg.gridDim = dim3((unsigned)(n * cluster), 1, 1);
+    return cudaLaunchKernelEx(&cfg, long_shrink_kernel<RMAX>, p);
+}
+
+template <int RMAX, int MODE>
+cudaError_t expand_rmax(const TileParams &p, int64_t max_units, cudaStream_t stream)
+{
+    using C = LongCfg<RMAX>;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int per_sm = resident_per_sm(long_expand_kernel<RMAX, MODE>, C::E_SMEM, C::E_TMEM);
+    const int64_t cap = (int64_t)sms * per_sm;
+    const int64_t n = max_units < cap ? max_units : cap;
+    if (n <= 0) return cudaSuccess;
+    long_expand_kernel<RMAX, MODE><<<(unsigned)n, PT, C::E_SMEM, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes)
+{
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+}
+
+template <int RMAX>
+cudaError_t set_long_attrs()
+{
+    using C = LongCfg<RMAX>;
+    cudaError_t e;
+    if ((e = set_smem(long_shrink_kernel<RMAX>, C::S_SMEM)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(long_shrink_kernel<RMAX>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess)
+        return e;
+    if ((e = set_smem(long_expand_kernel<RMAX, MODE_APPLY>, C::E_SMEM)) != cudaSuccess) return e;
+    return set_smem(long_expand_kernel<RMAX, MODE_EXPAND>, C::E_SMEM);
+}
+
+}  // namespace
+
+cudaError_t launch_long_shrink(int rmax_bucket, const TileParams &p, int64_t max_tiles,
+                               cudaStream_t stream)
+{
+    if (p.ksplit < 1 || p.ksplit > kMaxSplit) return cudaErrorInvalidValue;
+    switch (rmax_bucket) {
+    case 8:
+    case 16: return shrink_rmax<16>(p, max_tiles, stream);
+    case 32: return shrink_rmax<32>(p, max_tiles, stream);
+    case 64: return shrink_rmax<64>(p, max_tiles, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_long_expand(int rmax_bucket, int mode, const TileParams &p, int64_t max_units,
+                               cudaStream_t stream)
+{
+    const bool apply = mode == MODE_APPLY;
+    switch (rmax_bucket) {
+    case 8:
+    case 16: return apply ? expand_rmax<16, MODE_APPLY>(p, max_units, stream)
+                          : expand_rmax<16, MODE_EXPAND>(p, max_units, stream);
+    case 32: return apply ? expand_rmax<32, MODE_APPLY>(p, max_units, stream)
+                          : expand_rmax<32, MODE_EXPAND>(p, max_units, stream);
+    case 64: return apply ? expand_rmax<64, MODE_APPLY>(p, max_units, stream)
+                          : expand_rmax<64, MODE_EXPAND>(p, max_units, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t prepare_long_kernels()
+{
+    cudaError_t e;
+    if ((e = set_long_attrs<16>()) != cudaSuccess) return e;
+    if ((e = set_long_attrs<32>()) != cudaSuccess) return e;
+    return set_long_attrs<64>();
+}
+
+}  // namespace mlora

@@ -32,6 +32,9 @@ struct mlora_pool {
     unsigned int *d_status;
     std::vector<int32_t> h_rank;
     std::vector<float> h_alpha;
+    float *ws;              // H partial sums of the long-segment kernels (grown on demand)
+    size_t ws_bytes;
+    std::mutex ws_mutex;
 };
 
 namespace {
@@ -66,6 +69,7 @@ mlora_status prepare_device(int dev)
     if (dev < 0 || dev >= 128) return MLORA_ERR_INVALID_ARG;
     if (g_prepared[dev]) return MLORA_OK;
     if (mlora::prepare_tile_kernels() != cudaSuccess) return MLORA_ERR_CUDA;
+    if (mlora::prepare_long_kernels() != cudaSuccess) return MLORA_ERR_CUDA;
     g_prepared[dev] = true;
     return MLORA_OK;
 }
@@ -118,20 +122,94 @@ mlora::TileParams base_params(const mlora_pool *pool, const mlora_segments *s)
     return p;
 }
 
-mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::TileParams &p,
-                    void *stream)
+// Segments with at least this many rows go to the tensor-memory (long-segment) kernels.
+constexpr int kLongRows = 128;
+
+int sm_count(int dev)
 {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    return n;
+}
+
+// Make the pool's workspace hold `bytes`; growing it is not possible while the stream
+// is being captured into a graph.
+mlora_status ensure_workspace(mlora_pool *pool, size_t bytes, cudaStream_t stream)
+{
+    std::lock_guard<std::mutex> lock(pool->ws_mutex);
+    if (pool->ws_bytes >= bytes) return MLORA_OK;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return MLORA_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return MLORA_ERR_UNSUPPORTED;
+    if (pool->ws) {
+        if (cudaDeviceSynchronize() != cudaSuccess) return MLORA_ERR_CUDA;
+        cudaFree(pool->ws);
+        pool->ws = nullptr;
+        pool->ws_bytes = 0;
+    }
+    const size_t want = std::max<size_t>(bytes, (size_t)1 << 20);
+    if (cudaMalloc(&pool->ws, want) != cudaSuccess) {
+        cudaGetLastError();
+        return MLORA_ERR_OUT_OF_MEMORY;
+    }
+    pool->ws_bytes = want;
+    return MLORA_OK;
+}
+
+mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::TileParams &p,
+                    void *stream_v)
+{
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
     const int c = choose_cluster(pool->d_in, pool->d_out);
     p.k_slice = (int32_t)round_up((pool->d_in + c - 1) / c, 32);
     p.n_slice = (int32_t)round_up((pool->d_out + c - 1) / c, 8);
-    p.long_rows = 0x7fffffff;
-    // Upper bound on the number of work tiles of well-formed metadata.
-    const int64_t tiles = (int64_t)s->n_segments + (int64_t)s->n_tokens / mlora::kTileRows + 1;
+    // Long segments exist only if some segment may reach kLongRows (the host's hint,
+    // when given, rules them out); the decode kernel then leaves them alone.
+    const bool use_long = s->n_tokens >= kLongRows &&
+                          (s->max_segment_rows <= 0 || s->max_segment_rows >= kLongRows);
+    p.long_rows = use_long ? kLongRows : 0x7fffffff;
     mlora_status st = prepare_device(pool->device);
     if (st != MLORA_OK) return st;
-    cudaError_t e = mlora::launch_tile_kernel(mode, pool->r_bucket_max, p, c, tiles,
-                                              static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? MLORA_OK : MLORA_ERR_CUDA;
+
+    const int64_t tiles = (int64_t)s->n_segments + (int64_t)s->n_tokens / mlora::kTileRows + 1;
+    cudaError_t e = mlora::launch_tile_kernel(mode, pool->r_bucket_max, p, c, tiles, stream);
+    if (e != cudaSuccess) return MLORA_ERR_CUDA;
+    if (!use_long) return MLORA_OK;
+
+    const int sms = sm_count(pool->device);
+    const int64_t long_tiles = (int64_t)s->n_tokens / mlora::kLongTileRows + s->n_tokens / kLongRows + 1;
+    const int64_t est_tiles = std::max<int64_t>(1, s->n_tokens / mlora::kLongTileRows);
+    const int rk = std::max(16, pool->r_bucket_max);
+    // shrink: a cluster of ksplit CTAs per tile, each a part of d_in; about one CTA per SM
+    int ksplit = (int)std::min<int64_t>(8, std::max<int64_t>(1, sms / est_tiles));
+    p.k_part = (int32_t)round_up((pool->d_in + ksplit - 1) / ksplit, 64);
+    ksplit = (pool->d_in + p.k_part - 1) / p.k_part;
+    p.ksplit = ksplit;
+    // expand: ranges of whole 128-column chunks, about four units per SM
+    const int64_t chunks = (pool->d_out + 127) / 128;
+    const int64_t ranges = std::min<int64_t>(chunks, std::max<int64_t>(1, (4 * sms + est_tiles - 1) / est_tiles));
+    p.n_unit = (int32_t)(((chunks + ranges - 1) / ranges) * 128);
+    const int64_t nr = (pool->d_out + p.n_unit - 1) / p.n_unit;
+
+    if (mode == mlora::MODE_APPLY) {
+        const size_t bytes = (size_t)s->n_tokens * rk * sizeof(float);
+        st = ensure_workspace(pool, bytes, stream);
+        if (st != MLORA_OK) return st;
+        p.ws = pool->ws;
+        p.ws_ld = rk;
+    } else {
+        p.ws = p.H;
+        p.ws_ld = p.ldh;
+    }
+    if (mode != mlora::MODE_EXPAND) {
+        e = mlora::launch_long_shrink(pool->r_bucket_max, p, long_tiles, stream);
+        if (e != cudaSuccess) return MLORA_ERR_CUDA;
+    }
+    if (mode != mlora::MODE_SHRINK) {
+        e = mlora::launch_long_expand(pool->r_bucket_max, mode, p, long_tiles * nr, stream);
+        if (e != cudaSuccess) return MLORA_ERR_CUDA;
+    }
+    return MLORA_OK;
 }
 
 }  // namespace
@@ -185,6 +263,8 @@ mlora_status mlora_pool_create(int32_t d_in, int32_t d_out, int32_t n_slots, int
     pool->d_rank = nullptr;
     pool->d_scale = nullptr;
     pool->d_status = nullptr;
+    pool->ws = nullptr;
+    pool->ws_bytes = 0;
     pool->h_rank.assign(n_slots, 0);
     pool->h_alpha.assign(n_slots, 0.f);
 
@@ -220,6 +300,7 @@ mlora_status mlora_pool_destroy(mlora_pool *pool)
     if (pool->d_rank) cudaFree(pool->d_rank);
     if (pool->d_scale) cudaFree(pool->d_scale);
     if (pool->d_status) cudaFree(pool->d_status);
+    if (pool->ws) cudaFree(pool->ws);
     delete pool;
     return MLORA_OK;
 }
