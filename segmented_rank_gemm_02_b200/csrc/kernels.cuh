@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -67,6 +68,9 @@ struct TileParams {
     int32_t ksplit;            // CTAs per shrink cluster, each one part of d_in
     int32_t k_part;            // d_in columns per part (multiple of 64)
     int32_t n_unit;            // d_out columns per expand work unit (multiple of 128)
+    // TMA views (bf16, 128-byte swizzle) of X [n_rows, d_in] and Y [n_rows, d_out]:
+    // 64 x 128 tiles for runs of consecutive rows, 64 x 1 rows for gathers
+    CUtensorMap x_tile, x_rows, y_tile, y_rows;
 };
 
 // Rows per tile of the long-segment kernels (one M=128 tensor-memory tile).

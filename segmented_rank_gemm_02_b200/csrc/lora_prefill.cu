@@ -1,35 +1,36 @@
-// lora_prefill.cu -- long segments (prefill-shaped): tcgen05 tensor-core tiles.
+// lora_prefill.cu -- long segments (prefill-shaped): TMA + tcgen05 tensor-core tiles.
 //
 // The computation is the same as the decode family's (page "Multi-LoRA Serving:
 // adapter batching", sections "What metadata a segmented kernel needs" and
-// "Prefill and decode have different LoRA shapes": a prefill segment holds
-// hundreds to thousands of rows, so its two low-rank products are real matrix
+// "Prefill and decode have different LoRA shapes": a prefill segment holds hundreds
+// to thousands of rows, so its two low-rank products are real matrix
 // multiplications).  A work tile is (segment, 128 consecutive grouped positions),
 // one M=128 tensor-memory tile.
 //
 // Shrink (long_shrink_kernel).  A thread-block cluster of `ksplit` CTAs owns a tile;
-// CTA c covers one part of d_in.  128 threads gather the tile's X rows (through
-// token_indices) and the adapter's A columns with 16-byte cp.async into a 4-stage
-// ring laid out as the tensor core's canonical K-major, no-swizzle operand layout
-// (8x8 core matrices of 128 contiguous bytes), two blocks ahead of the tensor core;
-// one thread issues tcgen05.mma (M=128, N=rank bucket, K=16 per instruction) into an
-// fp32 accumulator in tensor memory and commits each stage to an mbarrier that
-// frees it.  The epilogue reads the accumulator back with tcgen05.ld (one row per
-// thread); the cluster sums its partial tiles through distributed shared memory in
-// a fixed order and writes H (fp32) once.
+// CTA c covers one part of d_in.  One thread drives a 6-stage ring: per 64-column
+// block it issues one TMA tile load of X (128 rows x 64 columns, 128-byte swizzle)
+// when the tile's rows are consecutive in X, else 32 four-row TMA gathers, plus one
+// bulk copy of the adapter's A block (pool layout [8 groups][R][8] is already the
+// tensor core's no-swizzle K-major layout), all completing on the stage's mbarrier;
+// four blocks later it issues tcgen05.mma (M=128, N=rank bucket, K=16 each) into an
+// fp32 accumulator in tensor memory and commits the stage.  The epilogue reads the
+// accumulator with tcgen05.ld; the cluster sums its partial tiles through
+// distributed shared memory in a fixed order and writes H (fp32) once.
 //
 // Expand (long_expand_kernel).  Work unit = (tile, range of d_out).  The tile's H is
-// written once to shared memory as bf16 hi + lo parts in the canonical layout; then
-// for each 128-column chunk -- double-buffered, the next chunk's B rows and Y0 rows
-// in flight while this one is multiplied and stored -- tcgen05.mma accumulates
-// H_hi B^T + H_lo B^T (M=128, N=128) in tensor memory, and the epilogue adds
-// s * acc to Y0, rounds to bf16 and stores each row with 16-byte stores.
+// written once to shared memory as bf16 hi + lo parts (no-swizzle K-major); then per
+// 128-column chunk -- three buffers, two chunks in flight -- one thread issues the
+// bulk copies of the adapter's B rows and the TMA loads (tile or gathers) of the Y0
+// rows, then tcgen05.mma accumulates H_hi B^T + H_lo B^T (M=128, N=128) in tensor
+// memory; the epilogue adds s * acc to Y0 in shared memory and all threads store
+// whole rows with coalesced 16-byte stores.
 //
 // Rank buckets: kernels are compiled for the pool's largest bucket and dispatch each
-// tile to code for its own bucket (rank 8 runs as 16 with zero columns).
-// Every mbarrier wait is bounded; on expiry the kernel flags a timeout, stores
-// nothing more, waits again (bounded) for its tensor-core work and frees its
-// tensor memory before it leaves.
+// tile to code for its own bucket (bucket 8 runs as 16; its missing operand half is
+// read from a block of zeros).  Every mbarrier wait is bounded; on expiry the kernel
+// flags a timeout, stores nothing more, waits again (bounded) for its tensor-core
+// work and frees its tensor memory before it leaves.
 #include <mutex>
 
 #include "kernels.cuh"
@@ -39,13 +40,16 @@ namespace mlora {
 
 namespace {
 
-constexpr int PT = 128;               // threads per CTA = rows per tile
-constexpr int PM = kLongTileRows;     // 128
-constexpr int KB = 64;                // d_in columns per shrink block
+constexpr int PT = 256;               // threads per CTA: two per tile row
+constexpr int PM = kLongTileRows;     // 128 rows per tile
+constexpr int KB = 64;                // d_in columns per shrink block (one 128-byte row)
 constexpr int NCH = 128;              // d_out columns per expand chunk
-constexpr int NS = 4;                 // shrink pipeline stages
-constexpr int PD = 2;                 // shrink prefetch distance (blocks ahead of the MMA)
+constexpr int NS = 6;                 // shrink pipeline stages
+constexpr int PD = 4;                 // shrink prefetch distance (blocks ahead of the MMA)
+constexpr int NB = 3;                 // expand chunk buffers
+constexpr int ED = 2;                 // expand prefetch distance (chunks ahead)
 constexpr int kMaxSplit = 8;          // CTAs per shrink cluster
+constexpr int kZeroBytes = 2048;      // zero operand half for rank bucket 8
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 __host__ __device__ constexpr int padded_rank(int r) { return r < 16 ? 16 : r; }
@@ -53,23 +57,24 @@ __host__ __device__ constexpr int padded_rank(int r) { return r < 16 ? 16 : r; }
 template <int RMAX>
 struct LongCfg {
     static constexpr int RK = padded_rank(RMAX);
-    static constexpr int X_STAGE = PM * KB * 2;         // 16 KB: [8 groups][16 row groups][8][8]
-    static constexpr int A_STAGE = KB * RK * 2;         // [8 groups][RK rows][8]
-    static constexpr int S_STAGE = X_STAGE + A_STAGE;
-    static constexpr int S_SMEM = NS * S_STAGE;
-    static constexpr int RED_PITCH = RK + 4;            // floats per row of a partial tile
-    static_assert(PM * RED_PITCH * 4 <= S_SMEM, "partial tile must fit in the ring");
+    static constexpr int X_STAGE = PM * KB * 2;          // 16 KB, 128-byte swizzle
+    static constexpr int A_STAGE = (8 * RK * 16 + 1023) / 1024 * 1024;   // [8][RK][8]
+    static constexpr int S_STAGE = X_STAGE + A_STAGE;    // multiple of 1024
+    static constexpr int RED_PITCH = RK + 4;             // floats per row of a partial tile
+    static constexpr int S_SMEM = 1024 + NS * S_STAGE + kZeroBytes;   // + alignment slack
+    static_assert(PM * RED_PITCH * 4 <= NS * S_STAGE, "partial tile must fit in the ring");
     static constexpr int S_TMEM = RK < 32 ? 32 : RK;
-    static constexpr int H_BYTES = PM * RK * 2;         // one of hi / lo: [RK/8][16][8][8]
-    static constexpr int B_BYTES = NCH * RK * 2;        // [RK/8][16 column groups][8][8]
-    static constexpr int YPITCH = NCH * 2 + 16;         // bytes per staged Y0 row
-    static constexpr int CHUNK_BYTES = B_BYTES + PM * YPITCH;
-    static constexpr int E_SMEM = 2 * H_BYTES + 2 * CHUNK_BYTES;
+    static constexpr int H_BYTES = PM * RK * 2;          // one of hi / lo: [RK/8][16][8][8]
+    static constexpr int B_BYTES = (NCH * RK * 2 + 1023) / 1024 * 1024;  // [RK/8][128][8]
+    static constexpr int Y_BYTES = PM * NCH * 2;         // two 64-column halves, swizzled
+    static constexpr int CHUNK_BYTES = B_BYTES + Y_BYTES;
+    static constexpr int E_SMEM = 1024 + NB * CHUNK_BYTES + 2 * H_BYTES + kZeroBytes;
     static constexpr int E_TMEM = NCH;
 };
 
 struct LongCtl {
-    uint64_t bar[NS];   // shrink: MMA completion per stage; expand: bar[0]
+    uint64_t bar[NS];   // MMA done per stage (expand: bar[0])
+    uint64_t full[NS];  // operands of a stage / chunk buffer landed
     uint32_t tmem;
     int scan[PT / 32];
     int tile[5];        // segment, first position, end position, slot, rank from metadata
@@ -77,10 +82,16 @@ struct LongCtl {
     int slot_rank;
     float slot_scale;
     int rows[PM];
+    int contiguous;     // the tile's rows are consecutive in X / Y
     int fail;
 };
 
 __device__ __forceinline__ void report(const TileParams &p, unsigned flag) { atomicOr(p.status, flag); }
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p)
+{
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
 
 // Block-wide scan of the long segments' tile counts; returns the number of tiles
 // and leaves tile `want` (if it exists) in ctl.tile.
@@ -136,26 +147,32 @@ __device__ int scan_long(const TileParams &p, int want, LongCtl &ctl)
     return running;
 }
 
-// Rows of the current tile, the slot's rank and scale; returns the rank bucket to run
-// (0 if the tile must be skipped) and sets ok (results may be stored).
+// Rows of the current tile, whether they are consecutive, the slot's rank and scale;
+// returns the rank bucket to run (0 if the tile must be skipped) and sets ok.
 __device__ int tile_setup(const TileParams &p, LongCtl &ctl, int nvalid, bool reporter, bool &ok,
                           int &rank)
 {
     const int tid = threadIdx.x;
     const int p0 = ctl.tile[1], slot = ctl.tile[3], r_meta = ctl.tile[4];
     int t = -1;
-    if (tid < nvalid) {
+    if (tid < PM && tid < nvalid) {
         t = p.token_indices ? p.token_indices[p0 + tid] : p0 + tid;
         if (t < 0 || t >= p.n_rows) {
             if (reporter) report(p, kFlagBadRow);
             t = -1;
         }
     }
-    ctl.rows[tid] = t;
+    if (tid < PM) ctl.rows[tid] = t;
     if (tid == 0) {
         ctl.slot_rank = p.slot_rank[slot];
         ctl.slot_scale = p.slot_scale[slot];
     }
+    __syncthreads();
+    // consecutive rows, all present: one TMA tile covers the tile's X / Y rows
+    const bool mine = tid >= PM || tid >= nvalid ||
+                      (ctl.rows[tid] >= 0 && ctl.rows[tid] == ctl.rows[0] + tid);
+    const int contiguous = __syncthreads_and(mine ? 1 : 0);
+    if (tid == 0) ctl.contiguous = contiguous;
     __syncthreads();
     const int r = ctl.slot_rank;
     ok = r > 0 && (p.ranks == nullptr || r_meta == r) && rank_bucket(r) != 0;
@@ -176,11 +193,30 @@ __device__ __forceinline__ bool wait_or_fail(const TileParams &p, LongCtl &ctl, 
     return true;
 }
 
+// Issue the loads of rows [0, 128) of a tile, 64 columns from c0, into a 16 KB
+// swizzled destination: one tile load when the rows are consecutive, else 32
+// four-row gathers (absent rows read past the end of the tensor, as zeros).
+__device__ __forceinline__ void load_rows(const LongCtl &ctl, const CUtensorMap *tile_map,
+                                          const CUtensorMap *rows_map, int n_rows, uint8_t *dst,
+                                          int c0, uint64_t *bar)
+{
+    if (ctl.contiguous) {
+        tma_load_2d(dst, tile_map, c0, ctl.rows[0], bar);
+    } else {
+        for (int i = 0; i < PM; i += 4) {
+            int r[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) r[q] = ctl.rows[i + q] >= 0 ? ctl.rows[i + q] : n_rows;
+            tma_gather4(dst + i * 128, rows_map, c0, r[0], r[1], r[2], r[3], bar);
+        }
+    }
+}
+
 // ------------------------------------------------------------------ shrink
 template <int RMAX, int R>
-__device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *smem, uint32_t tmem,
-                            uint32_t &gb, uint32_t crank, uint32_t csize, int nvalid, int rank,
-                            bool ok)
+__device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, uint8_t *zero,
+                            uint32_t tmem, uint32_t &gb, uint32_t crank, uint32_t csize,
+                            int nvalid, int rank, bool ok)
 {
     using C = LongCfg<RMAX>;
     constexpr int RK = padded_rank(R);
@@ -190,71 +226,68 @@ __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *smem, ui
     const int k0 = min(p.d_in, (int)crank * p.k_part);
     const int k1 = min(p.d_in, k0 + p.k_part);
     const int nkb = (k1 - k0 + KB - 1) / KB;
-    const int trow = ctl.rows[tid];
-    const __nv_bfloat16 *xrow = p.X + (int64_t)(trow >= 0 ? trow : 0) * p.ldx;
     const uint32_t idesc = umma_idesc_bf16(PM, RK);
+    constexpr uint32_t A_BYTES = 8 * R * 16;
 
-    auto produce = [&](int b) {
-        const uint32_t G = gb + b;
-        const int s = G % NS;
-        if (G >= NS) wait_or_fail(p, ctl, &ctl.bar[s], ((G / NS) - 1) & 1u);
-        uint8_t *xs = smem + s * C::S_STAGE;
-        uint8_t *as = xs + C::X_STAGE;
-        const int kb0 = k0 + b * KB;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {   // this thread's row, eight 8-column groups
-            const int k = kb0 + 8 * j;
-            const bool v = trow >= 0 && k < k1;
-            cp_async16(xs + (j * (PM / 8) + tid / 8) * 128 + (tid % 8) * 16, v ? xrow + k : p.X, v);
-        }
-        for (int c = tid; c < 8 * RK; c += PT) {   // RK adapter rows (>= R are zero)
-            const int j = c / RK, n = c % RK;
-            const int k = kb0 + 8 * j;
-            const bool v = n < R && k < k1;
-            cp_async16(as + (j * RK + n) * 16, v ? slotA + ((int64_t)(k / 8) * R + n) * 8 : p.pool, v);
-        }
-    };
-    auto consume = [&](int b) {
-        const uint32_t G = gb + b;
-        const int s = G % NS;
-        cp_async_wait<PD>();
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0 && !ctl.fail) {
+    // one thread drives the ring: loads PD blocks ahead of the tensor core
+    if (tid == 0) {
+        auto produce = [&](int b) {
+            const uint32_t G = gb + b;
+            const int s = G % NS;
+            if (G >= NS) wait_or_fail(p, ctl, &ctl.bar[s], ((G / NS) - 1) & 1u);
+            uint8_t *xs = ring + s * C::S_STAGE;
+            uint8_t *as = xs + C::X_STAGE;
+            const int kb0 = k0 + b * KB;
+            mbar_arrive_expect_tx(&ctl.full[s], (uint32_t)C::X_STAGE + A_BYTES);
+            load_rows(ctl, &p.x_tile, &p.x_rows, p.n_rows, xs, kb0, &ctl.full[s]);
+            bulk_load(as, slotA + (int64_t)(kb0 / 8) * R * 8, A_BYTES, &ctl.full[s]);
+        };
+        auto consume = [&](int b) {
+            const uint32_t G = gb + b;
+            const int s = G % NS;
+            if (!wait_or_fail(p, ctl, &ctl.full[s], (G / NS) & 1u)) return;
             tc_fence_after();
-            const uint32_t xs = smem_addr(smem + s * C::S_STAGE);
+            const uint32_t xs = smem_addr(ring + s * C::S_STAGE);
             const uint32_t as = xs + C::X_STAGE;
 #pragma unroll
             for (int st = 0; st < KB / 16; ++st) {
-                const uint64_t ad = umma_desc_kmajor(xs + st * 2 * (PM / 8) * 128, (PM / 8) * 128, 128);
-                const uint64_t bd = umma_desc_kmajor(as + st * 2 * RK * 16, RK * 16, 128);
+                const uint32_t a0 = as + st * 2 * R * 16;
+                // adapter rows 8 .. 15 of bucket 8 come from the zero block
+                const uint32_t sbo = (R == 8) ? smem_addr(zero) - a0 : 128;
+                const uint64_t ad = umma_desc_sw128(xs + st * 32);
+                const uint64_t bd = umma_desc_kmajor(a0, R * 16, sbo);
                 umma_bf16(tmem, ad, bd, idesc, (b > 0 || st > 0) ? 1u : 0u);
             }
             umma_commit(&ctl.bar[s]);
+        };
+        for (int b = 0; b < nkb + PD; ++b) {
+            if (b < nkb) produce(b);
+            if (b >= PD) consume(b - PD);
         }
-    };
-
-    for (int b = 0; b < PD; ++b) {
-        if (b < nkb) produce(b);
-        cp_async_commit();
-    }
-    for (int b = 0; b < nkb; ++b) {
-        if (b + PD < nkb) produce(b + PD);
-        cp_async_commit();
-        consume(b);
+        if (nkb > 0) {
+            const uint32_t G = gb + nkb - 1;
+            wait_or_fail(p, ctl, &ctl.bar[G % NS], (G / NS) & 1u);
+        }
     }
     gb += nkb;
-
-    // this CTA's partial tile: thread = row, read back from tensor memory
-    if (nkb > 0) {
-        const uint32_t G = gb - 1;
-        wait_or_fail(p, ctl, &ctl.bar[G % NS], (G / NS) & 1u);
-    }
+    tc_fence_before();
+    __syncthreads();
     tc_fence_after();
-    float h[RK];
+
+    // this CTA's partial tile from tensor memory: warp w holds rows 32 (w % 4) .. +31
+    // and columns [(w / 4) * RK/2, +RK/2)
+    constexpr int HC = RK / 2;
+    float h[HC];
+    const int col0 = (warp / 4) * HC;
     if (nkb > 0) {
-        const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16);
-        if constexpr (RK == 16) {
+        const uint32_t taddr = tmem + ((uint32_t)(32 * (warp % 4)) << 16) + col0;
+        if constexpr (HC == 8) {
+            uint32_t v0[8];
+            tmem_ld8(taddr, v0);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h[j] = __uint_as_float(v0[j]);
+        } else if constexpr (HC == 16) {
             uint32_t v0[8], v1[8];
             tmem_ld8(taddr, v0);
             tmem_ld8(taddr + 8, v1);
@@ -265,29 +298,30 @@ __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *smem, ui
                 h[8 + j] = __uint_as_float(v1[j]);
             }
         } else {
+            uint32_t v[32];
+            tmem_ld32(taddr, v);
+            tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < RK / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld32(taddr + 32 * c, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) h[32 * c + j] = __uint_as_float(v[j]);
-            }
+            for (int j = 0; j < 32; ++j) h[j] = __uint_as_float(v[j]);
         }
     } else {
 #pragma unroll
-        for (int j = 0; j < RK; ++j) h[j] = 0.f;
+        for (int j = 0; j < HC; ++j) h[j] = 0.f;
     }
     // every block of this tile has been consumed, so the ring holds the partial tile
-    float *red = reinterpret_cast<float *>(smem);
+    float *red = reinterpret_cast<float *>(ring);
+    const int trow = 32 * (warp % 4) + (tid & 31);
 #pragma unroll
-    for (int j = 0; j < RK; j += 4)
-        *reinterpret_cast<float4 *>(red + tid * C::RED_PITCH + j) = make_float4(h[j], h[j + 1], h[j + 2], h[j + 3]);
+    for (int j = 0; j < HC; j += 4)
+        *reinterpret_cast<float4 *>(red + trow * C::RED_PITCH + col0 + j) =
+            make_float4(h[j], h[j + 1], h[j + 2], h[j + 3]);
     tc_fence_before();
     cluster_arrive_release();
     cluster_wait_acquire();
-    // rows r with r % csize == crank: sum the cluster's partials in CTA order, write H
-    if ((uint32_t)tid % csize == crank && ok && !ctl.fail && tid < nvalid && trow >= 0) {
+    // rows r with r % csize == crank (one thread each): sum the cluster's partials in
+    // CTA order and write H
+    if (tid < PM && (uint32_t)tid % csize == crank && ok && !ctl.fail && tid < nvalid &&
+        ctl.rows[tid] >= 0) {
         float acc[RK];
 #pragma unroll
         for (int j = 0; j < RK; ++j) acc[j] = 0.f;
@@ -311,6 +345,7 @@ __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *smem, ui
     // peers are done reading this CTA's partial tile before the ring is refilled
     cluster_arrive_release();
     cluster_wait_acquire();
+    fence_proxy_async_smem();   // the ring is next written by TMA
     __syncthreads();
     tc_fence_after();
 }
@@ -319,8 +354,10 @@ template <int RMAX>
 __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__ TileParams p)
 {
     using C = LongCfg<RMAX>;
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ LongCtl ctl;
+    uint8_t *ring = align1024(smem_raw);
+    uint8_t *zero = ring + NS * C::S_STAGE;
     const int tid = threadIdx.x, warp = tid >> 5;
     const uint32_t crank = cluster_rank(), csize = cluster_size();
     const int n_clusters = (int)(gridDim.x / csize);
@@ -328,12 +365,17 @@ __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__
         tmem_alloc(&ctl.tmem, C::S_TMEM);
         tmem_relinquish();
     }
+    for (int i = tid; i < kZeroBytes / 16; i += PT) reinterpret_cast<uint4 *>(zero)[i] = make_uint4(0, 0, 0, 0);
     if (tid == 0) {
 #pragma unroll
-        for (int s = 0; s < NS; ++s) mbar_init(&ctl.bar[s], 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&ctl.bar[s], 1);
+            mbar_init(&ctl.full[s], 1);
+        }
         fence_mbar_init();
         ctl.fail = 0;
     }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -348,21 +390,26 @@ __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__
         int rank;
         const int R = tile_setup(p, ctl, nvalid, crank == 0, ok, rank);
         if (R == 8) {
-            shrink_tile<RMAX, 8>(p, ctl, smem, tmem, gb, crank, csize, nvalid, rank, ok);
+            shrink_tile<RMAX, 8>(p, ctl, ring, zero, tmem, gb, crank, csize, nvalid, rank, ok);
         } else if (R == 16) {
-            shrink_tile<RMAX, 16>(p, ctl, smem, tmem, gb, crank, csize, nvalid, rank, ok);
+            shrink_tile<RMAX, 16>(p, ctl, ring, zero, tmem, gb, crank, csize, nvalid, rank, ok);
         } else if (R == 32) {
-            if constexpr (RMAX >= 32) shrink_tile<RMAX, 32>(p, ctl, smem, tmem, gb, crank, csize, nvalid, rank, ok);
+            if constexpr (RMAX >= 32)
+                shrink_tile<RMAX, 32>(p, ctl, ring, zero, tmem, gb, crank, csize, nvalid, rank, ok);
         } else if (R == 64) {
-            if constexpr (RMAX >= 64) shrink_tile<RMAX, 64>(p, ctl, smem, tmem, gb, crank, csize, nvalid, rank, ok);
+            if constexpr (RMAX >= 64)
+                shrink_tile<RMAX, 64>(p, ctl, ring, zero, tmem, gb, crank, csize, nvalid, rank, ok);
         }
         __syncthreads();
     }
-    // leave: no copies in flight, tensor-core work done, tensor memory freed
-    cp_async_wait<0>();
+    // leave: tensor-core work done, tensor memory freed
     if (ctl.fail && tid == 0 && gb > 0) {
         const uint32_t G = gb - 1;
         mbar_wait_bounded(&ctl.bar[G % NS], (G / NS) & 1u, kWaitNs);
+        // let copies still in flight land before shared memory is released
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 2000000ull) {
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -372,102 +419,119 @@ __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__
 
 // ------------------------------------------------------------------ expand
 template <int RMAX, int MODE, int R>
-__device__ void expand_unit(const TileParams &p, LongCtl &ctl, uint8_t *smem, uint32_t tmem,
-                            uint32_t &phase, int n_lo, int n_hi, int nvalid, int rank, bool ok,
-                            float scale)
+__device__ void expand_unit(const TileParams &p, LongCtl &ctl, uint8_t *bufs, uint8_t *hbuf,
+                            uint8_t *zero, uint32_t tmem, uint32_t &cg, int n_lo, int n_hi,
+                            int nvalid, int rank, bool ok, float scale)
 {
     using C = LongCfg<RMAX>;
     constexpr int RK = padded_rank(R);
     const int tid = threadIdx.x, warp = tid >> 5;
+    const int row = tid % PM, half = tid / PM;   // two threads per row
     const int p0 = ctl.tile[1], slot = ctl.tile[3];
     const __nv_bfloat16 *slotB = p.pool + (int64_t)slot * p.slot_stride + p.b_offset;
-    uint8_t *ahi = smem;
-    uint8_t *alo = smem + C::H_BYTES;
-    uint8_t *chunk0 = smem + 2 * C::H_BYTES;
-    const int trow = ctl.rows[tid];
-    const bool hrow = ok && tid < nvalid;
-    const bool store = hrow && trow >= 0 && !ctl.fail;
-    __nv_bfloat16 *yrow = p.Y + (int64_t)(trow >= 0 ? trow : 0) * p.ldy;
+    uint8_t *ahi = hbuf;
+    uint8_t *alo = hbuf + C::H_BYTES;
+    const bool hrow = ok && row < nvalid;
 
-    // this thread's H row as bf16 hi + lo, canonical K-major layout
-    const float *hsrc = p.ws + (int64_t)(p0 + (hrow ? tid : 0)) * p.ws_ld;
-    float h[RK];
+    // this thread's half of its H row as bf16 hi + lo, canonical no-swizzle K-major layout
+    {
+        constexpr int HC = RK / 2;
+        const float *hsrc = p.ws + (int64_t)(p0 + (hrow ? row : 0)) * p.ws_ld + half * HC;
+        float h[HC];
 #pragma unroll
-    for (int j = 0; j < RK; ++j) h[j] = (hrow && j < rank) ? hsrc[j] : 0.f;
+        for (int j = 0; j < HC; ++j) h[j] = (hrow && half * HC + j < rank) ? hsrc[j] : 0.f;
 #pragma unroll
-    for (int j = 0; j < RK / 8; ++j) {
-        uint4 hi, lo;
-        uint32_t *ph = reinterpret_cast<uint32_t *>(&hi);
-        uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
+        for (int jg = 0; jg < HC / 8; ++jg) {
+            uint4 hi, lo;
+            uint32_t *ph = reinterpret_cast<uint32_t *>(&hi);
+            uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            float h0, l0, h1, l1;
-            split_bf16(h[8 * j + 2 * c], h0, l0);
-            split_bf16(h[8 * j + 2 * c + 1], h1, l1);
-            ph[c] = pack_bf16x2(h0, h1);
-            pl[c] = pack_bf16x2(l0, l1);
+            for (int c = 0; c < 4; ++c) {
+                float h0, l0, h1, l1;
+                split_bf16(h[8 * jg + 2 * c], h0, l0);
+                split_bf16(h[8 * jg + 2 * c + 1], h1, l1);
+                ph[c] = pack_bf16x2(h0, h1);
+                pl[c] = pack_bf16x2(l0, l1);
+            }
+            const int j = half * (HC / 8) + jg;
+            const int off = (j * (PM / 8) + row / 8) * 128 + (row % 8) * 16;
+            *reinterpret_cast<uint4 *>(ahi + off) = hi;
+            *reinterpret_cast<uint4 *>(alo + off) = lo;
         }
-        const int off = (j * (PM / 8) + tid / 8) * 128 + (tid % 8) * 16;
-        *reinterpret_cast<uint4 *>(ahi + off) = hi;
-        *reinterpret_cast<uint4 *>(alo + off) = lo;
     }
+    fence_proxy_async_smem();   // the H tile is read by the tensor core
+    __syncthreads();
 
-    auto issue = [&](int c0, uint8_t *buf) {
-        const int len = min(NCH, n_hi - c0);
+    const int nch = (n_hi - n_lo + NCH - 1) / NCH;
+    const bool load_y = ok && !ctl.fail;
+    // chunk ci of this unit uses buffer (cg + ci) % NB; cg counts chunks across units
+    auto issue = [&](int ci) {   // thread 0
+        const uint32_t G = cg + ci;
+        uint8_t *buf = bufs + (G % NB) * C::CHUNK_BYTES;
         uint8_t *bs = buf;
         uint8_t *ys = buf + C::B_BYTES;
-#pragma unroll
-        for (int j = 0; j < RK / 8; ++j) {   // B rows of the chunk: column tid, RK/8 groups
-            const bool v = tid < len && 8 * j < R;
-            cp_async16(bs + (j * (NCH / 8) + tid / 8) * 128 + (tid % 8) * 16,
-                       v ? slotB + ((int64_t)j * p.d_out + c0 + tid) * 8 : p.pool, v);
-        }
-        if (store)
-            for (int q = 0; q < len / 8; ++q) cp_async16(ys + tid * C::YPITCH + 16 * q, yrow + c0 + 8 * q, true);
-    };
-
-    const uint32_t idesc = umma_idesc_bf16(PM, NCH);
-    const int nch = (n_hi - n_lo + NCH - 1) / NCH;
-    if (nch > 0) issue(n_lo, chunk0);
-    cp_async_commit();
-    for (int ci = 0; ci < nch; ++ci) {
         const int c0 = n_lo + ci * NCH;
         const int len = min(NCH, n_hi - c0);
-        uint8_t *buf = chunk0 + (ci & 1) * C::CHUNK_BYTES;
-        if (ci + 1 < nch) issue(c0 + NCH, chunk0 + ((ci + 1) & 1) * C::CHUNK_BYTES);
-        cp_async_commit();
-        cp_async_wait<1>();
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0 && !ctl.fail) {
-            tc_fence_after();
-            const uint32_t a_hi = smem_addr(ahi), a_lo = smem_addr(alo), b_s = smem_addr(buf);
-#pragma unroll
-            for (int st = 0; st < RK / 16; ++st) {
-                const uint32_t koff = st * 2 * (PM / 8) * 128;
-                const uint64_t bd = umma_desc_kmajor(b_s + st * 2 * (NCH / 8) * 128, (NCH / 8) * 128, 128);
-                umma_bf16(tmem, umma_desc_kmajor(a_hi + koff, (PM / 8) * 128, 128), bd, idesc,
-                          st > 0 ? 1u : 0u);
-                umma_bf16(tmem, umma_desc_kmajor(a_lo + koff, (PM / 8) * 128, 128), bd, idesc, 1u);
-            }
-            umma_commit(&ctl.bar[0]);
+        uint32_t bytes = (uint32_t)(R / 8) * len * 16;
+        if (load_y) bytes += (len > 64 ? 2 : 1) * PM * 64 * 2;
+        mbar_arrive_expect_tx(&ctl.full[G % NB], bytes);
+        for (int j = 0; j < R / 8; ++j)   // B rows c0.., rank group j: len x 16 bytes
+            bulk_load(bs + j * NCH * 16, slotB + ((int64_t)j * p.d_out + c0) * 8, len * 16, &ctl.full[G % NB]);
+        if (load_y) {
+            load_rows(ctl, &p.y_tile, &p.y_rows, p.n_rows, ys, c0, &ctl.full[G % NB]);
+            if (len > 64) load_rows(ctl, &p.y_tile, &p.y_rows, p.n_rows, ys + PM * 128, c0 + 64, &ctl.full[G % NB]);
         }
-        wait_or_fail(p, ctl, &ctl.bar[0], phase);
-        phase ^= 1u;
+    };
+    if (tid == 0)
+        for (int q = 0; q < ED && q < nch; ++q) issue(q);
+
+    const uint32_t idesc = umma_idesc_bf16(PM, NCH);
+    // epilogue geometry: warp w computes rows 32 (w % 4) .. and columns [64 (w / 4), +64)
+    // (= swizzled half w / 4) into the staged Y0 rows; then all threads store whole rows
+    const int erow = 32 * (warp % 4) + (tid & 31);
+    const bool compute = ok && erow < nvalid && ctl.rows[erow] >= 0;
+    const int ehalf = warp / 4;
+    for (int ci = 0; ci < nch; ++ci) {
+        const uint32_t G = cg + ci;
+        const int c0 = n_lo + ci * NCH;
+        const int len = min(NCH, n_hi - c0);
+        uint8_t *buf = bufs + (G % NB) * C::CHUNK_BYTES;
+        uint8_t *ys = buf + C::B_BYTES;
+        if (tid == 0) {
+            if (ci + ED < nch) issue(ci + ED);
+            if (wait_or_fail(p, ctl, &ctl.full[G % NB], (G / NB) & 1u)) {
+                tc_fence_after();
+                const uint32_t a_hi = smem_addr(ahi), a_lo = smem_addr(alo), b_s = smem_addr(buf);
+#pragma unroll
+                for (int st = 0; st < RK / 16; ++st) {
+                    const uint32_t koff = st * 2 * (PM / 8) * 128;
+                    const uint32_t b0 = b_s + st * 2 * NCH * 16;
+                    // bucket 8: the second rank group of B is the zero block
+                    const uint32_t lbo = (R == 8) ? smem_addr(zero) - b0 : NCH * 16;
+                    const uint64_t bd = umma_desc_kmajor(b0, lbo, 128);
+                    umma_bf16(tmem, umma_desc_kmajor(a_hi + koff, (PM / 8) * 128, 128), bd, idesc,
+                              st > 0 ? 1u : 0u);
+                    umma_bf16(tmem, umma_desc_kmajor(a_lo + koff, (PM / 8) * 128, 128), bd, idesc, 1u);
+                }
+                umma_commit(&ctl.bar[0]);
+            }
+        }
+        wait_or_fail(p, ctl, &ctl.bar[0], G & 1u);
         tc_fence_after();
-        // epilogue: thread = row; accumulator lanes 32*warp.. are this warp's rows
-        const uint8_t *ys = buf + C::B_BYTES;
-        const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16);
-        for (int cb = 0; cb < len; cb += 32) {
+        const uint32_t taddr = tmem + ((uint32_t)(32 * (warp % 4)) << 16) + 64 * ehalf;
+        uint8_t *yh = ys + ehalf * PM * 128 + erow * 128;   // this row of this half, swizzled
+#pragma unroll
+        for (int cb = 0; cb < 64; cb += 32) {
+            if (64 * ehalf + cb >= len) break;
             uint32_t v[32];
             tmem_ld32(taddr + cb, v);
             tmem_wait_ld();
-            if (store) {
-                const int ncol = min(32, len - cb);
+            if (compute) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    if (8 * q >= ncol) break;
-                    const uint4 y0 = *reinterpret_cast<const uint4 *>(ys + tid * C::YPITCH + (cb + 8 * q) * 2);
+                    const int chunk = cb / 8 + q;                      // 16-byte chunk in the row
+                    uint4 *yp = reinterpret_cast<uint4 *>(yh + ((chunk ^ (erow & 7)) * 16));
+                    const uint4 y0 = *yp;
                     const __nv_bfloat162 *y2 = reinterpret_cast<const __nv_bfloat162 *>(&y0);
                     uint4 out;
                     uint32_t *o = reinterpret_cast<uint32_t *>(&out);
@@ -477,37 +541,58 @@ __device__ void expand_unit(const TileParams &p, LongCtl &ctl, uint8_t *smem, ui
                         o[e] = pack_bf16x2(fmaf(scale, __uint_as_float(v[8 * q + 2 * e]), f.x),
                                            fmaf(scale, __uint_as_float(v[8 * q + 2 * e + 1]), f.y));
                     }
-                    *reinterpret_cast<uint4 *>(yrow + c0 + cb + 8 * q) = out;
+                    *yp = out;
                 }
             }
         }
         tc_fence_before();
-        __syncthreads();   // this buffer and the accumulator are reused
+        __syncthreads();
+        // coalesced stores: sixteen lanes per row, 16 bytes each
+#pragma unroll
+        for (int k = 0; k < (PM * NCH / 8) / PT; ++k) {
+            const int i = tid + k * PT;
+            const int r = i / (NCH / 8), q = i % (NCH / 8);
+            const int tr = ctl.rows[r];
+            if (ok && !ctl.fail && r < nvalid && tr >= 0 && 8 * q < len) {
+                const uint8_t *src = ys + (q / 8) * PM * 128 + r * 128 + (((q % 8) ^ (r & 7)) * 16);
+                *reinterpret_cast<uint4 *>(p.Y + (int64_t)tr * p.ldy + c0 + 8 * q) =
+                    *reinterpret_cast<const uint4 *>(src);
+            }
+        }
+        fence_proxy_async_smem();   // this buffer is next written by TMA
+        __syncthreads();
     }
-    cp_async_wait<0>();
+    cg += nch;
 }
 
 template <int RMAX, int MODE>
 __global__ void __launch_bounds__(PT) long_expand_kernel(const __grid_constant__ TileParams p)
 {
     using C = LongCfg<RMAX>;
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ LongCtl ctl;
+    uint8_t *bufs = align1024(smem_raw);
+    uint8_t *hbuf = bufs + NB * C::CHUNK_BYTES;
+    uint8_t *zero = hbuf + 2 * C::H_BYTES;
     const int tid = threadIdx.x, warp = tid >> 5;
     if (warp == 0) {
         tmem_alloc(&ctl.tmem, C::E_TMEM);
         tmem_relinquish();
     }
+    for (int i = tid; i < kZeroBytes / 16; i += PT) reinterpret_cast<uint4 *>(zero)[i] = make_uint4(0, 0, 0, 0);
     if (tid == 0) {
         mbar_init(&ctl.bar[0], 1);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) mbar_init(&ctl.full[b], 1);
         fence_mbar_init();
         ctl.fail = 0;
     }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl.tmem;
-    uint32_t phase = 0;
+    uint32_t cg = 0;   // chunks multiplied so far (buffer and barrier phases)
     const int nr = n_ranges(p);
     for (int unit = blockIdx.x;; unit += gridDim.x) {
         const int tile = unit / nr, range = unit % nr;
@@ -521,20 +606,24 @@ __global__ void __launch_bounds__(PT) long_expand_kernel(const __grid_constant__
         const float scale = p.scales ? ctl.seg_scale : ctl.slot_scale;
         const int n_lo = range * p.n_unit, n_hi = min(p.d_out, n_lo + p.n_unit);
         if (R == 8) {
-            expand_unit<RMAX, MODE, 8>(p, ctl, smem, tmem, phase, n_lo, n_hi, nvalid, rank, ok, scale);
+            expand_unit<RMAX, MODE, 8>(p, ctl, bufs, hbuf, zero, tmem, cg, n_lo, n_hi, nvalid, rank, ok, scale);
         } else if (R == 16) {
-            expand_unit<RMAX, MODE, 16>(p, ctl, smem, tmem, phase, n_lo, n_hi, nvalid, rank, ok, scale);
+            expand_unit<RMAX, MODE, 16>(p, ctl, bufs, hbuf, zero, tmem, cg, n_lo, n_hi, nvalid, rank, ok, scale);
         } else if (R == 32) {
             if constexpr (RMAX >= 32)
-                expand_unit<RMAX, MODE, 32>(p, ctl, smem, tmem, phase, n_lo, n_hi, nvalid, rank, ok, scale);
+                expand_unit<RMAX, MODE, 32>(p, ctl, bufs, hbuf, zero, tmem, cg, n_lo, n_hi, nvalid, rank, ok, scale);
         } else if (R == 64) {
             if constexpr (RMAX >= 64)
-                expand_unit<RMAX, MODE, 64>(p, ctl, smem, tmem, phase, n_lo, n_hi, nvalid, rank, ok, scale);
+                expand_unit<RMAX, MODE, 64>(p, ctl, bufs, hbuf, zero, tmem, cg, n_lo, n_hi, nvalid, rank, ok, scale);
         }
         __syncthreads();
     }
-    cp_async_wait<0>();
-    if (ctl.fail && tid == 0) mbar_wait_bounded(&ctl.bar[0], phase ^ 1u, kWaitNs);
+    if (ctl.fail && tid == 0) {
+        if (cg > 0) mbar_wait_bounded(&ctl.bar[0], (cg - 1) & 1u, kWaitNs);
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 2000000ull) {
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

@@ -18,6 +18,7 @@
 #include <vector>
 
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include "kernels.cuh"
 
@@ -125,6 +126,36 @@ mlora::TileParams base_params(const mlora_pool *pool, const mlora_segments *s)
 // Segments with at least this many rows go to the tensor-memory (long-segment) kernels.
 constexpr int kLongRows = 128;
 
+// cuTensorMapEncodeTiled, fetched once through the runtime (no link to the driver library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// bf16 [rows, cols] with row stride ld (elements), 128-byte swizzle, box 64 x box_rows.
+bool encode_rows_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, int64_t ld,
+                     uint32_t box_rows)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (enc == nullptr || base == nullptr || rows <= 0 || cols <= 0) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t elem[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, elem,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count(int dev)
 {
     int n = 0;
@@ -165,8 +196,9 @@ mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::
     p.n_slice = (int32_t)round_up((pool->d_out + c - 1) / c, 8);
     // Long segments exist only if some segment may reach kLongRows (the host's hint,
     // when given, rules them out); the decode kernel then leaves them alone.
-    const bool use_long = s->n_tokens >= kLongRows &&
-                          (s->max_segment_rows <= 0 || s->max_segment_rows >= kLongRows);
+    const bool use_long = s->n_tokens >= kLongRows && pool->d_in % 64 == 0 &&
+                          (s->max_segment_rows <= 0 || s->max_segment_rows >= kLongRows) &&
+                          tensor_map_encoder() != nullptr;
     p.long_rows = use_long ? kLongRows : 0x7fffffff;
     mlora_status st = prepare_device(pool->device);
     if (st != MLORA_OK) return st;
@@ -191,6 +223,15 @@ mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::
     p.n_unit = (int32_t)(((chunks + ranges - 1) / ranges) * 128);
     const int64_t nr = (pool->d_out + p.n_unit - 1) / p.n_unit;
 
+    // TMA views of the activations (tiles of consecutive rows, and single rows for gathers)
+    if (mode != mlora::MODE_EXPAND &&
+        (!encode_rows_map(&p.x_tile, p.X, s->n_rows, pool->d_in, p.ldx, mlora::kLongTileRows) ||
+         !encode_rows_map(&p.x_rows, p.X, s->n_rows, pool->d_in, p.ldx, 1)))
+        return MLORA_ERR_CUDA;
+    if (mode != mlora::MODE_SHRINK &&
+        (!encode_rows_map(&p.y_tile, p.Y, s->n_rows, pool->d_out, p.ldy, mlora::kLongTileRows) ||
+         !encode_rows_map(&p.y_rows, p.Y, s->n_rows, pool->d_out, p.ldy, 1)))
+        return MLORA_ERR_CUDA;
     if (mode == mlora::MODE_APPLY) {
         const size_t bytes = (size_t)s->n_tokens * rk * sizeof(float);
         st = ensure_workspace(pool, bytes, stream);

@@ -271,6 +271,13 @@ __device__ __forceinline__ void cp_async16(void *dst_smem, const void *src, bool
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
+// Arrive on `bar` once every cp.async issued so far by this thread has completed
+// (the barrier's expected count includes this thread; no increment).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
@@ -364,5 +371,48 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8])
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+}  // namespace mlora
+
+// ---------------------------------------------------------------- TMA tensor copies
+namespace mlora {
+
+// 2-D tile load [c0, c0 + box_cols) x [r0, r0 + box_rows) described by `map` (kernel
+// parameter space).  Out-of-range rows and columns read as zero.
+__device__ __forceinline__ void tma_load_2d(void *dst_smem, const void *map, int c0, int r0,
+                                            uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_addr(dst_smem)), "l"(map), "r"(c0), "r"(r0), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Four rows r0..r3 (any order, out-of-range rows read as zero), columns
+// [c0, c0 + box_cols), placed one after another; the map's box is one row high.
+__device__ __forceinline__ void tma_gather4(void *dst_smem, const void *map, int c0, int r0, int r1,
+                                            int r2, int r3, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+        ::"r"(smem_addr(dst_smem)), "l"(map), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+          "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Shared-memory descriptor: K-major, 128-byte swizzle (rows of 128 bytes in 8-row,
+// 1024-byte atoms).  K advances inside the atom by moving the start address.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_byte_addr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_byte_addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;             // leading byte offset: unused for this layout (16 B)
+    d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset: 8-row atoms
+    d |= (uint64_t)1 << 46;             // descriptor version of this architecture
+    d |= (uint64_t)2 << 61;             // layout: 128-byte swizzle
+    return d;
+}
 
 }  // namespace mlora
