@@ -167,6 +167,34 @@ mlora_status mlora_apply(mlora_pool *pool, const mlora_segments *segs, const voi
                          int64_t ldx, void *Y, int64_t ldy, void *stream);
 
 /*
+ * mlora_apply for callers that cannot allocate device memory.  The paper has no
+ * counterpart: this entry point is an interface choice of this library.
+ *
+ * Same operation, arguments and errors as mlora_apply.  mlora_apply keeps the fp32
+ * H values of long segments (128 rows or more) in a workspace that the pool grows
+ * with cudaMalloc the first time a batch needs more.  Some callers cannot allow
+ * that: a serving engine that reserves nearly all of HBM for weights and KV cache
+ * up front and hands out memory only from its own allocator (a library cudaMalloc
+ * would fail or eat into that reservation), or a latency-critical loop that must not
+ * hit the device-wide synchronisation a cudaMalloc / cudaFree can cause.  This
+ * variant takes the workspace from a fixed scratch array in the library's own device
+ * memory instead, and calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - The scratch array is 4 MiB; every GPU that loads the library holds it until
+ *     the process exits.  A batch needs n_tokens * max(16, bucket(r_max)) * 4 bytes
+ *     (up to 16384 grouped rows for a rank-64 pool, 65536 for r_max <= 16); larger
+ *     batches return MLORA_ERR_UNSUPPORTED with nothing launched.
+ *   - The first call on a device looks up the array's device address (with the
+ *     pool's device current) and keeps it; make that first call before any stream
+ *     capture.
+ *   - Every call shares the one array, which keeps the last call's contents (no
+ *     part of it needs to start at zero: each call writes the H values it reads).
+ *     Calls whose kernels overlap on the GPU -- on different streams, from several
+ *     threads, or for several pools -- race on it: serialise them.
+ */
+mlora_status mlora_apply_noalloc(mlora_pool *pool, const mlora_segments *segs, const void *X,
+                                 int64_t ldx, void *Y, int64_t ldy, void *stream);
+
+/*
  * Host helper: group rows by slot (row_slots[t] = slot of row t, -1 = base).
  * Segments come in the order their slot first appears; rows keep their original
  * order inside a segment.  Outputs are HOST arrays the caller sizes:

@@ -31,7 +31,8 @@ FLAG_BAD_OFFSETS, FLAG_BAD_SLOT, FLAG_BAD_RANK, FLAG_BAD_ROW, FLAG_SLOT_EMPTY, F
 EXPORTS = ("mlora_pool_create", "mlora_pool_destroy", "mlora_pool_load_slot",
            "mlora_pool_clear_slot", "mlora_pool_slot_info", "mlora_pool_shape",
            "mlora_pool_check", "mlora_shrink", "mlora_expand", "mlora_apply",
-           "mlora_build_segments", "mlora_status_string", "mlora_version")
+           "mlora_apply_noalloc", "mlora_build_segments", "mlora_status_string",
+           "mlora_version")
 
 
 class MloraError(RuntimeError):
@@ -66,6 +67,7 @@ def _load():
         "mlora_shrink": [vp, seg_p, vp, i64, vp, i64, vp],
         "mlora_expand": [vp, seg_p, vp, i64, vp, i64, vp],
         "mlora_apply": [vp, seg_p, vp, i64, vp, i64, vp],
+        "mlora_apply_noalloc": [vp, seg_p, vp, i64, vp, i64, vp],
         "mlora_build_segments": [vp, i32, vp, vp, vp, i32p, i32p, vp, vp],
     }
     for name, args in sig.items():
@@ -251,6 +253,13 @@ def apply(pool: Pool, segs: DeviceSegments, X, Y, stream=None) -> None:
     """Y[t] = bf16(Y[t] + s (X[t] A^T) B^T) in place (mlora_apply)."""
     _check(lib().mlora_apply(pool.handle, ctypes.byref(segs.struct), _ptr(X), _ld(X, "X"),
                             _ptr(Y), _ld(Y, "Y"), _stream_ptr(stream)), "mlora_apply")
+
+
+def apply_noalloc(pool: Pool, segs: DeviceSegments, X, Y, stream=None) -> None:
+    """mlora_apply with the long-segment scratch in the library's fixed device array
+    (mlora_apply_noalloc): allocates nothing; concurrent calls on the GPU race."""
+    _check(lib().mlora_apply_noalloc(pool.handle, ctypes.byref(segs.struct), _ptr(X), _ld(X, "X"),
+                                     _ptr(Y), _ld(Y, "Y"), _stream_ptr(stream)), "mlora_apply_noalloc")
 
 
 def shrink(pool: Pool, segs: DeviceSegments, X, H, stream=None) -> None:

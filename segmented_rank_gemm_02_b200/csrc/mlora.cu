@@ -187,8 +187,10 @@ mlora_status ensure_workspace(mlora_pool *pool, size_t bytes, cudaStream_t strea
     return MLORA_OK;
 }
 
+// `ext_ws` (optional): caller-provided memory of `ext_ws_bytes` for the long-segment H
+// workspace, used instead of the pool's own (which is then never grown).
 mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::TileParams &p,
-                    void *stream_v)
+                    void *stream_v, float *ext_ws = nullptr, size_t ext_ws_bytes = 0)
 {
     cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
     const int c = choose_cluster(pool->d_in, pool->d_out);
@@ -232,7 +234,11 @@ mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::
         (!encode_rows_map(&p.y_tile, p.Y, s->n_rows, pool->d_out, p.ldy, mlora::kLongTileRows) ||
          !encode_rows_map(&p.y_rows, p.Y, s->n_rows, pool->d_out, p.ldy, 1)))
         return MLORA_ERR_CUDA;
-    if (mode == mlora::MODE_APPLY) {
+    if (mode == mlora::MODE_APPLY && ext_ws != nullptr) {
+        if ((size_t)s->n_tokens * rk * sizeof(float) > ext_ws_bytes) return MLORA_ERR_UNSUPPORTED;
+        p.ws = ext_ws;
+        p.ws_ld = rk;
+    } else if (mode == mlora::MODE_APPLY) {
         const size_t bytes = (size_t)s->n_tokens * rk * sizeof(float);
         st = ensure_workspace(pool, bytes, stream);
         if (st != MLORA_OK) return st;
@@ -254,6 +260,32 @@ mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::
 }
 
 }  // namespace
+
+// Fused apply whose long-segment workspace is caller-provided memory (no allocation);
+// used by mlora_apply_noalloc.  Same checks as mlora_apply, plus the size limit.
+mlora_status mlora_apply_with_workspace(mlora_pool *pool, const mlora_segments *segs,
+                                        const void *X, int64_t ldx, void *Y, int64_t ldy,
+                                        void *stream, float *ws, size_t ws_bytes)
+{
+    mlora_status st = check_segments(pool, segs);
+    if (st != MLORA_OK) return st;
+    if ((size_t)segs->n_tokens * std::max(16, pool->r_bucket_max) * sizeof(float) > ws_bytes)
+        return MLORA_ERR_UNSUPPORTED;
+    if (segs->n_segments == 0 || segs->n_tokens == 0) return MLORA_OK;
+    if (X == nullptr || Y == nullptr || !aligned16(X) || !aligned16(Y)) return MLORA_ERR_INVALID_ARG;
+    if (ldx < pool->d_in || ldx % 8 != 0 || ldy < pool->d_out || ldy % 8 != 0)
+        return MLORA_ERR_INVALID_ARG;
+    DeviceGuard guard(pool->device);
+    if (!guard.ok) return MLORA_ERR_CUDA;
+    mlora::TileParams p = base_params(pool, segs);
+    p.X = static_cast<const __nv_bfloat16 *>(X);
+    p.ldx = ldx;
+    p.Y = static_cast<__nv_bfloat16 *>(Y);
+    p.ldy = ldy;
+    return launch(pool, segs, mlora::MODE_APPLY, p, stream, ws, ws_bytes);
+}
+
+int mlora_pool_device(const mlora_pool *pool) { return pool ? pool->device : -1; }
 
 extern "C" {
 
