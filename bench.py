@@ -72,6 +72,47 @@ def workload_facts(W) -> dict:
             "bytes": total_bytes, "flops": flops, "per_projection": per_proj}
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """Largest ``x`` over all ranks of the process group (``x`` itself without one).
+    Every rank must call it the same number of times."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, steps: int, world: int, seconds: float) -> float:
+    """Units that all ranks processed (each rank its own batch) per second of the
+    slowest rank's time."""
+    return units_per_rank * steps * world / seconds
+
+
+def graph_kernel_count(graph):
+    """Kernel nodes in a captured torch CUDA graph (the launches one replay makes), or
+    None if the graph cannot be inspected."""
+    try:
+        from cuda.bindings import runtime as cudart
+        g = cudart.cudaGraph_t(init_value=int(graph.raw_cuda_graph()))
+        err, _, n = cudart.cudaGraphGetNodes(g, numNodes=0)
+        if err != cudart.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = cudart.cudaGraphGetNodes(g, numNodes=n)
+        if err != cudart.cudaError_t.cudaSuccess:
+            return None
+        count = 0
+        for node in nodes[:n]:
+            err, t = cudart.cudaGraphNodeGetType(node)
+            if err != cudart.cudaError_t.cudaSuccess:
+                return None
+            count += int(t == cudart.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+        return count
+    except Exception:
+        return None
+
+
 def measured_peaks() -> dict:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -285,6 +326,11 @@ def run_ours(args, rank: int, world: int, device_index: int):
     with torch.cuda.stream(stream):
         graph.replay()   # first replay uploads the graph; not timed
     stream.synchronize()
+    launches = graph_kernel_count(graph)
+    per_apply = (launches / (args.steps * n_proj)) if launches else None
+    kernel_desc = ("mlora_apply: lora_decode_kernel" if per_apply == 1 else
+                   "mlora_apply: lora_decode_kernel + long_shrink_kernel + long_expand_kernel"
+                   if per_apply == 3 else "mlora_apply")
 
     dist = None
     if world > 1:
@@ -317,21 +363,17 @@ def run_ours(args, rank: int, world: int, device_index: int):
         clocks = clk.summary(t0, t1)
         clocks["remeasured"] = True
 
-    ms_max = ms
-    if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dev)
     del graph
 
     # end to end through the public API with host buffers: host grouping, H2D of the
     # metadata, X and Y0 from pinned memory, mlora_apply, D2H of Y
-    e2e = run_e2e(args, W, projs, meta, sets[0], dev, stream)
+    e2e = run_e2e(args, W, projs, meta, sets[0], dev, stream, world)
 
     tokens = facts["adapter_rows"]
     steps = args.steps
     sec = ms_max / 1e3
-    value = tokens * steps * world / sec
+    value = whole_job_rate(tokens, steps, world, sec)
     per_launch_s = (ms / 1e3) / steps
     peaks = measured_peaks()
     achieved = facts["bytes"] / per_launch_s / 1e9
@@ -357,10 +399,10 @@ def run_ours(args, rank: int, world: int, device_index: int):
             "peak_source": peaks["source"], "algorithmic_bytes_per_step": facts["bytes"],
             "flops_per_step": facts["flops"],
             "tensor_frac": facts["flops"] / per_launch_s / 1e12 / peaks["bf16_tflops"],
-            "kernel": "lora_tile_kernel (fused apply)",
+            "kernel": kernel_desc,
         },
         "e2e": e2e,
-        "gpu_launches": steps * n_proj,
+        "gpu_launches": launches,
         "clocks": clocks,
         "parity": {"rows_checked": int(rows.size), "max_err_over_tolerance": worst},
     }
@@ -374,7 +416,7 @@ def run_ours(args, rank: int, world: int, device_index: int):
     return result
 
 
-def run_e2e(args, W, projs, meta0, entries, dev, stream):
+def run_e2e(args, W, projs, meta0, entries, dev, stream, world: int = 1):
     import torch
     import segmented_rank_gemm_02_b200 as mlora
 
@@ -430,6 +472,7 @@ def run_e2e(args, W, projs, meta0, entries, dev, stream):
     torch.cuda.synchronize()
     est = time.perf_counter() - t
     steps = int(max(3, min(args.steps, args.e2e_seconds / max(est, 1e-6))))
+    steps = int(max_over_ranks(steps, dev))   # the same count on every rank
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
@@ -440,10 +483,13 @@ def run_e2e(args, W, projs, meta0, entries, dev, stream):
         end.record(stream)
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
+    # every rank ran the same number of steps (the count is agreed on first)
     tokens = int((W.row_slot >= 0).sum())
+    ms = max_over_ranks(ms, dev)
     h2d = meta_host[0].numel() * 4 + sum(x.numel() * 2 + y.numel() * 2 for x, y in zip(Xh, Y0h))
     d2h = sum(y.numel() * 2 for y in Yout)
-    return {"value": tokens * steps / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+    return {"value": whole_job_rate(tokens, steps, world, ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": ms / steps,
             "includes": "host grouping (mlora_build_segments), H2D metadata+X+Y0 from pinned "
                         "memory, mlora_apply, D2H Y"}

@@ -61,6 +61,12 @@ struct TileParams {
     // segments with at least this many grouped positions go to the long-segment
     // (tensor-memory) kernels; the others to the decode-shaped kernel
     int32_t long_rows;
+    // decode-shaped kernel launched with programmatic dependent launch: its CTAs may
+    // start while the previous kernel finishes, prefetch their first tile's adapter
+    // slices into L2 and wait for that kernel before reading anything else.  Used
+    // only for batches without long segments (the long-segment kernels want the
+    // opposite shared-memory / L1 split and stream enough to evict the prefetch).
+    int32_t early;
     // long-segment kernels: H of the long tiles, [n_tokens][ws_ld] fp32 (the pool's
     // workspace in the fused apply, the caller's H in standalone shrink / expand)
     float *ws;

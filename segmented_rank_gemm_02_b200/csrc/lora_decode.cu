@@ -35,6 +35,13 @@
 // hi + lo parts and both are multiplied on the tensor cores, so H enters the
 // product with about 2^-17 relative error instead of bf16's 2^-9.
 //
+// Back-to-back launches.  For batches without long segments the kernel is launched
+// with programmatic dependent launch: its CTAs may start while the previous kernel
+// in the stream finishes, bring their first tile's adapter slices into L2 from a
+// speculative read of the metadata (adapter weights only change through
+// load_slot), and wait (griddepcontrol.wait) before reading the metadata, X or Y
+// for real.  A stale guess costs bandwidth, never correctness.
+//
 // Invalid metadata never traps: bad segments and rows are skipped and flagged in
 // the status word; every CTA of a cluster reaches the same decisions, so cluster
 // barriers always match.  The kernel has no spin-waits.
@@ -114,6 +121,9 @@ __device__ __forceinline__ uint2 ldg_nc2(const void *p)
 
 // Block-wide scan of per-segment tile counts.  Returns the number of tiles; if
 // tile `want` exists, its segment and first position are left in ctl.tile.
+// SPEC: a speculative pass made before the grids this launch depends on have
+// finished (the metadata may still change): relaxed loads, nothing reported.
+template <bool SPEC = false>
 __device__ int scan_tiles(const TileParams &p, int want, SharedCtl &ctl, bool reporter)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -125,11 +135,19 @@ __device__ int scan_tiles(const TileParams &p, int want, SharedCtl &ctl, bool re
         int cnt = 0, p0 = 0, p1 = 0, a = -1, rk = -1;
         float sc = 0.f;
         if (g < p.n_segments) {
-            a = p.slots[g];
-            p0 = p.offsets[g];
-            p1 = p.offsets[g + 1];
-            if (p.ranks) rk = p.ranks[g];
-            if (p.scales) sc = p.scales[g];
+            if constexpr (SPEC) {
+                a = ld_relaxed_s32(p.slots + g);
+                p0 = ld_relaxed_s32(p.offsets + g);
+                p1 = ld_relaxed_s32(p.offsets + g + 1);
+                if (p.ranks) rk = ld_relaxed_s32(p.ranks + g);
+                reporter = false;
+            } else {
+                a = p.slots[g];
+                p0 = p.offsets[g];
+                p1 = p.offsets[g + 1];
+                if (p.ranks) rk = p.ranks[g];
+                if (p.scales) sc = p.scales[g];
+            }
             if (a != -1) {
                 if (a < -1 || a >= p.n_slots) {
                     if (reporter) report(p, kFlagBadSlot);
@@ -279,6 +297,47 @@ __device__ __forceinline__ void mma_expand_store(const ExpandOps<R> &o, const ui
 // One tile, specialised for rank bucket R.  Loads are issued as early as their
 // addresses are known: adapter blocks right away, rows once their indices land,
 // the expand's operands before the cluster reduction.
+// Speculative L2 prefetch of this CTA's share of its first tile's adapter (A slice
+// and B slice), made before the launch's dependencies have finished: adapter
+// weights do not change between loads, so their fetch overlaps the end of the
+// previous kernel.  The metadata read here may be stale; a wrong guess only costs
+// bandwidth (every address stays inside the pool), never correctness, since the
+// tile's real loads come after griddep_wait.
+template <int RMAX, int MODE>
+__device__ void prefetch_first_tile(const TileParams &p, int want, SharedCtl &ctl, uint32_t crank)
+{
+    if (want >= scan_tiles<true>(p, want, ctl, false)) return;
+    const int tid = threadIdx.x;
+    const int slot = ctl.tile[3];
+    if (slot < 0 || slot >= p.n_slots) return;
+    int R = rank_bucket(ctl.tile[4]);
+    if (p.ranks == nullptr || R == 0 || R > RMAX) R = rank_bucket(ld_relaxed_s32(p.slot_rank + slot));
+    if (R == 0 || R > RMAX) return;
+    const int p0 = ctl.tile[1];
+    if (tid == 32 && p.token_indices != nullptr && p0 >= 0 && p0 < p.n_tokens)
+        prefetch_l2_line(p.token_indices + p0);
+    const char *slotA = reinterpret_cast<const char *>(p.pool + (int64_t)slot * p.slot_stride);
+    constexpr uint32_t kChunk = 16384;
+    if (MODE != MODE_EXPAND && tid < 8) {
+        // A block [d_in/8][R][8]: the slice [k_begin, k_end) is one contiguous run
+        const int k0 = min(p.d_in, (int)crank * p.k_slice);
+        const int k1 = min(p.d_in, k0 + p.k_slice);
+        const int64_t beg = (int64_t)k0 * R * 2, len = (int64_t)(k1 - k0) * R * 2;
+        for (int64_t off = (int64_t)tid * kChunk; off < len; off += 8 * kChunk)
+            prefetch_l2_bulk(slotA + beg + off, (uint32_t)(len - off < kChunk ? len - off : kChunk));
+    }
+    if (MODE != MODE_SHRINK && tid >= 64 && tid < 64 + R / 8) {
+        // B block [R/8][d_out][8]: rows [n_begin, n_end) of rank group j, contiguous
+        const int j = tid - 64;
+        const int n0 = min(p.d_out, (int)crank * p.n_slice);
+        const int n1 = min(p.d_out, n0 + p.n_slice);
+        const char *b = slotA + (p.b_offset + ((int64_t)j * p.d_out + n0) * 8) * 2;
+        const int64_t len = (int64_t)(n1 - n0) * 16;
+        for (int64_t off = 0; off < len; off += kChunk)
+            prefetch_l2_bulk(b + off, (uint32_t)(len - off < kChunk ? len - off : kChunk));
+    }
+}
+
 template <int RMAX, int MODE, int R>
 __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float seg_scale,
                          SharedCtl &ctl, float *smem_f, uint32_t crank, uint32_t csize)
@@ -481,6 +540,10 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<RMAX>::MIN_BLOCKS)
     const bool reporter = blockIdx.x == 0;
 
     int tile = (int)cluster_index();
+    // the next launch may start its CTAs now (they wait before touching our results)
+    griddep_launch_dependents();
+    if (p.early) prefetch_first_tile<RMAX, MODE>(p, tile, ctl, crank);
+    griddep_wait();
     const int total = scan_tiles(p, tile, ctl, reporter);
     for (; tile < total; tile += n_clusters) {
         if (tile != (int)cluster_index()) scan_tiles(p, tile, ctl, false);
@@ -524,11 +587,15 @@ cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, cuda
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = DecodeCfg<RMAX>::SMEM;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // programmatic dependent launch: CTAs may start while the previous kernel in the
+    // stream finishes; the kernel waits (griddepcontrol.wait) before reading inputs
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
 
@@ -552,6 +619,7 @@ cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, cuda
     }
     const int64_t n = max_tiles < active ? max_tiles : active;
     cfg.gridDim = dim3((unsigned)(n * cluster), 1, 1);
+    cfg.numAttrs = p.early ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, lora_decode_kernel<RMAX, MODE>, p);
 }
 
@@ -567,6 +635,9 @@ cudaError_t launch_rmax(int mode, const TileParams &p, int cluster, int64_t max_
     }
 }
 
+// The shared-memory carveout is left to the driver: a preference for more L1
+// starves the kernel of resident CTAs, one for more shared memory shrinks the L1
+// through which its register operands stream (both measured slower).
 template <int RMAX>
 cudaError_t set_attrs()
 {

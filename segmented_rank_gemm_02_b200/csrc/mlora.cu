@@ -202,6 +202,7 @@ mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::
                           (s->max_segment_rows <= 0 || s->max_segment_rows >= kLongRows) &&
                           tensor_map_encoder() != nullptr;
     p.long_rows = use_long ? kLongRows : 0x7fffffff;
+    p.early = use_long ? 0 : 1;
     mlora_status st = prepare_device(pool->device);
     if (st != MLORA_OK) return st;
 

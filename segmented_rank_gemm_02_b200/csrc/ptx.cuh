@@ -415,4 +415,43 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_byte_addr)
     return d;
 }
 
+// ---- programmatic dependent launch and L2 prefetch
+
+// Wait until the grids this launch depends on have completed and their memory
+// operations are visible (returns at once when the launch has no such dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next launch in the stream (if it opted in) to start its CTAs now; they
+// still wait for this grid's completion before touching its results.
+__device__ __forceinline__ void griddep_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Relaxed gpu-scope loads: no L1 allocation, no data race with a concurrent writer.
+__device__ __forceinline__ int ld_relaxed_s32(const int32_t *p)
+{
+    int v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ float ld_relaxed_f32(const float *p)
+{
+    float v;
+    asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Bring [p, p + bytes) into L2 (p 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void prefetch_l2_line(const void *p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
+}
+
 }  // namespace mlora
