@@ -319,14 +319,15 @@ def run_ours(args, rank: int, world: int, device_index: int):
         for k in range(args.warmup):
             step(k)
     stream.synchronize()
-    graph = torch.cuda.CUDAGraph()
+    graph = torch.cuda.CUDAGraph(keep_graph=True)   # kept so its kernel nodes can be counted
     with torch.cuda.graph(graph, stream=stream):
         for k in range(args.steps):
             step(k)
+    launches = graph_kernel_count(graph)
+    graph.instantiate()
     with torch.cuda.stream(stream):
         graph.replay()   # first replay uploads the graph; not timed
     stream.synchronize()
-    launches = graph_kernel_count(graph)
     per_apply = (launches / (args.steps * n_proj)) if launches else None
     kernel_desc = ("mlora_apply: lora_decode_kernel" if per_apply == 1 else
                    "mlora_apply: lora_decode_kernel + long_shrink_kernel + long_expand_kernel"

@@ -73,7 +73,6 @@ struct TileParams {
     int64_t ws_ld;
     int32_t ksplit;            // CTAs per shrink cluster, each one part of d_in
     int32_t k_part;            // d_in columns per part (multiple of 64)
-    int32_t n_unit;            // d_out columns per expand work unit (multiple of 128)
     // TMA views (bf16, 128-byte swizzle) of X [n_rows, d_in] and Y [n_rows, d_out]:
     // 64 x 128 tiles for runs of consecutive rows, 64 x 1 rows for gathers
     CUtensorMap x_tile, x_rows, y_tile, y_rows;
@@ -81,14 +80,12 @@ struct TileParams {
 
 // Rows per tile of the long-segment kernels (one M=128 tensor-memory tile).
 constexpr int kLongTileRows = 128;
-// Long-segment kernels: number of d_out ranges of n_unit columns.
-__host__ __device__ inline int n_ranges(const TileParams &p) { return (p.d_out + p.n_unit - 1) / p.n_unit; }
 
 // Long-segment shrink (H of the long tiles into p.ws) and expand (reads p.ws; in
 // MODE_EXPAND it also reports the tiles' metadata problems); persistent grids.
 cudaError_t launch_long_shrink(int rmax_bucket, const TileParams &p, int64_t max_tiles,
                                cudaStream_t stream);
-cudaError_t launch_long_expand(int rmax_bucket, int mode, const TileParams &p, int64_t max_units,
+cudaError_t launch_long_expand(int rmax_bucket, int mode, const TileParams &p, int64_t max_tiles,
                                cudaStream_t stream);
 cudaError_t prepare_long_kernels();
 

@@ -18,13 +18,16 @@
 // accumulator with tcgen05.ld; the cluster sums its partial tiles through
 // distributed shared memory in a fixed order and writes H (fp32) once.
 //
-// Expand (long_expand_kernel).  Work unit = (tile, range of d_out).  The tile's H is
-// written once to shared memory as bf16 hi + lo parts (no-swizzle K-major); then per
-// 128-column chunk -- three buffers, two chunks in flight -- one thread issues the
-// bulk copies of the adapter's B rows and the TMA loads (tile or gathers) of the Y0
-// rows, then tcgen05.mma accumulates H_hi B^T + H_lo B^T (M=128, N=128) in tensor
-// memory; the epilogue adds s * acc to Y0 in shared memory and all threads store
-// whole rows with coalesced 16-byte stores.
+// Expand (long_expand_kernel).  Warp-specialised and persistent: the (tile,
+// 128-column chunk) pairs of all long tiles are cut into one contiguous range per
+// CTA.  A producer warp streams each chunk's B rows (bulk copies) and Y0 rows (TMA
+// tile, or four-row gathers) into a ring of stages; an MMA warp multiplies
+// H_hi B^T + H_lo B^T (M=128, N=128) into one of two fp32 accumulators in tensor
+// memory; eight epilogue warps (two threads per row) add s * acc to Y0 in shared
+// memory and write the rows back -- one TMA tile store for a full tile of
+// consecutive rows, coalesced 16-byte stores otherwise -- and stage the next
+// unit's H as bf16 hi + lo parts (two buffers) ahead of its chunks.  The roles
+// meet only at mbarriers, so copies, tensor-core work and epilogue overlap.
 //
 // Rank buckets: kernels are compiled for the pool's largest bucket and dispatch each
 // tile to code for its own bucket (bucket 8 runs as 16; its missing operand half is
@@ -46,8 +49,8 @@ constexpr int KB = 64;                // d_in columns per shrink block (one 128-
 constexpr int NCH = 128;              // d_out columns per expand chunk
 constexpr int NS = 6;                 // shrink pipeline stages
 constexpr int PD = 4;                 // shrink prefetch distance (blocks ahead of the MMA)
-constexpr int NB = 3;                 // expand chunk buffers
-constexpr int ED = 2;                 // expand prefetch distance (chunks ahead)
+constexpr int kMaxExpandStages = 6;  // expand chunk ring, as deep as shared memory allows
+constexpr int kExpandSmemCap = 224 * 1024;   // dynamic shared memory of one expand CTA
 constexpr int kMaxSplit = 8;          // CTAs per shrink cluster
 constexpr int kZeroBytes = 2048;      // zero operand half for rank bucket 8
 constexpr uint64_t kWaitNs = 1000000000ull;
@@ -67,9 +70,13 @@ struct LongCfg {
     static constexpr int H_BYTES = PM * RK * 2;          // one of hi / lo: [RK/8][16][8][8]
     static constexpr int B_BYTES = (NCH * RK * 2 + 1023) / 1024 * 1024;  // [RK/8][128][8]
     static constexpr int Y_BYTES = PM * NCH * 2;         // two 64-column halves, swizzled
-    static constexpr int CHUNK_BYTES = B_BYTES + Y_BYTES;
-    static constexpr int E_SMEM = 1024 + NB * CHUNK_BYTES + 2 * H_BYTES + kZeroBytes;
-    static constexpr int E_TMEM = NCH;
+    static constexpr int E_STAGE = B_BYTES + Y_BYTES;    // one 128-column chunk
+    static constexpr int E_FIXED = 1024 + 2 * 2 * H_BYTES + kZeroBytes;   // + H hi/lo x 2
+    static constexpr int E_NB_FIT = (kExpandSmemCap - E_FIXED) / E_STAGE;
+    static constexpr int E_NB = E_NB_FIT < kMaxExpandStages ? E_NB_FIT : kMaxExpandStages;
+    static_assert(E_NB >= 2, "expand stage ring");
+    static constexpr int E_SMEM = E_FIXED + E_NB * E_STAGE;
+    static constexpr int E_TMEM = 2 * NCH;               // two accumulators
 };
 
 struct LongCtl {
@@ -418,208 +425,447 @@ __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__
 }
 
 // ------------------------------------------------------------------ expand
-template <int RMAX, int MODE, int R>
-__device__ void expand_unit(const TileParams &p, LongCtl &ctl, uint8_t *bufs, uint8_t *hbuf,
-                            uint8_t *zero, uint32_t tmem, uint32_t &cg, int n_lo, int n_hi,
-                            int nvalid, int rank, bool ok, float scale)
+// Warp roles.  Warp 0 copies (one lane issues the B-row bulk copies and Y0 tile
+// loads; every lane issues its own four-row gathers), warp 1 owns tensor memory and
+// issues the tensor-core work, warps 2..9 stage H and run the epilogue (two threads
+// per tile row, one 64-column half each).  The roles meet only at mbarriers:
+//   full[s] / empty[s]      stage ring (B rows + Y0 rows of one 128-column chunk)
+//   acc_full[a] / acc_empty[a]  two fp32 accumulators of 128 columns in tensor memory
+//   h_full[b] / h_empty[b]  two H buffers (hi + lo), one per work unit in flight
+constexpr int E_WARPS = 10;
+constexpr int ET = E_WARPS * 32;     // threads per expand CTA
+constexpr int E_EPI = 256;           // epilogue threads (warps 2..9)
+constexpr int kEpiBar = 1;           // named barrier of the epilogue warps
+constexpr int kMaxUnits = 64;        // work units per CTA (the host sizes the grid)
+
+struct ExpUnit {
+    int p0, p1;        // first grouped position of the tile, end of its segment
+    int slot, r_meta;  // slot and rank from the metadata (-1 if none)
+    float seg_scale;   // scale from the metadata
+    int c_begin, c_end;   // 128-column chunks [c_begin, c_end) of d_out
+};
+
+struct ExpCtl {
+    uint64_t full[kMaxExpandStages], empty[kMaxExpandStages];
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t h_full[2], h_empty[2];
+    uint32_t tmem;
+    volatile int fail;
+    int scan[E_WARPS];
+    int rows[2][PM];   // original row of each tile position (epilogue), -1 = none
+    int full_tile[2];  // the unit's tile is 128 consecutive rows
+    ExpUnit unit[kMaxUnits];
+};
+
+// Rank and scale of a unit's slot; every role derives the same values.
+struct UnitInfo {
+    int nvalid, R, rank, ok, n_lo, n_hi, nch;
+    float scale;
+};
+
+__device__ __forceinline__ UnitInfo unit_info(const TileParams &p, const ExpUnit &u)
 {
-    using C = LongCfg<RMAX>;
-    constexpr int RK = padded_rank(R);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int row = tid % PM, half = tid / PM;   // two threads per row
-    const int p0 = ctl.tile[1], slot = ctl.tile[3];
-    const __nv_bfloat16 *slotB = p.pool + (int64_t)slot * p.slot_stride + p.b_offset;
-    uint8_t *ahi = hbuf;
-    uint8_t *alo = hbuf + C::H_BYTES;
-    const bool hrow = ok && row < nvalid;
+    UnitInfo i;
+    i.nvalid = min(PM, u.p1 - u.p0);
+    const int r = p.slot_rank[u.slot];
+    i.ok = r > 0 && (p.ranks == nullptr || u.r_meta == r) && rank_bucket(r) != 0;
+    i.rank = i.ok ? r : 0;
+    i.R = i.ok ? rank_bucket(r) : 8;
+    i.scale = p.scales ? u.seg_scale : p.slot_scale[u.slot];
+    i.n_lo = u.c_begin * NCH;
+    i.n_hi = min(p.d_out, u.c_end * NCH);
+    i.nch = u.c_end - u.c_begin;
+    return i;
+}
 
-    // this thread's half of its H row as bf16 hi + lo, canonical no-swizzle K-major layout
-    {
-        constexpr int HC = RK / 2;
-        const float *hsrc = p.ws + (int64_t)(p0 + (hrow ? row : 0)) * p.ws_ld + half * HC;
-        float h[HC];
-#pragma unroll
-        for (int j = 0; j < HC; ++j) h[j] = (hrow && half * HC + j < rank) ? hsrc[j] : 0.f;
-#pragma unroll
-        for (int jg = 0; jg < HC / 8; ++jg) {
-            uint4 hi, lo;
-            uint32_t *ph = reinterpret_cast<uint32_t *>(&hi);
-            uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float h0, l0, h1, l1;
-                split_bf16(h[8 * jg + 2 * c], h0, l0);
-                split_bf16(h[8 * jg + 2 * c + 1], h1, l1);
-                ph[c] = pack_bf16x2(h0, h1);
-                pl[c] = pack_bf16x2(l0, l1);
-            }
-            const int j = half * (HC / 8) + jg;
-            const int off = (j * (PM / 8) + row / 8) * 128 + (row % 8) * 16;
-            *reinterpret_cast<uint4 *>(ahi + off) = hi;
-            *reinterpret_cast<uint4 *>(alo + off) = lo;
-        }
+__device__ __forceinline__ bool exp_wait(const TileParams &p, ExpCtl &ctl, uint64_t *bar, uint32_t parity)
+{
+    if (ctl.fail) return false;
+    if (!mbar_wait_bounded(bar, parity, kWaitNs)) {
+        ctl.fail = 1;
+        report(p, kFlagTimeout);
+        return false;
     }
-    fence_proxy_async_smem();   // the H tile is read by the tensor core
-    __syncthreads();
+    return true;
+}
 
-    const int nch = (n_hi - n_lo + NCH - 1) / NCH;
-    const bool load_y = ok && !ctl.fail;
-    // chunk ci of this unit uses buffer (cg + ci) % NB; cg counts chunks across units
-    auto issue = [&](int ci) {   // thread 0
-        const uint32_t G = cg + ci;
-        uint8_t *buf = bufs + (G % NB) * C::CHUNK_BYTES;
-        uint8_t *bs = buf;
-        uint8_t *ys = buf + C::B_BYTES;
-        const int c0 = n_lo + ci * NCH;
-        const int len = min(NCH, n_hi - c0);
-        uint32_t bytes = (uint32_t)(R / 8) * len * 16;
-        if (load_y) bytes += (len > 64 ? 2 : 1) * PM * 64 * 2;
-        mbar_arrive_expect_tx(&ctl.full[G % NB], bytes);
-        for (int j = 0; j < R / 8; ++j)   // B rows c0.., rank group j: len x 16 bytes
-            bulk_load(bs + j * NCH * 16, slotB + ((int64_t)j * p.d_out + c0) * 8, len * 16, &ctl.full[G % NB]);
-        if (load_y) {
-            load_rows(ctl, &p.y_tile, &p.y_rows, p.n_rows, ys, c0, &ctl.full[G % NB]);
-            if (len > 64) load_rows(ctl, &p.y_tile, &p.y_rows, p.n_rows, ys + PM * 128, c0 + 64, &ctl.full[G % NB]);
-        }
-    };
-    if (tid == 0)
-        for (int q = 0; q < ED && q < nch; ++q) issue(q);
-
-    const uint32_t idesc = umma_idesc_bf16(PM, NCH);
-    // epilogue geometry: warp w computes rows 32 (w % 4) .. and columns [64 (w / 4), +64)
-    // (= swizzled half w / 4) into the staged Y0 rows; then all threads store whole rows
-    const int erow = 32 * (warp % 4) + (tid & 31);
-    const bool compute = ok && erow < nvalid && ctl.rows[erow] >= 0;
-    const int ehalf = warp / 4;
-    for (int ci = 0; ci < nch; ++ci) {
-        const uint32_t G = cg + ci;
-        const int c0 = n_lo + ci * NCH;
-        const int len = min(NCH, n_hi - c0);
-        uint8_t *buf = bufs + (G % NB) * C::CHUNK_BYTES;
-        uint8_t *ys = buf + C::B_BYTES;
-        if (tid == 0) {
-            if (ci + ED < nch) issue(ci + ED);
-            if (wait_or_fail(p, ctl, &ctl.full[G % NB], (G / NB) & 1u)) {
-                tc_fence_after();
-                const uint32_t a_hi = smem_addr(ahi), a_lo = smem_addr(alo), b_s = smem_addr(buf);
-#pragma unroll
-                for (int st = 0; st < RK / 16; ++st) {
-                    const uint32_t koff = st * 2 * (PM / 8) * 128;
-                    const uint32_t b0 = b_s + st * 2 * NCH * 16;
-                    // bucket 8: the second rank group of B is the zero block
-                    const uint32_t lbo = (R == 8) ? smem_addr(zero) - b0 : NCH * 16;
-                    const uint64_t bd = umma_desc_kmajor(b0, lbo, 128);
-                    umma_bf16(tmem, umma_desc_kmajor(a_hi + koff, (PM / 8) * 128, 128), bd, idesc,
-                              st > 0 ? 1u : 0u);
-                    umma_bf16(tmem, umma_desc_kmajor(a_lo + koff, (PM / 8) * 128, 128), bd, idesc, 1u);
-                }
-                umma_commit(&ctl.bar[0]);
+// Work split.  The (tile, 128-column chunk) pairs of all long tiles, tile-major, are
+// cut into gridDim.x equal contiguous ranges; CTA b takes range b.  A unit is the run
+// of one tile's chunks inside the range, so a CTA stages H once per tile it touches.
+//
+// Pass over the segments: with want_lo < 0 it only counts the long tiles; otherwise it
+// also fills ctl.unit[t - want_lo] for every tile t in [want_lo, want_hi].
+__device__ int scan_units(const TileParams &p, ExpCtl &ctl, int want_lo, int want_hi)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int running = 0;
+    for (int base = 0; base < p.n_segments; base += ET) {
+        const int g = base + tid;
+        int cnt = 0, p0 = 0, p1 = 0, a = -1, rk = -1;
+        float sc = 0.f;
+        if (g < p.n_segments) {
+            a = p.slots[g];
+            p0 = p.offsets[g];
+            p1 = p.offsets[g + 1];
+            if (want_lo >= 0) {
+                if (p.ranks) rk = p.ranks[g];
+                if (p.scales) sc = p.scales[g];
             }
+            if (a >= 0 && a < p.n_slots && p0 >= 0 && p1 >= p0 && p1 <= p.n_tokens &&
+                p1 - p0 >= p.long_rows)
+                cnt = (p1 - p0 + PM - 1) / PM;
         }
-        wait_or_fail(p, ctl, &ctl.bar[0], G & 1u);
-        tc_fence_after();
-        const uint32_t taddr = tmem + ((uint32_t)(32 * (warp % 4)) << 16) + 64 * ehalf;
-        uint8_t *yh = ys + ehalf * PM * 128 + erow * 128;   // this row of this half, swizzled
+        int incl = cnt;
 #pragma unroll
-        for (int cb = 0; cb < 64; cb += 32) {
-            if (64 * ehalf + cb >= len) break;
-            uint32_t v[32];
-            tmem_ld32(taddr + cb, v);
-            tmem_wait_ld();
-            if (compute) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int chunk = cb / 8 + q;                      // 16-byte chunk in the row
-                    uint4 *yp = reinterpret_cast<uint4 *>(yh + ((chunk ^ (erow & 7)) * 16));
-                    const uint4 y0 = *yp;
-                    const __nv_bfloat162 *y2 = reinterpret_cast<const __nv_bfloat162 *>(&y0);
-                    uint4 out;
-                    uint32_t *o = reinterpret_cast<uint32_t *>(&out);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(y2[e]);
-                        o[e] = pack_bf16x2(fmaf(scale, __uint_as_float(v[8 * q + 2 * e]), f.x),
-                                           fmaf(scale, __uint_as_float(v[8 * q + 2 * e + 1]), f.y));
-                    }
-                    *yp = out;
-                }
-            }
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
         }
-        tc_fence_before();
+        if (lane == 31) ctl.scan[warp] = incl;
         __syncthreads();
-        // coalesced stores: sixteen lanes per row, 16 bytes each
+        int before = 0, total = 0;
 #pragma unroll
-        for (int k = 0; k < (PM * NCH / 8) / PT; ++k) {
-            const int i = tid + k * PT;
-            const int r = i / (NCH / 8), q = i % (NCH / 8);
-            const int tr = ctl.rows[r];
-            if (ok && !ctl.fail && r < nvalid && tr >= 0 && 8 * q < len) {
-                const uint8_t *src = ys + (q / 8) * PM * 128 + r * 128 + (((q % 8) ^ (r & 7)) * 16);
-                *reinterpret_cast<uint4 *>(p.Y + (int64_t)tr * p.ldy + c0 + 8 * q) =
-                    *reinterpret_cast<const uint4 *>(src);
+        for (int w = 0; w < E_WARPS; ++w) {
+            const int v = ctl.scan[w];
+            before += (w < warp) ? v : 0;
+            total += v;
+        }
+        if (want_lo >= 0 && cnt > 0) {
+            const int lo = running + before + incl - cnt;   // this segment's first tile
+            const int t0 = max(lo, want_lo), t1 = min(lo + cnt - 1, want_hi);
+            for (int t = t0; t <= t1; ++t) {
+                ExpUnit &e = ctl.unit[t - want_lo];
+                e.p0 = p0 + (t - lo) * PM;
+                e.p1 = p1;
+                e.slot = a;
+                e.r_meta = rk;
+                e.seg_scale = sc;
             }
         }
-        fence_proxy_async_smem();   // this buffer is next written by TMA
+        running += total;
         __syncthreads();
     }
-    cg += nch;
+    return running;
 }
 
 template <int RMAX, int MODE>
-__global__ void __launch_bounds__(PT) long_expand_kernel(const __grid_constant__ TileParams p)
+__global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constant__ TileParams p)
 {
     using C = LongCfg<RMAX>;
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    __shared__ LongCtl ctl;
-    uint8_t *bufs = align1024(smem_raw);
-    uint8_t *hbuf = bufs + NB * C::CHUNK_BYTES;
-    uint8_t *zero = hbuf + 2 * C::H_BYTES;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    if (warp == 0) {
+    __shared__ ExpCtl ctl;
+    uint8_t *stages = align1024(smem_raw);
+    uint8_t *hbufs = stages + C::E_NB * C::E_STAGE;   // [2][hi, lo]
+    uint8_t *zero = hbufs + 2 * 2 * C::H_BYTES;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (warp == 1) {
         tmem_alloc(&ctl.tmem, C::E_TMEM);
         tmem_relinquish();
     }
-    for (int i = tid; i < kZeroBytes / 16; i += PT) reinterpret_cast<uint4 *>(zero)[i] = make_uint4(0, 0, 0, 0);
+    for (int i = tid; i < kZeroBytes / 16; i += ET) reinterpret_cast<uint4 *>(zero)[i] = make_uint4(0, 0, 0, 0);
     if (tid == 0) {
-        mbar_init(&ctl.bar[0], 1);
-#pragma unroll
-        for (int b = 0; b < NB; ++b) mbar_init(&ctl.full[b], 1);
+        for (int s = 0; s < C::E_NB; ++s) {
+            mbar_init(&ctl.full[s], 1);
+            mbar_init(&ctl.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl.acc_full[b], 1);
+            mbar_init(&ctl.acc_empty[b], E_EPI / 32);
+            mbar_init(&ctl.h_full[b], 1);
+            mbar_init(&ctl.h_empty[b], 1);
+        }
         fence_mbar_init();
         ctl.fail = 0;
+    }
+    // this CTA's share of the (tile, chunk) pairs
+    const int cpt = (p.d_out + NCH - 1) / NCH;   // chunks per tile
+    const int ntiles = scan_units(p, ctl, -1, -1);
+    const int64_t total = (int64_t)ntiles * cpt;
+    const int64_t lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
+    int n_my = 0;
+    if (hi > lo) {
+        const int t_lo = (int)(lo / cpt), t_hi = (int)((hi - 1) / cpt);
+        n_my = t_hi - t_lo + 1;
+        if (n_my > kMaxUnits) {   // the host sizes the grid so that this never happens
+            if (tid == 0) report(p, kFlagTimeout);
+            n_my = 0;
+        } else {
+            scan_units(p, ctl, t_lo, t_hi);
+            for (int k = tid; k < n_my; k += ET) {
+                const int64_t t = t_lo + k;
+                ctl.unit[k].c_begin = (int)((lo > t * cpt ? lo : t * cpt) - t * cpt);
+                ctl.unit[k].c_end = (int)((hi < (t + 1) * cpt ? hi : (t + 1) * cpt) - t * cpt);
+            }
+        }
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl.tmem;
-    uint32_t cg = 0;   // chunks multiplied so far (buffer and barrier phases)
-    const int nr = n_ranges(p);
-    for (int unit = blockIdx.x;; unit += gridDim.x) {
-        const int tile = unit / nr, range = unit % nr;
-        const int ntiles = scan_long(p, tile, ctl);
-        if (tile >= ntiles || ctl.fail) break;
-        const int nvalid = min(PM, ctl.tile[2] - ctl.tile[1]);
-        bool ok;
-        int rank;
-        // in the fused apply the shrink kernel reported this tile's metadata problems
-        const int R = tile_setup(p, ctl, nvalid, MODE == MODE_EXPAND && range == 0, ok, rank);
-        const float scale = p.scales ? ctl.seg_scale : ctl.slot_scale;
-        const int n_lo = range * p.n_unit, n_hi = min(p.d_out, n_lo + p.n_unit);
-        if (R == 8) {
-            expand_unit<RMAX, MODE, 8>(p, ctl, bufs, hbuf, zero, tmem, cg, n_lo, n_hi, nvalid, rank, ok, scale);
-        } else if (R == 16) {
-            expand_unit<RMAX, MODE, 16>(p, ctl, bufs, hbuf, zero, tmem, cg, n_lo, n_hi, nvalid, rank, ok, scale);
-        } else if (R == 32) {
-            if constexpr (RMAX >= 32)
-                expand_unit<RMAX, MODE, 32>(p, ctl, bufs, hbuf, zero, tmem, cg, n_lo, n_hi, nvalid, rank, ok, scale);
-        } else if (R == 64) {
-            if constexpr (RMAX >= 64)
-                expand_unit<RMAX, MODE, 64>(p, ctl, bufs, hbuf, zero, tmem, cg, n_lo, n_hi, nvalid, rank, ok, scale);
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- copies
+        uint32_t g = 0;
+        for (int k = 0; k < n_my; ++k) {
+            if (__shfl_sync(0xffffffffu, ctl.fail, 0)) break;
+            const ExpUnit u = ctl.unit[k];
+            const UnitInfo ui = unit_info(p, u);
+            // this lane's four rows of the tile: gathers and the contiguity test
+            int t[4];
+            bool mine = true;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int i = 4 * lane + q;
+                t[q] = -1;
+                if (i < ui.nvalid) {
+                    const int v = p.token_indices ? p.token_indices[u.p0 + i] : u.p0 + i;
+                    t[q] = (v >= 0 && v < p.n_rows) ? v : -1;
+                }
+            }
+            const int row0 = __shfl_sync(0xffffffffu, t[0], 0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int i = 4 * lane + q;
+                if (i < ui.nvalid) mine = mine && t[q] >= 0 && t[q] == row0 + i;
+            }
+            const bool contiguous = __all_sync(0xffffffffu, mine);
+            const __nv_bfloat16 *slotB = p.pool + (int64_t)u.slot * p.slot_stride + p.b_offset;
+            for (int ci = 0; ci < ui.nch; ++ci, ++g) {
+                const int s = (int)(g % C::E_NB);
+                bool go = true;
+                if (lane == 0 && g >= (uint32_t)C::E_NB)
+                    go = exp_wait(p, ctl, &ctl.empty[s], ((g / C::E_NB) - 1) & 1u);
+                go = __shfl_sync(0xffffffffu, go ? 1 : 0, 0) != 0;
+                if (!go) break;
+                uint8_t *bs = stages + s * C::E_STAGE;
+                uint8_t *ys = bs + C::B_BYTES;
+                const int c0 = ui.n_lo + ci * NCH;
+                const int len = min(NCH, ui.n_hi - c0);
+                const int halves = len > 64 ? 2 : 1;
+                if (lane == 0) {
+                    uint32_t bytes = (uint32_t)(ui.R / 8) * len * 16;
+                    if (ui.ok) bytes += (uint32_t)halves * PM * 64 * 2;
+                    mbar_arrive_expect_tx(&ctl.full[s], bytes);
+                    for (int j = 0; j < ui.R / 8; ++j)   // B rows c0.., rank group j
+                        bulk_load(bs + j * NCH * 16, slotB + ((int64_t)j * p.d_out + c0) * 8, len * 16,
+                                  &ctl.full[s]);
+                    if (ui.ok && contiguous)
+                        for (int h = 0; h < halves; ++h)
+                            tma_load_2d(ys + h * PM * 128, &p.y_tile, c0 + 64 * h, row0, &ctl.full[s]);
+                }
+                __syncwarp();
+                if (ui.ok && !contiguous) {
+                    int r[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) r[q] = t[q] >= 0 ? t[q] : p.n_rows;   // absent: zeros
+                    for (int h = 0; h < halves; ++h)
+                        tma_gather4(ys + h * PM * 128 + lane * 4 * 128, &p.y_rows, c0 + 64 * h, r[0], r[1],
+                                    r[2], r[3], &ctl.full[s]);
+                }
+            }
         }
-        __syncthreads();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- tensor core
+        if (lane == 0) {
+            uint32_t g = 0, a = 0;
+            const uint32_t idesc = umma_idesc_bf16(PM, NCH);
+            for (int k = 0; k < n_my && !ctl.fail; ++k) {
+                const UnitInfo ui = unit_info(p, ctl.unit[k]);
+                const int hb = k & 1;
+                if (!exp_wait(p, ctl, &ctl.h_full[hb], (uint32_t)(k >> 1) & 1u)) break;
+                const uint32_t a_hi = smem_addr(hbufs + hb * 2 * C::H_BYTES);
+                const uint32_t a_lo = a_hi + C::H_BYTES;
+                const int RK = padded_rank(ui.R);
+                for (int ci = 0; ci < ui.nch; ++ci, ++g, ++a) {
+                    const int s = (int)(g % C::E_NB);
+                    const int ab = (int)(a & 1);
+                    if (!exp_wait(p, ctl, &ctl.full[s], (g / C::E_NB) & 1u)) break;
+                    if (a >= 2 && !exp_wait(p, ctl, &ctl.acc_empty[ab], ((a >> 1) - 1) & 1u)) break;
+                    tc_fence_after();
+                    const uint32_t b_s = smem_addr(stages + s * C::E_STAGE);
+                    const uint32_t d = tmem + ab * NCH;
+                    for (int st = 0; st < RK / 16; ++st) {
+                        const uint32_t koff = st * 2 * (PM / 8) * 128;
+                        const uint32_t b0 = b_s + st * 2 * NCH * 16;
+                        // bucket 8: the second rank group of B is the zero block
+                        const uint32_t lbo = (ui.R == 8) ? smem_addr(zero) - b0 : NCH * 16;
+                        const uint64_t bd = umma_desc_kmajor(b0, lbo, 128);
+                        umma_bf16(d, umma_desc_kmajor(a_hi + koff, (PM / 8) * 128, 128), bd, idesc,
+                                  st > 0 ? 1u : 0u);
+                        umma_bf16(d, umma_desc_kmajor(a_lo + koff, (PM / 8) * 128, 128), bd, idesc, 1u);
+                    }
+                    umma_commit(&ctl.acc_full[ab]);
+                }
+                umma_commit(&ctl.h_empty[hb]);   // this unit's H buffer is free once its MMAs end
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- H staging + epilogue
+        const int et = tid - 64;
+        const int quarter = warp & 3, half = (warp - 2) >> 2;
+        const int row = 32 * quarter + lane;                 // tensor-memory lane = tile row
+        // Every wait of the epilogue warps ends in a vote, so they all leave together
+        // (a named barrier has no time limit).
+        auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
+            const bool ok = exp_wait(p, ctl, bar, parity);
+            return named_sync_and(kEpiBar, E_EPI, ok);
+        };
+        // Stage unit k: its rows, whether they form one full run, and H as bf16 hi + lo
+        // in buffer k & 1 (free once unit k - 2's tensor-core work has ended).
+        auto stage = [&](int k) -> bool {
+            const ExpUnit u = ctl.unit[k];
+            const UnitInfo ui = unit_info(p, u);
+            const int hb = k & 1;
+            int t = -1;
+            if (row < ui.nvalid) {
+                const int v = p.token_indices ? p.token_indices[u.p0 + row] : u.p0 + row;
+                if (v >= 0 && v < p.n_rows) t = v;
+                else if (MODE == MODE_EXPAND && u.c_begin == 0 && half == 0) report(p, kFlagBadRow);
+            }
+            if (MODE == MODE_EXPAND && u.c_begin == 0 && et == 0 && !ui.ok)
+                report(p, p.slot_rank[u.slot] <= 0 ? kFlagSlotEmpty : kFlagBadRank);
+            if (k >= 2 && !wait_all(&ctl.h_empty[hb], (uint32_t)((k >> 1) - 1) & 1u)) return false;
+            if (half == 0) ctl.rows[hb][row] = t;
+            const int RK = padded_rank(ui.R);
+            const int HC = RK / 2;                            // H columns of this thread
+            const bool hrow = ui.ok && row < ui.nvalid;
+            const float *hsrc = p.ws + (int64_t)(u.p0 + (hrow ? row : 0)) * p.ws_ld + half * HC;
+            uint8_t *ahi = hbufs + hb * 2 * C::H_BYTES;
+            uint8_t *alo = ahi + C::H_BYTES;
+            for (int jg = 0; jg < HC / 8; ++jg) {
+                float h[8];
+                if (hrow && half * HC + 8 * jg + 8 <= ui.rank) {
+                    const float4 v0 = *reinterpret_cast<const float4 *>(hsrc + 8 * jg);
+                    const float4 v1 = *reinterpret_cast<const float4 *>(hsrc + 8 * jg + 4);
+                    h[0] = v0.x; h[1] = v0.y; h[2] = v0.z; h[3] = v0.w;
+                    h[4] = v1.x; h[5] = v1.y; h[6] = v1.z; h[7] = v1.w;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const int col = half * HC + 8 * jg + c;
+                        h[c] = (hrow && col < ui.rank) ? hsrc[8 * jg + c] : 0.f;
+                    }
+                }
+                uint4 hi, lo;
+                uint32_t *ph = reinterpret_cast<uint32_t *>(&hi);
+                uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float h0, l0, h1, l1;
+                    split_bf16(h[2 * c], h0, l0);
+                    split_bf16(h[2 * c + 1], h1, l1);
+                    ph[c] = pack_bf16x2(h0, h1);
+                    pl[c] = pack_bf16x2(l0, l1);
+                }
+                const int j = half * (HC / 8) + jg;
+                const int off = (j * (PM / 8) + row / 8) * 128 + (row % 8) * 16;
+                *reinterpret_cast<uint4 *>(ahi + off) = hi;
+                *reinterpret_cast<uint4 *>(alo + off) = lo;
+            }
+            fence_proxy_async_smem();   // the H tile is read by the tensor core
+            named_sync(kEpiBar, E_EPI);
+            const bool run = named_sync_and(kEpiBar, E_EPI, ui.nvalid == PM && ctl.rows[hb][row] >= 0 &&
+                                                                ctl.rows[hb][row] == ctl.rows[hb][0] + row);
+            if (et == 0) {
+                ctl.full_tile[hb] = run ? 1 : 0;
+                mbar_arrive(&ctl.h_full[hb]);
+            }
+            return true;
+        };
+
+        uint32_t g = 0, a = 0;
+        bool alive = n_my > 0 ? stage(0) : false;
+        for (int k = 0; k < n_my && alive; ++k) {
+            // the next unit's H is staged before this unit's chunks, so the tensor core
+            // never waits for it
+            if (k + 1 < n_my && !stage(k + 1)) break;
+            const ExpUnit u = ctl.unit[k];
+            const UnitInfo ui = unit_info(p, u);
+            const int hb = k & 1;
+            const int row0 = ctl.rows[hb][0];
+            const bool full_tile = ctl.full_tile[hb] != 0;
+            const bool compute = ui.ok && row < ui.nvalid && ctl.rows[hb][row] >= 0;
+
+            for (int ci = 0; ci < ui.nch; ++ci, ++g, ++a) {
+                const int s = (int)(g % C::E_NB);
+                const int ab = (int)(a & 1);
+                const int c0 = ui.n_lo + ci * NCH;
+                const int len = min(NCH, ui.n_hi - c0);
+                uint8_t *ys = stages + s * C::E_STAGE + C::B_BYTES;
+                if (!wait_all(&ctl.acc_full[ab], (a >> 1) & 1u) || !wait_all(&ctl.full[s], (g / C::E_NB) & 1u)) {
+                    alive = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t taddr = tmem + ((uint32_t)(32 * quarter) << 16) + ab * NCH + 64 * half;
+                uint32_t v0[32], v1[32];
+                tmem_ld32(taddr, v0);
+                tmem_ld32(taddr + 32, v1);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl.acc_empty[ab]);
+                if (compute && 64 * half < len) {
+                    uint8_t *yh = ys + half * PM * 128 + row * 128;   // this row of this half, swizzled
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        uint4 *yp = reinterpret_cast<uint4 *>(yh + ((q ^ (row & 7)) * 16));
+                        const uint4 y0 = *yp;
+                        const __nv_bfloat162 *y2 = reinterpret_cast<const __nv_bfloat162 *>(&y0);
+                        uint4 out;
+                        uint32_t *o = reinterpret_cast<uint32_t *>(&out);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(y2[e]);
+                            const uint32_t a0 = q < 4 ? v0[8 * q + 2 * e] : v1[8 * (q - 4) + 2 * e];
+                            const uint32_t a1 = q < 4 ? v0[8 * q + 2 * e + 1] : v1[8 * (q - 4) + 2 * e + 1];
+                            o[e] = pack_bf16x2(fmaf(ui.scale, __uint_as_float(a0), f.x),
+                                               fmaf(ui.scale, __uint_as_float(a1), f.y));
+                        }
+                        *yp = out;
+                    }
+                }
+                if (full_tile && ui.ok) {
+                    fence_proxy_async_smem();   // the results are read by the TMA store
+                    named_sync(kEpiBar, E_EPI);
+                    if (et == 0) {
+                        tma_store_2d(&p.y_tile, c0, row0, ys);
+                        if (len > 64) tma_store_2d(&p.y_tile, c0 + 64, row0, ys + PM * 128);
+                        bulk_commit();
+                        bulk_wait_read_all();
+                        mbar_arrive(&ctl.empty[s]);
+                    }
+                } else {
+                    named_sync(kEpiBar, E_EPI);
+                    // coalesced stores: sixteen threads per row, 16 bytes each
+                    if (ui.ok) {
+#pragma unroll
+                        for (int it = 0; it < (PM * NCH / 8) / E_EPI; ++it) {
+                            const int i = et + it * E_EPI;
+                            const int r = i / (NCH / 8), q = i % (NCH / 8);
+                            const int tr = ctl.rows[hb][r];
+                            if (r < ui.nvalid && tr >= 0 && 8 * q < len) {
+                                const uint8_t *src = ys + (q / 8) * PM * 128 + r * 128 + (((q % 8) ^ (r & 7)) * 16);
+                                *reinterpret_cast<uint4 *>(p.Y + (int64_t)tr * p.ldy + c0 + 8 * q) =
+                                    *reinterpret_cast<const uint4 *>(src);
+                            }
+                        }
+                    }
+                    fence_proxy_async_smem();   // the stage is next written by TMA
+                    named_sync(kEpiBar, E_EPI);
+                    if (et == 0) mbar_arrive(&ctl.empty[s]);
+                }
+            }
+        }
+        if (et == 0) bulk_wait_all();
     }
+
+    // leave: tensor-core work done, copies landed, tensor memory freed
+    __syncthreads();
     if (ctl.fail && tid == 0) {
-        if (cg > 0) mbar_wait_bounded(&ctl.bar[0], (cg - 1) & 1u, kWaitNs);
         const uint64_t t0 = global_timer_ns();
         while (global_timer_ns() - t0 < 2000000ull) {
         }
@@ -627,16 +873,16 @@ __global__ void __launch_bounds__(PT) long_expand_kernel(const __grid_constant__
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, C::E_TMEM);
+    if (warp == 1) tmem_dealloc(tmem, C::E_TMEM);
 }
 
 // ------------------------------------------------------------------ launches
 // CTAs of `kernel` resident per SM with `smem` bytes, limited by tensor memory.
 template <typename K>
-int resident_per_sm(K kernel, int smem, int tmem_cols)
+int resident_per_sm(K kernel, int threads, int smem, int tmem_cols)
 {
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, PT, smem) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess)
         per_sm = 0;
     if (per_sm <= 0) per_sm = 1;
     return per_sm < 512 / tmem_cols ? per_sm : 512 / tmem_cols;
@@ -686,17 +932,21 @@ cudaError_t shrink_rmax(const TileParams &p, int64_t max_tiles, cudaStream_t str
 }
 
 template <int RMAX, int MODE>
-cudaError_t expand_rmax(const TileParams &p, int64_t max_units, cudaStream_t stream)
+cudaError_t expand_rmax(const TileParams &p, int64_t max_tiles, cudaStream_t stream)
 {
     using C = LongCfg<RMAX>;
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int per_sm = resident_per_sm(long_expand_kernel<RMAX, MODE>, C::E_SMEM, C::E_TMEM);
-    const int64_t cap = (int64_t)sms * per_sm;
-    const int64_t n = max_units < cap ? max_units : cap;
+    const int per_sm = resident_per_sm(long_expand_kernel<RMAX, MODE>, ET, C::E_SMEM, C::E_TMEM);
+    int64_t n = (int64_t)sms * per_sm;
+    // a CTA's share of the (tile, chunk) pairs spans at most kMaxUnits tiles
+    const int64_t need = (max_tiles + kMaxUnits - 3) / (kMaxUnits - 2);
+    if (n < need) n = need;
+    const int64_t chunks = max_tiles * ((p.d_out + NCH - 1) / NCH);
+    if (n > chunks) n = chunks;
     if (n <= 0) return cudaSuccess;
-    long_expand_kernel<RMAX, MODE><<<(unsigned)n, PT, C::E_SMEM, stream>>>(p);
+    long_expand_kernel<RMAX, MODE><<<(unsigned)n, ET, C::E_SMEM, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -735,18 +985,18 @@ cudaError_t launch_long_shrink(int rmax_bucket, const TileParams &p, int64_t max
     }
 }
 
-cudaError_t launch_long_expand(int rmax_bucket, int mode, const TileParams &p, int64_t max_units,
+cudaError_t launch_long_expand(int rmax_bucket, int mode, const TileParams &p, int64_t max_tiles,
                                cudaStream_t stream)
 {
     const bool apply = mode == MODE_APPLY;
     switch (rmax_bucket) {
     case 8:
-    case 16: return apply ? expand_rmax<16, MODE_APPLY>(p, max_units, stream)
-                          : expand_rmax<16, MODE_EXPAND>(p, max_units, stream);
-    case 32: return apply ? expand_rmax<32, MODE_APPLY>(p, max_units, stream)
-                          : expand_rmax<32, MODE_EXPAND>(p, max_units, stream);
-    case 64: return apply ? expand_rmax<64, MODE_APPLY>(p, max_units, stream)
-                          : expand_rmax<64, MODE_EXPAND>(p, max_units, stream);
+    case 16: return apply ? expand_rmax<16, MODE_APPLY>(p, max_tiles, stream)
+                          : expand_rmax<16, MODE_EXPAND>(p, max_tiles, stream);
+    case 32: return apply ? expand_rmax<32, MODE_APPLY>(p, max_tiles, stream)
+                          : expand_rmax<32, MODE_EXPAND>(p, max_tiles, stream);
+    case 64: return apply ? expand_rmax<64, MODE_APPLY>(p, max_tiles, stream)
+                          : expand_rmax<64, MODE_EXPAND>(p, max_tiles, stream);
     default: return cudaErrorInvalidValue;
     }
 }

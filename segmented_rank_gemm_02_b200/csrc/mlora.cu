@@ -220,11 +220,6 @@ mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::
     p.k_part = (int32_t)round_up((pool->d_in + ksplit - 1) / ksplit, 64);
     ksplit = (pool->d_in + p.k_part - 1) / p.k_part;
     p.ksplit = ksplit;
-    // expand: ranges of whole 128-column chunks, about four units per SM
-    const int64_t chunks = (pool->d_out + 127) / 128;
-    const int64_t ranges = std::min<int64_t>(chunks, std::max<int64_t>(1, (4 * sms + est_tiles - 1) / est_tiles));
-    p.n_unit = (int32_t)(((chunks + ranges - 1) / ranges) * 128);
-    const int64_t nr = (pool->d_out + p.n_unit - 1) / p.n_unit;
 
     // TMA views of the activations (tiles of consecutive rows, and single rows for gathers)
     if (mode != mlora::MODE_EXPAND &&
@@ -254,7 +249,7 @@ mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::
         if (e != cudaSuccess) return MLORA_ERR_CUDA;
     }
     if (mode != mlora::MODE_SHRINK) {
-        e = mlora::launch_long_expand(pool->r_bucket_max, mode, p, long_tiles * nr, stream);
+        e = mlora::launch_long_expand(pool->r_bucket_max, mode, p, long_tiles, stream);
         if (e != cudaSuccess) return MLORA_ERR_CUDA;
     }
     return MLORA_OK;

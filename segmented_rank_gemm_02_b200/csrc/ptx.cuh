@@ -74,6 +74,34 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
 }
 
+// Plain arrival (count one) on `bar`.
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// ---------------------------------------------------------------- named barriers
+// Barrier `id` (1..15) over `nthreads` threads (a multiple of 32).
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Same barrier; returns whether `pred` holds on every participating thread.
+__device__ __forceinline__ bool named_sync_and(uint32_t id, uint32_t nthreads, bool pred)
+{
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(out)
+        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+        : "memory");
+    return out != 0;
+}
+
 // ---------------------------------------------------------------- bulk copies
 // global -> this CTA's shared memory, completion counted in bytes on `bar`.
 __device__ __forceinline__ void bulk_load(void *dst_smem, const void *src_gmem, uint32_t bytes,
@@ -400,6 +428,16 @@ __device__ __forceinline__ void tma_gather4(void *dst_smem, const void *map, int
         ::"r"(smem_addr(dst_smem)), "l"(map), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
           "r"(smem_addr(bar))
         : "memory");
+}
+
+// 2-D tile store of this CTA's shared memory to [c0, c0 + box_cols) x [r0, r0 +
+// box_rows) of `map`'s tensor (parts outside the tensor are not written), tracked by
+// bulk async-groups.  c0 and r0 must not be negative.
+__device__ __forceinline__ void tma_store_2d(const void *map, int c0, int r0, const void *src_smem)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];"
+                 ::"l"(map), "r"(c0), "r"(r0), "r"(smem_addr(src_smem))
+                 : "memory");
 }
 
 // Shared-memory descriptor: K-major, 128-byte swizzle (rows of 128 bytes in 8-row,
