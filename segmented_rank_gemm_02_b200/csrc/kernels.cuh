@@ -89,6 +89,10 @@ cudaError_t launch_long_expand(int rmax_bucket, int mode, const TileParams &p, i
                                cudaStream_t stream);
 cudaError_t prepare_long_kernels();
 
+// CTAs per shrink cluster (1..8) for about `tiles` long tiles: the split of d_in
+// that minimises waves of resident clusters times 64-column blocks per CTA.
+int long_shrink_split(int rmax_bucket, int d_in, int64_t tiles);
+
 // Launch the tile kernel for the pool's largest rank bucket `rmax_bucket`
 // (8/16/32/64) in mode `mode`, with clusters of `cluster` CTAs: as many clusters as
 // can be resident at once, but no more than `max_tiles` (each loops over tiles).

@@ -8,15 +8,16 @@
 // one M=128 tensor-memory tile.
 //
 // Shrink (long_shrink_kernel).  A thread-block cluster of `ksplit` CTAs owns a tile;
-// CTA c covers one part of d_in.  One thread drives a 6-stage ring: per 64-column
-// block it issues one TMA tile load of X (128 rows x 64 columns, 128-byte swizzle)
-// when the tile's rows are consecutive in X, else 32 four-row TMA gathers, plus one
-// bulk copy of the adapter's A block (pool layout [8 groups][R][8] is already the
-// tensor core's no-swizzle K-major layout), all completing on the stage's mbarrier;
-// four blocks later it issues tcgen05.mma (M=128, N=rank bucket, K=16 each) into an
-// fp32 accumulator in tensor memory and commits the stage.  The epilogue reads the
-// accumulator with tcgen05.ld; the cluster sums its partial tiles through
-// distributed shared memory in a fixed order and writes H (fp32) once.
+// CTA c covers one part of d_in, and two CTAs fit on an SM.  Warp 0 streams the
+// part through a 4-stage ring: per 64-column block one TMA tile load of X (128 rows
+// x 64 columns, 128-byte swizzle) when the tile's rows are consecutive in X, else
+// one four-row TMA gather per lane, plus one bulk copy of the adapter's A block
+// (pool layout [8 groups][R][8] is already the tensor core's no-swizzle K-major
+// layout).  One thread of warp 1 issues tcgen05.mma (M=128, N=rank bucket, K=16
+// each) into an fp32 accumulator in tensor memory as stages land.  The epilogue
+// reads the accumulator with tcgen05.ld; the cluster sums its partial tiles through
+// distributed shared memory in a fixed order, each CTA a contiguous share written
+// to H (fp32) with coalesced stores.
 //
 // Expand (long_expand_kernel).  Warp-specialised and persistent: the (tile,
 // 128-column chunk) pairs of all long tiles are cut into one contiguous range per
@@ -47,8 +48,7 @@ constexpr int PT = 256;               // threads per CTA: two per tile row
 constexpr int PM = kLongTileRows;     // 128 rows per tile
 constexpr int KB = 64;                // d_in columns per shrink block (one 128-byte row)
 constexpr int NCH = 128;              // d_out columns per expand chunk
-constexpr int NS = 6;                 // shrink pipeline stages
-constexpr int PD = 4;                 // shrink prefetch distance (blocks ahead of the MMA)
+constexpr int NS = 4;                 // shrink pipeline stages (two CTAs fit on an SM)
 constexpr int kMaxExpandStages = 6;  // expand chunk ring, as deep as shared memory allows
 constexpr int kExpandSmemCap = 224 * 1024;   // dynamic shared memory of one expand CTA
 constexpr int kMaxSplit = 8;          // CTAs per shrink cluster
@@ -80,8 +80,9 @@ struct LongCfg {
 };
 
 struct LongCtl {
-    uint64_t bar[NS];   // MMA done per stage (expand: bar[0])
-    uint64_t full[NS];  // operands of a stage / chunk buffer landed
+    uint64_t bar[NS];   // stage free (its MMAs ended)
+    uint64_t full[NS];  // operands of a stage landed
+    uint64_t done;      // the tile's accumulator is complete
     uint32_t tmem;
     int scan[PT / 32];
     int tile[5];        // segment, first position, end position, slot, rank from metadata
@@ -90,7 +91,7 @@ struct LongCtl {
     float slot_scale;
     int rows[PM];
     int contiguous;     // the tile's rows are consecutive in X / Y
-    int fail;
+    volatile int fail;
 };
 
 __device__ __forceinline__ void report(const TileParams &p, unsigned flag) { atomicOr(p.status, flag); }
@@ -200,59 +201,63 @@ __device__ __forceinline__ bool wait_or_fail(const TileParams &p, LongCtl &ctl, 
     return true;
 }
 
-// Issue the loads of rows [0, 128) of a tile, 64 columns from c0, into a 16 KB
-// swizzled destination: one tile load when the rows are consecutive, else 32
-// four-row gathers (absent rows read past the end of the tensor, as zeros).
-__device__ __forceinline__ void load_rows(const LongCtl &ctl, const CUtensorMap *tile_map,
-                                          const CUtensorMap *rows_map, int n_rows, uint8_t *dst,
-                                          int c0, uint64_t *bar)
-{
-    if (ctl.contiguous) {
-        tma_load_2d(dst, tile_map, c0, ctl.rows[0], bar);
-    } else {
-        for (int i = 0; i < PM; i += 4) {
-            int r[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) r[q] = ctl.rows[i + q] >= 0 ? ctl.rows[i + q] : n_rows;
-            tma_gather4(dst + i * 128, rows_map, c0, r[0], r[1], r[2], r[3], bar);
-        }
-    }
-}
-
 // ------------------------------------------------------------------ shrink
+// One tile per cluster iteration.  Warp 0 streams this CTA's part of d_in (X rows by
+// TMA tile or lane-parallel four-row gathers, the adapter's A block by one bulk copy
+// per 64-column block) through an NS-stage ring; lane 0 of warp 1 issues the
+// tensor-core work as stages land and frees each stage with tcgen05.commit.  Then
+// the CTA's partial tile goes from tensor memory to shared memory, and the cluster
+// sums its partials through distributed shared memory, each CTA one contiguous
+// share of the tile, written to H with coalesced 16-byte stores.
 template <int RMAX, int R>
 __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, uint8_t *zero,
-                            uint32_t tmem, uint32_t &gb, uint32_t crank, uint32_t csize,
+                            uint32_t tmem, uint32_t &gb, uint32_t &tc, uint32_t crank, uint32_t csize,
                             int nvalid, int rank, bool ok)
 {
     using C = LongCfg<RMAX>;
     constexpr int RK = padded_rank(R);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int p0 = ctl.tile[1], slot = ctl.tile[3];
     const __nv_bfloat16 *slotA = p.pool + (int64_t)slot * p.slot_stride;
     const int k0 = min(p.d_in, (int)crank * p.k_part);
     const int k1 = min(p.d_in, k0 + p.k_part);
     const int nkb = (k1 - k0 + KB - 1) / KB;
-    const uint32_t idesc = umma_idesc_bf16(PM, RK);
     constexpr uint32_t A_BYTES = 8 * R * 16;
 
-    // one thread drives the ring: loads PD blocks ahead of the tensor core
-    if (tid == 0) {
-        auto produce = [&](int b) {
+    if (warp == 0) {
+        // ---- copies: X block (tile or gathers) + A block per stage
+        const bool contiguous = ctl.contiguous != 0;
+        int r[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int t = ctl.rows[4 * lane + q];
+            r[q] = t >= 0 ? t : p.n_rows;   // absent rows read as zeros
+        }
+        for (int b = 0; b < nkb; ++b) {
             const uint32_t G = gb + b;
-            const int s = G % NS;
-            if (G >= NS) wait_or_fail(p, ctl, &ctl.bar[s], ((G / NS) - 1) & 1u);
+            const int s = (int)(G % NS);
+            bool go = true;
+            if (lane == 0 && G >= (uint32_t)NS) go = wait_or_fail(p, ctl, &ctl.bar[s], ((G / NS) - 1) & 1u);
+            if (__shfl_sync(0xffffffffu, go ? 1 : 0, 0) == 0) break;
             uint8_t *xs = ring + s * C::S_STAGE;
             uint8_t *as = xs + C::X_STAGE;
             const int kb0 = k0 + b * KB;
-            mbar_arrive_expect_tx(&ctl.full[s], (uint32_t)C::X_STAGE + A_BYTES);
-            load_rows(ctl, &p.x_tile, &p.x_rows, p.n_rows, xs, kb0, &ctl.full[s]);
-            bulk_load(as, slotA + (int64_t)(kb0 / 8) * R * 8, A_BYTES, &ctl.full[s]);
-        };
-        auto consume = [&](int b) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&ctl.full[s], (uint32_t)C::X_STAGE + A_BYTES);
+                if (contiguous) tma_load_2d(xs, &p.x_tile, kb0, ctl.rows[0], &ctl.full[s]);
+                bulk_load(as, slotA + (int64_t)(kb0 / 8) * R * 8, A_BYTES, &ctl.full[s]);
+            }
+            __syncwarp();
+            if (!contiguous)
+                tma_gather4(xs + lane * 4 * 128, &p.x_rows, kb0, r[0], r[1], r[2], r[3], &ctl.full[s]);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---- tensor core: 4 K=16 steps per block into one fp32 accumulator
+        const uint32_t idesc = umma_idesc_bf16(PM, RK);
+        for (int b = 0; b < nkb; ++b) {
             const uint32_t G = gb + b;
-            const int s = G % NS;
-            if (!wait_or_fail(p, ctl, &ctl.full[s], (G / NS) & 1u)) return;
+            const int s = (int)(G % NS);
+            if (!wait_or_fail(p, ctl, &ctl.full[s], (G / NS) & 1u)) break;
             tc_fence_after();
             const uint32_t xs = smem_addr(ring + s * C::S_STAGE);
             const uint32_t as = xs + C::X_STAGE;
@@ -265,20 +270,18 @@ __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, ui
                 const uint64_t bd = umma_desc_kmajor(a0, R * 16, sbo);
                 umma_bf16(tmem, ad, bd, idesc, (b > 0 || st > 0) ? 1u : 0u);
             }
-            umma_commit(&ctl.bar[s]);
-        };
-        for (int b = 0; b < nkb + PD; ++b) {
-            if (b < nkb) produce(b);
-            if (b >= PD) consume(b - PD);
+            umma_commit(&ctl.bar[s]);   // stage s is free once these MMAs end
         }
-        if (nkb > 0) {
-            const uint32_t G = gb + nkb - 1;
-            wait_or_fail(p, ctl, &ctl.bar[G % NS], (G / NS) & 1u);
-        }
+        umma_commit(&ctl.done);         // the partial tile is complete
     }
     gb += nkb;
-    tc_fence_before();
+    // the other threads (and lanes 1..31 of warp 1) wait here, at a hardware barrier,
+    // instead of spinning beside the copy and MMA loops
     __syncthreads();
+    // everyone: the accumulator is final (bounded wait; a timeout leaves zeros)
+    // (warp-uniform: tcgen05.ld below is a warp-wide instruction)
+    const bool acc_ok = __all_sync(0xffffffffu, wait_or_fail(p, ctl, &ctl.done, tc & 1u));
+    ++tc;
     tc_fence_after();
 
     // this CTA's partial tile from tensor memory: warp w holds rows 32 (w % 4) .. +31
@@ -286,7 +289,7 @@ __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, ui
     constexpr int HC = RK / 2;
     float h[HC];
     const int col0 = (warp / 4) * HC;
-    if (nkb > 0) {
+    if (nkb > 0 && acc_ok) {
         const uint32_t taddr = tmem + ((uint32_t)(32 * (warp % 4)) << 16) + col0;
         if constexpr (HC == 8) {
             uint32_t v0[8];
@@ -325,29 +328,36 @@ __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, ui
     tc_fence_before();
     cluster_arrive_release();
     cluster_wait_acquire();
-    // rows r with r % csize == crank (one thread each): sum the cluster's partials in
-    // CTA order and write H
-    if (tid < PM && (uint32_t)tid % csize == crank && ok && !ctl.fail && tid < nvalid &&
-        ctl.rows[tid] >= 0) {
-        float acc[RK];
-#pragma unroll
-        for (int j = 0; j < RK; ++j) acc[j] = 0.f;
-        const uint32_t row_addr = smem_addr(red + tid * C::RED_PITCH);
-        for (uint32_t c = 0; c < csize; ++c) {
-            const uint32_t base = map_to_rank(row_addr, c);
-#pragma unroll
-            for (int j = 0; j < RK; j += 4) {
-                const float4 v = ld_dsmem_f32x4(base + 4u * j);
-                acc[j] += v.x;
-                acc[j + 1] += v.y;
-                acc[j + 2] += v.z;
-                acc[j + 3] += v.w;
+    // CTA crank sums the cluster's partials (in CTA order) for its share of the tile's
+    // float4 slots, row-major, and writes them to H: consecutive threads write
+    // consecutive columns of a row
+    if (ok && !ctl.fail) {
+        constexpr int F4 = RK / 4;                       // float4 slots per row
+        const int total = PM * F4;
+        const int per = (total + (int)csize - 1) / (int)csize;
+        const int f_lo = (int)crank * per, f_hi = min(total, f_lo + per);
+        for (int f = f_lo + tid; f < f_hi; f += PT) {
+            const int row = f / F4, c4 = f % F4;
+            if (row >= nvalid || ctl.rows[row] < 0 || 4 * c4 >= rank) continue;
+            const uint32_t addr = smem_addr(red + row * C::RED_PITCH + 4 * c4);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (uint32_t c = 0; c < csize; ++c) {
+                const float4 v = ld_dsmem_f32x4(map_to_rank(addr, c));
+                acc.x += v.x;
+                acc.y += v.y;
+                acc.z += v.z;
+                acc.w += v.w;
+            }
+            float *dst = p.ws + (int64_t)(p0 + row) * p.ws_ld + 4 * c4;
+            if (4 * c4 + 4 <= rank) {
+                *reinterpret_cast<float4 *>(dst) = acc;
+            } else {   // columns >= rank are left alone
+                const int n = rank - 4 * c4;
+                dst[0] = acc.x;
+                if (n > 1) dst[1] = acc.y;
+                if (n > 2) dst[2] = acc.z;
             }
         }
-        float *dst = p.ws + (int64_t)(p0 + tid) * p.ws_ld;
-#pragma unroll
-        for (int j = 0; j < RK; ++j)
-            if (j < rank) dst[j] = acc[j];
     }
     // peers are done reading this CTA's partial tile before the ring is refilled
     cluster_arrive_release();
@@ -379,6 +389,7 @@ __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__
             mbar_init(&ctl.bar[s], 1);
             mbar_init(&ctl.full[s], 1);
         }
+        mbar_init(&ctl.done, 1);
         fence_mbar_init();
         ctl.fail = 0;
     }
@@ -387,7 +398,7 @@ __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl.tmem;
-    uint32_t gb = 0;
+    uint32_t gb = 0, tc = 0;
     // every CTA of a cluster reads the same metadata and takes the same tiles
     for (int tile = (int)cluster_index();; tile += n_clusters) {
         const int ntiles = scan_long(p, tile, ctl);
@@ -397,22 +408,20 @@ __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__
         int rank;
         const int R = tile_setup(p, ctl, nvalid, crank == 0, ok, rank);
         if (R == 8) {
-            shrink_tile<RMAX, 8>(p, ctl, ring, zero, tmem, gb, crank, csize, nvalid, rank, ok);
+            shrink_tile<RMAX, 8>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
         } else if (R == 16) {
-            shrink_tile<RMAX, 16>(p, ctl, ring, zero, tmem, gb, crank, csize, nvalid, rank, ok);
+            shrink_tile<RMAX, 16>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
         } else if (R == 32) {
             if constexpr (RMAX >= 32)
-                shrink_tile<RMAX, 32>(p, ctl, ring, zero, tmem, gb, crank, csize, nvalid, rank, ok);
+                shrink_tile<RMAX, 32>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
         } else if (R == 64) {
             if constexpr (RMAX >= 64)
-                shrink_tile<RMAX, 64>(p, ctl, ring, zero, tmem, gb, crank, csize, nvalid, rank, ok);
+                shrink_tile<RMAX, 64>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
         }
         __syncthreads();
     }
     // leave: tensor-core work done, tensor memory freed
-    if (ctl.fail && tid == 0 && gb > 0) {
-        const uint32_t G = gb - 1;
-        mbar_wait_bounded(&ctl.bar[G % NS], (G / NS) & 1u, kWaitNs);
+    if (ctl.fail && tid == 0) {
         // let copies still in flight land before shared memory is released
         const uint64_t t0 = global_timer_ns();
         while (global_timer_ns() - t0 < 2000000ull) {
@@ -428,11 +437,14 @@ __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__
 // Warp roles.  Warp 0 copies (one lane issues the B-row bulk copies and Y0 tile
 // loads; every lane issues its own four-row gathers), warp 1 owns tensor memory and
 // issues the tensor-core work, warps 2..9 stage H and run the epilogue (two threads
-// per tile row, one 64-column half each).  The roles meet only at mbarriers:
+// per tile row, one 64-column half each), warp 10 writes finished chunks of full
+// tiles back with TMA stores and releases the stages.  The roles meet only at
+// mbarriers:
 //   full[s] / empty[s]      stage ring (B rows + Y0 rows of one 128-column chunk)
+//   res[s]                  the epilogue is done with stage s (results in place)
 //   acc_full[a] / acc_empty[a]  two fp32 accumulators of 128 columns in tensor memory
 //   h_full[b] / h_empty[b]  two H buffers (hi + lo), one per work unit in flight
-constexpr int E_WARPS = 10;
+constexpr int E_WARPS = 11;
 constexpr int ET = E_WARPS * 32;     // threads per expand CTA
 constexpr int E_EPI = 256;           // epilogue threads (warps 2..9)
 constexpr int kEpiBar = 1;           // named barrier of the epilogue warps
@@ -443,17 +455,17 @@ struct ExpUnit {
     int slot, r_meta;  // slot and rank from the metadata (-1 if none)
     float seg_scale;   // scale from the metadata
     int c_begin, c_end;   // 128-column chunks [c_begin, c_end) of d_out
+    int full, row0;       // set when staged: 128 consecutive rows from row0
 };
 
 struct ExpCtl {
-    uint64_t full[kMaxExpandStages], empty[kMaxExpandStages];
+    uint64_t full[kMaxExpandStages], empty[kMaxExpandStages], res[kMaxExpandStages];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t h_full[2], h_empty[2];
     uint32_t tmem;
     volatile int fail;
     int scan[E_WARPS];
     int rows[2][PM];   // original row of each tile position (epilogue), -1 = none
-    int full_tile[2];  // the unit's tile is 128 consecutive rows
     ExpUnit unit[kMaxUnits];
 };
 
@@ -568,6 +580,7 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
         for (int s = 0; s < C::E_NB; ++s) {
             mbar_init(&ctl.full[s], 1);
             mbar_init(&ctl.empty[s], 1);
+            mbar_init(&ctl.res[s], E_EPI / 32);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl.acc_full[b], 1);
@@ -702,7 +715,7 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
             }
         }
         __syncwarp();
-    } else {
+    } else if (warp < 2 + E_EPI / 32) {
         // ---------------------------------------------------------------- H staging + epilogue
         const int et = tid - 64;
         const int quarter = warp & 3, half = (warp - 2) >> 2;
@@ -770,7 +783,8 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
             const bool run = named_sync_and(kEpiBar, E_EPI, ui.nvalid == PM && ctl.rows[hb][row] >= 0 &&
                                                                 ctl.rows[hb][row] == ctl.rows[hb][0] + row);
             if (et == 0) {
-                ctl.full_tile[hb] = run ? 1 : 0;
+                ctl.unit[k].full = run ? 1 : 0;
+                ctl.unit[k].row0 = ctl.rows[hb][0];
                 mbar_arrive(&ctl.h_full[hb]);
             }
             return true;
@@ -785,8 +799,7 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
             const ExpUnit u = ctl.unit[k];
             const UnitInfo ui = unit_info(p, u);
             const int hb = k & 1;
-            const int row0 = ctl.rows[hb][0];
-            const bool full_tile = ctl.full_tile[hb] != 0;
+            const bool full_tile = ctl.unit[k].full != 0;
             const bool compute = ui.ok && row < ui.nvalid && ctl.rows[hb][row] >= 0;
 
             for (int ci = 0; ci < ui.nch; ++ci, ++g, ++a) {
@@ -829,15 +842,10 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
                     }
                 }
                 if (full_tile && ui.ok) {
-                    fence_proxy_async_smem();   // the results are read by the TMA store
-                    named_sync(kEpiBar, E_EPI);
-                    if (et == 0) {
-                        tma_store_2d(&p.y_tile, c0, row0, ys);
-                        if (len > 64) tma_store_2d(&p.y_tile, c0 + 64, row0, ys + PM * 128);
-                        bulk_commit();
-                        bulk_wait_read_all();
-                        mbar_arrive(&ctl.empty[s]);
-                    }
+                    // the store warp writes the chunk back with TMA and frees the stage
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ctl.res[s]);
                 } else {
                     named_sync(kEpiBar, E_EPI);
                     // coalesced stores: sixteen threads per row, 16 bytes each
@@ -855,12 +863,38 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
                         }
                     }
                     fence_proxy_async_smem();   // the stage is next written by TMA
-                    named_sync(kEpiBar, E_EPI);
-                    if (et == 0) mbar_arrive(&ctl.empty[s]);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ctl.res[s]);
                 }
             }
         }
-        if (et == 0) bulk_wait_all();
+    } else {
+        // ---------------------------------------------------------------- stores (warp 10)
+        if (lane == 0) {
+            uint32_t g = 0;
+            for (int k = 0; k < n_my && !ctl.fail; ++k) {
+                const UnitInfo ui = unit_info(p, ctl.unit[k]);
+                for (int ci = 0; ci < ui.nch; ++ci, ++g) {
+                    const int s = (int)(g % C::E_NB);
+                    if (!exp_wait(p, ctl, &ctl.res[s], (g / C::E_NB) & 1u)) break;
+                    // the epilogue staged unit k (its run flag and first row) before it
+                    // released any of the unit's chunks
+                    if (ctl.unit[k].full && ui.ok) {
+                        const int c0 = ui.n_lo + ci * NCH;
+                        const int len = min(NCH, ui.n_hi - c0);
+                        uint8_t *ys = stages + s * C::E_STAGE + C::B_BYTES;
+                        const int row0 = ctl.unit[k].row0;
+                        tma_store_2d(&p.y_tile, c0, row0, ys);
+                        if (len > 64) tma_store_2d(&p.y_tile, c0 + 64, row0, ys + PM * 128);
+                        bulk_commit();
+                        bulk_wait_read<0>();   // the stage is free once the store has read it
+                    }
+                    mbar_arrive(&ctl.empty[s]);
+                }
+            }
+            bulk_wait_all();
+        }
+        __syncwarp();
     }
 
     // leave: tensor-core work done, copies landed, tensor memory freed
@@ -888,12 +922,53 @@ int resident_per_sm(K kernel, int threads, int smem, int tmem_cols)
     return per_sm < 512 / tmem_cols ? per_sm : 512 / tmem_cols;
 }
 
+// Clusters of `cluster` shrink CTAs resident at once on the current device (cached).
+template <int RMAX>
+cudaError_t shrink_active(int cluster, int &active)
+{
+    using C = LongCfg<RMAX>;
+    static std::mutex mu;
+    static int cached[64][kMaxSplit + 1] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    active = cached[dev][cluster];
+    if (active > 0) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cluster, 1, 1);
+    cfg.blockDim = dim3(PT, 1, 1);
+    cfg.dynamicSmemBytes = C::S_SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&active, long_shrink_kernel<RMAX>, &cfg);
+    if (e != cudaSuccess) return e;
+    if (active <= 0) return cudaErrorInvalidConfiguration;
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // tensor memory: at most 512 / S_TMEM CTAs per SM
+    const int cap = sms * (512 / C::S_TMEM) / cluster;
+    if (cap > 0 && active > cap) active = cap;
+    cached[dev][cluster] = active;
+    return cudaSuccess;
+}
+
 template <int RMAX>
 cudaError_t shrink_rmax(const TileParams &p, int64_t max_tiles, cudaStream_t stream)
 {
     using C = LongCfg<RMAX>;
     const int cluster = p.ksplit;
+    int active = 0;
+    cudaError_t e = shrink_active<RMAX>(cluster, active);
+    if (e != cudaSuccess) return e;
+    const int64_t n = max_tiles < active ? max_tiles : active;
+    if (n <= 0) return cudaSuccess;
     cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(n * cluster), 1, 1);
     cfg.blockDim = dim3(PT, 1, 1);
     cfg.dynamicSmemBytes = C::S_SMEM;
     cfg.stream = stream;
@@ -904,30 +979,6 @@ cudaError_t shrink_rmax(const TileParams &p, int64_t max_tiles, cudaStream_t str
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    static std::mutex mu;
-    static int cached[64][kMaxSplit + 1] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    int active;
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        active = cached[dev][cluster];
-        if (active == 0) {
-            cfg.gridDim = dim3((unsigned)cluster, 1, 1);
-            cudaError_t e = cudaOccupancyMaxActiveClusters(&active, long_shrink_kernel<RMAX>, &cfg);
-            if (e != cudaSuccess) return e;
-            if (active <= 0) return cudaErrorInvalidConfiguration;
-            int sms = 0;
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-            // tensor memory: at most 512 / S_TMEM CTAs per SM
-            const int cap = sms * (512 / C::S_TMEM) / cluster;
-            if (cap > 0 && active > cap) active = cap;
-            cached[dev][cluster] = active;
-        }
-    }
-    const int64_t n = max_tiles < active ? max_tiles : active;
-    if (n <= 0) return cudaSuccess;
-    cfg.gridDim = dim3((unsigned)(n * cluster), 1, 1);
     return cudaLaunchKernelEx(&cfg, long_shrink_kernel<RMAX>, p);
 }
 
@@ -971,6 +1022,29 @@ cudaError_t set_long_attrs()
 }
 
 }  // namespace
+
+int long_shrink_split(int rmax_bucket, int d_in, int64_t tiles)
+{
+    // cost of a split: waves of resident clusters x 64-column blocks per CTA
+    int best = 1;
+    int64_t best_cost = -1;
+    for (int k = 1; k <= kMaxSplit; ++k) {
+        int active = 0;
+        cudaError_t e = rmax_bucket <= 16 ? shrink_active<16>(k, active)
+                        : rmax_bucket <= 32 ? shrink_active<32>(k, active)
+                                            : shrink_active<64>(k, active);
+        if (e != cudaSuccess || active <= 0) continue;
+        const int k_part = (((d_in + k - 1) / k) + KB - 1) / KB * KB;
+        if ((d_in + k_part - 1) / k_part != k) continue;   // k parts would not all be used
+        const int64_t waves = (tiles + active - 1) / active;
+        const int64_t cost = waves * (k_part / KB);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = k;
+        }
+    }
+    return best;
+}
 
 cudaError_t launch_long_shrink(int rmax_bucket, const TileParams &p, int64_t max_tiles,
                                cudaStream_t stream)

@@ -156,12 +156,6 @@ bool encode_rows_map(CUtensorMap *map, const void *base, int64_t rows, int64_t c
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count(int dev)
-{
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    return n;
-}
 
 // Make the pool's workspace hold `bytes`; growing it is not possible while the stream
 // is being captured into a graph.
@@ -211,12 +205,11 @@ mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::
     if (e != cudaSuccess) return MLORA_ERR_CUDA;
     if (!use_long) return MLORA_OK;
 
-    const int sms = sm_count(pool->device);
     const int64_t long_tiles = (int64_t)s->n_tokens / mlora::kLongTileRows + s->n_tokens / kLongRows + 1;
-    const int64_t est_tiles = std::max<int64_t>(1, s->n_tokens / mlora::kLongTileRows);
+    const int64_t est_tiles = std::max<int64_t>(1, (s->n_tokens + mlora::kLongTileRows - 1) / mlora::kLongTileRows);
     const int rk = std::max(16, pool->r_bucket_max);
-    // shrink: a cluster of ksplit CTAs per tile, each a part of d_in; about one CTA per SM
-    int ksplit = (int)std::min<int64_t>(8, std::max<int64_t>(1, sms / est_tiles));
+    // shrink: a cluster of ksplit CTAs per tile, each a part of d_in
+    int ksplit = mlora::long_shrink_split(pool->r_bucket_max, pool->d_in, est_tiles);
     p.k_part = (int32_t)round_up((pool->d_in + ksplit - 1) / ksplit, 64);
     ksplit = (pool->d_in + p.k_part - 1) / p.k_part;
     p.ksplit = ksplit;
