@@ -76,10 +76,29 @@ struct TileParams {
     // TMA views (bf16, 128-byte swizzle) of X [n_rows, d_in] and Y [n_rows, d_out]:
     // 64 x 128 tiles for runs of consecutive rows, 64 x 1 rows for gathers
     CUtensorMap x_tile, x_rows, y_tile, y_rows;
+    // TMA views of the pool's B blocks, one per rank bucket 8, 16, 32, 64: a box is
+    // one 128-column chunk of one slot's B (all its rank groups)
+    CUtensorMap b_map[4];
 };
+
+// A segment [p0, p1) goes to the long-segment kernels when it holds at least
+// long_rows grouped positions whose rows are consecutive in X and Y -- a prefill
+// request -- judged from its first and last row; scattered rows of a much-used
+// adapter (decode rows of many requests) stay with the decode-shaped kernel.  Every
+// kernel applies the same test to the same metadata, so each segment is taken by
+// exactly one of them.  (A segment whose rows are a permuted run still passes; the
+// long kernels then gather its rows, which is correct, only slower.)
+__device__ __forceinline__ bool long_segment(const TileParams &p, int p0, int p1)
+{
+    if (p1 - p0 < p.long_rows) return false;
+    if (p.token_indices == nullptr) return true;
+    return p.token_indices[p1 - 1] - p.token_indices[p0] == p1 - p0 - 1;
+}
 
 // Rows per tile of the long-segment kernels (one M=128 tensor-memory tile).
 constexpr int kLongTileRows = 128;
+// d_out columns per chunk of the long-segment expand.
+constexpr int kExpandChunk = 128;
 
 // Long-segment shrink (H of the long tiles into p.ws) and expand (reads p.ws; in
 // MODE_EXPAND it also reports the tiles' metadata problems); persistent grids.

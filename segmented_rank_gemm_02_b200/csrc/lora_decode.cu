@@ -153,7 +153,7 @@ __device__ int scan_tiles(const TileParams &p, int want, SharedCtl &ctl, bool re
                     if (reporter) report(p, kFlagBadSlot);
                 } else if (p0 < 0 || p1 < p0 || p1 > p.n_tokens) {
                     if (reporter) report(p, kFlagBadOffsets);
-                } else if (p1 - p0 < p.long_rows) {
+                } else if (!long_segment(p, p0, p1)) {
                     cnt = (p1 - p0 + TM - 1) / TM;
                 }
             }

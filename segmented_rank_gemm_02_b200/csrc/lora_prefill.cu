@@ -47,7 +47,7 @@ namespace {
 constexpr int PT = 256;               // threads per CTA: two per tile row
 constexpr int PM = kLongTileRows;     // 128 rows per tile
 constexpr int KB = 64;                // d_in columns per shrink block (one 128-byte row)
-constexpr int NCH = 128;              // d_out columns per expand chunk
+constexpr int NCH = kExpandChunk;     // d_out columns per expand chunk
 constexpr int NS = 4;                 // shrink pipeline stages (two CTAs fit on an SM)
 constexpr int kMaxExpandStages = 6;  // expand chunk ring, as deep as shared memory allows
 constexpr int kExpandSmemCap = 224 * 1024;   // dynamic shared memory of one expand CTA
@@ -121,7 +121,7 @@ __device__ int scan_long(const TileParams &p, int want, LongCtl &ctl)
             if (p.scales) sc = p.scales[g];
             // malformed segments are reported by the decode-shaped kernel's scan
             if (a >= 0 && a < p.n_slots && p0 >= 0 && p1 >= p0 && p1 <= p.n_tokens &&
-                p1 - p0 >= p.long_rows)
+                long_segment(p, p0, p1))
                 cnt = (p1 - p0 + PM - 1) / PM;
         }
         int incl = cnt;
@@ -378,6 +378,8 @@ __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__
     const int tid = threadIdx.x, warp = tid >> 5;
     const uint32_t crank = cluster_rank(), csize = cluster_size();
     const int n_clusters = (int)(gridDim.x / csize);
+    // the expand kernel may start its CTAs now, on SMs this grid leaves free
+    griddep_launch_dependents();
     if (warp == 0) {
         tmem_alloc(&ctl.tmem, C::S_TMEM);
         tmem_relinquish();
@@ -420,6 +422,9 @@ __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__
         }
         __syncthreads();
     }
+    // Nothing here reads what the decode-shaped kernel before us writes (other rows of
+    // Y and H), so the wait for it comes only now: this grid ends after it.
+    griddep_wait();
     // leave: tensor-core work done, tensor memory freed
     if (ctl.fail && tid == 0) {
         // let copies still in flight land before shared memory is released
@@ -524,7 +529,7 @@ __device__ int scan_units(const TileParams &p, ExpCtl &ctl, int want_lo, int wan
                 if (p.scales) sc = p.scales[g];
             }
             if (a >= 0 && a < p.n_slots && p0 >= 0 && p1 >= p0 && p1 <= p.n_tokens &&
-                p1 - p0 >= p.long_rows)
+                long_segment(p, p0, p1))
                 cnt = (p1 - p0 + PM - 1) / PM;
         }
         int incl = cnt;
@@ -644,7 +649,6 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
                 if (i < ui.nvalid) mine = mine && t[q] >= 0 && t[q] == row0 + i;
             }
             const bool contiguous = __all_sync(0xffffffffu, mine);
-            const __nv_bfloat16 *slotB = p.pool + (int64_t)u.slot * p.slot_stride + p.b_offset;
             for (int ci = 0; ci < ui.nch; ++ci, ++g) {
                 const int s = (int)(g % C::E_NB);
                 bool go = true;
@@ -658,12 +662,13 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
                 const int len = min(NCH, ui.n_hi - c0);
                 const int halves = len > 64 ? 2 : 1;
                 if (lane == 0) {
-                    uint32_t bytes = (uint32_t)(ui.R / 8) * len * 16;
+                    // B: one box of 128 columns x all rank groups (columns past d_out read
+                    // as zeros); Y0: one or two 64-column halves of the tile's rows
+                    uint32_t bytes = (uint32_t)ui.R * NCH * 2;
                     if (ui.ok) bytes += (uint32_t)halves * PM * 64 * 2;
                     mbar_arrive_expect_tx(&ctl.full[s], bytes);
-                    for (int j = 0; j < ui.R / 8; ++j)   // B rows c0.., rank group j
-                        bulk_load(bs + j * NCH * 16, slotB + ((int64_t)j * p.d_out + c0) * 8, len * 16,
-                                  &ctl.full[s]);
+                    const int bi = ui.R == 8 ? 0 : ui.R == 16 ? 1 : ui.R == 32 ? 2 : 3;
+                    tma_load_4d(bs, &p.b_map[bi], 0, c0, 0, u.slot, &ctl.full[s]);
                     if (ui.ok && contiguous)
                         for (int h = 0; h < halves; ++h)
                             tma_load_2d(ys + h * PM * 128, &p.y_tile, c0 + 64 * h, row0, &ctl.full[s]);
@@ -791,6 +796,8 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
         };
 
         uint32_t g = 0, a = 0;
+        // H comes from the shrink kernel launched just before this one
+        griddep_wait();
         bool alive = n_my > 0 ? stage(0) : false;
         for (int k = 0; k < n_my && alive; ++k) {
             // the next unit's H is staged before this unit's chunks, so the tensor core
@@ -813,19 +820,23 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
                     break;
                 }
                 tc_fence_after();
-                const uint32_t taddr = tmem + ((uint32_t)(32 * quarter) << 16) + ab * NCH + 64 * half;
+                constexpr int CT = NCH / 2;                  // columns per thread
+                const uint32_t taddr = tmem + ((uint32_t)(32 * quarter) << 16) + ab * NCH + CT * half;
                 uint32_t v0[32], v1[32];
                 tmem_ld32(taddr, v0);
-                tmem_ld32(taddr + 32, v1);
+                if constexpr (CT == 64) tmem_ld32(taddr + 32, v1);
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl.acc_empty[ab]);
-                if (compute && 64 * half < len) {
-                    uint8_t *yh = ys + half * PM * 128 + row * 128;   // this row of this half, swizzled
+                if (compute && CT * half < len) {
+                    // this thread's columns [CT * half, +CT): 64-column swizzled block and
+                    // first 16-byte chunk inside its 128-byte row
+                    const int blk = (CT * half) / 64, q0 = ((CT * half) % 64) / 8;
+                    uint8_t *yh = ys + blk * PM * 128 + row * 128;
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        uint4 *yp = reinterpret_cast<uint4 *>(yh + ((q ^ (row & 7)) * 16));
+                    for (int q = 0; q < CT / 8; ++q) {
+                        uint4 *yp = reinterpret_cast<uint4 *>(yh + (((q0 + q) ^ (row & 7)) * 16));
                         const uint4 y0 = *yp;
                         const __nv_bfloat162 *y2 = reinterpret_cast<const __nv_bfloat162 *>(&y0);
                         uint4 out;
@@ -972,13 +983,16 @@ cudaError_t shrink_rmax(const TileParams &p, int64_t max_tiles, cudaStream_t str
     cfg.blockDim = dim3(PT, 1, 1);
     cfg.dynamicSmemBytes = C::S_SMEM;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // programmatic dependent launch after the decode-shaped kernel of the same call
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, long_shrink_kernel<RMAX>, p);
 }
 
@@ -997,8 +1011,19 @@ cudaError_t expand_rmax(const TileParams &p, int64_t max_tiles, cudaStream_t str
     const int64_t chunks = max_tiles * ((p.d_out + NCH - 1) / NCH);
     if (n > chunks) n = chunks;
     if (n <= 0) return cudaSuccess;
-    long_expand_kernel<RMAX, MODE><<<(unsigned)n, ET, C::E_SMEM, stream>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)n, 1, 1);
+    cfg.blockDim = dim3(ET, 1, 1);
+    cfg.dynamicSmemBytes = C::E_SMEM;
+    cfg.stream = stream;
+    // programmatic dependent launch after the shrink: copies of B and Y0 start while
+    // it finishes; the epilogue waits for it before reading H
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, long_expand_kernel<RMAX, MODE>, p);
 }
 
 template <typename K>

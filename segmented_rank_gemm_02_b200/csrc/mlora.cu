@@ -36,6 +36,10 @@ struct mlora_pool {
     float *ws;              // H partial sums of the long-segment kernels (grown on demand)
     size_t ws_bytes;
     std::mutex ws_mutex;
+    // TMA views of the B blocks for rank buckets 8, 16, 32, 64 (those <= r_bucket_max):
+    // one load brings one 128-column chunk of one slot's B, all its rank groups
+    CUtensorMap b_maps[4];
+    bool b_maps_ok;
 };
 
 namespace {
@@ -120,6 +124,7 @@ mlora::TileParams base_params(const mlora_pool *pool, const mlora_segments *s)
     p.ranks = s->ranks;
     p.scales = s->scales;
     p.token_indices = s->token_indices;
+    for (int i = 0; i < 4; ++i) p.b_map[i] = pool->b_maps[i];
     return p;
 }
 
@@ -156,6 +161,21 @@ bool encode_rows_map(CUtensorMap *map, const void *base, int64_t rows, int64_t c
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The pool's B blocks as a 4-D tensor [slot][rank group][d_out][8] (bf16), box
+// {8, 128, R/8, 1}: one 128-column chunk of one slot's B for rank bucket R.
+bool encode_b_map(CUtensorMap *map, const mlora_pool *pool, int R)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (enc == nullptr) return false;
+    const int groups = pool->r_bucket_max / 8;
+    cuuint64_t dims[4] = {8, (cuuint64_t)pool->d_out, (cuuint64_t)groups, (cuuint64_t)pool->n_slots};
+    cuuint64_t strides[3] = {16, (cuuint64_t)pool->d_out * 16, (cuuint64_t)pool->slot_stride * 2};
+    cuuint32_t box[4] = {8, (cuuint32_t)mlora::kExpandChunk, (cuuint32_t)(R / 8), 1};
+    cuuint32_t elem[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, pool->buf + pool->b_offset, dims, strides, box,
+               elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 // Make the pool's workspace hold `bytes`; growing it is not possible while the stream
 // is being captured into a graph.
@@ -194,7 +214,7 @@ mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::
     // when given, rules them out); the decode kernel then leaves them alone.
     const bool use_long = s->n_tokens >= kLongRows && pool->d_in % 64 == 0 &&
                           (s->max_segment_rows <= 0 || s->max_segment_rows >= kLongRows) &&
-                          tensor_map_encoder() != nullptr;
+                          pool->b_maps_ok;
     p.long_rows = use_long ? kLongRows : 0x7fffffff;
     p.early = use_long ? 0 : 1;
     mlora_status st = prepare_device(pool->device);
@@ -343,6 +363,11 @@ mlora_status mlora_pool_create(int32_t d_in, int32_t d_out, int32_t n_slots, int
         st = MLORA_ERR_CUDA;
     } else {
         st = prepare_device(dev);
+    }
+    if (st == MLORA_OK) {
+        pool->b_maps_ok = tensor_map_encoder() != nullptr;
+        for (int i = 0; i < 4 && pool->b_maps_ok; ++i)
+            if ((8 << i) <= rb) pool->b_maps_ok = encode_b_map(&pool->b_maps[i], pool, 8 << i);
     }
     if (st != MLORA_OK) {
         cudaGetLastError();   // clear a sticky allocation error

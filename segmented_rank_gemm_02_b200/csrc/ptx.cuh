@@ -424,6 +424,17 @@ __device__ __forceinline__ void tma_load_2d(void *dst_smem, const void *map, int
         : "memory");
 }
 
+// 4-D tile load at coordinates {c0, c1, c2, c3} (innermost first).
+__device__ __forceinline__ void tma_load_4d(void *dst_smem, const void *map, int c0, int c1, int c2,
+                                            int c3, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];"
+        ::"r"(smem_addr(dst_smem)), "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_addr(bar))
+        : "memory");
+}
+
 // Four rows r0..r3 (any order, out-of-range rows read as zero), columns
 // [c0, c0 + box_cols), placed one after another; the map's box is one row high.
 __device__ __forceinline__ void tma_gather4(void *dst_smem, const void *map, int c0, int r0, int r1,

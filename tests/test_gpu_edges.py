@@ -85,6 +85,33 @@ def test_length_one_segments_and_one_big_segment():
     assert_close(Y, oracle.reference(W, proj), "single segment")
 
 
+def test_long_segments_consecutive_scattered_and_permuted():
+    """Segments of >= 128 rows: consecutive rows (a prefill request: long-segment
+    kernels, TMA tiles), rows scattered among another adapter's (decode-shaped kernel),
+    and a permuted run of consecutive rows (long-segment kernels with row gathers)."""
+    rng = np.random.default_rng(21)
+    W = wl.random_case(21, 700, 512, 384, 3, (16, 64), base_frac=0.0, r_max=64)
+    row_slot = np.empty(700, np.int32)
+    row_slot[:260] = 0                       # rows 0..259: one request on slot 0
+    row_slot[260:] = np.where(rng.random(440) < 0.5, 1, 2)   # slots 1, 2 interleaved
+    W.row_slot = row_slot
+    proj = W.projection(0)
+    meta = _meta_from_oracle(W)
+    assert int(np.diff(meta["offsets"]).min()) >= 128
+    # permute the interior of the consecutive segment, keeping its first and last row
+    ti = meta["token_indices"].copy()
+    inner = ti[1:259].copy()
+    rng.shuffle(inner)
+    ti[1:259] = inner
+    meta["token_indices"] = ti
+    for name, m in (("consecutive + scattered", _meta_from_oracle(W)), ("permuted run", meta)):
+        Y, flags, _ = run_apply(W, proj, meta=m)
+        assert flags == 0
+        ref, f = _ref(W, proj, m)
+        assert f == 0
+        assert_close(Y, ref, name)
+
+
 def test_partial_coverage_and_empty_segments():
     W = wl.random_case(6, 90, 384, 256, 4, (16, 32), base_frac=0.0)
     proj = W.projection(0)
