@@ -10,8 +10,10 @@
 // Work decomposition.  A work tile is (segment, up to 8 consecutive grouped
 // positions).  A thread-block cluster of C CTAs owns a tile: CTA c covers its
 // slice of d_in in the shrink (split-K) and its slice of d_out in the expand.
-// The C partial H tiles (8 x R fp32) are summed through distributed shared
-// memory, so in the fused mode H never leaves the chip.  The grid holds as many
+// Each CTA pushes its partial H tile (8 x R fp32) into every CTA of the cluster
+// with st.async (distributed shared memory, completion counted on the receiver's
+// mbarrier), and each sums the C partials in CTA order, so in the fused mode H
+// never leaves the chip.  The grid holds as many
 // clusters as can be resident at once; each loops over tiles.
 //
 // Split-K GEMV with register operands.  Decode tiles are too small for staged
@@ -63,10 +65,11 @@ constexpr int kMaxCluster = 8;
 template <int RMAX>
 struct DecodeCfg {
     static constexpr int WPART_FLOATS = kWarps * TM * RMAX;   // per-warp partial H
-    static constexpr int HPART_FLOATS = TM * RMAX;            // this CTA's partial H
+    // partial H tiles pushed by the cluster's CTAs, [tile parity][source CTA][TM * R]
+    static constexpr int RECV_FLOATS = 2 * kMaxCluster * TM * RMAX;
     static constexpr int HPITCH = RMAX + 4;
     static constexpr int HFULL_FLOATS = TM * HPITCH;          // full H (after the cluster sum)
-    static constexpr int SMEM = 4 * (WPART_FLOATS + HPART_FLOATS + HFULL_FLOATS);
+    static constexpr int SMEM = 4 * (WPART_FLOATS + RECV_FLOATS + HFULL_FLOATS);
     static constexpr int MIN_BLOCKS = RMAX <= 16 ? 4 : 2;
 };
 
@@ -92,6 +95,7 @@ struct ExpandOps {
 };
 
 struct SharedCtl {
+    uint64_t hbar[2];   // partial H tiles of the cluster landed (one per tile parity)
     int scan[kWarps];
     int rows[TM];       // original row of each tile position, -1 = absent or invalid
     int tile[5];        // segment, first position, end position, slot, rank from metadata
@@ -340,15 +344,15 @@ __device__ void prefetch_first_tile(const TileParams &p, int want, SharedCtl &ct
 
 template <int RMAX, int MODE, int R>
 __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float seg_scale,
-                         SharedCtl &ctl, float *smem_f, uint32_t crank, uint32_t csize)
+                         SharedCtl &ctl, float *smem_f, uint32_t crank, uint32_t csize, uint32_t nt)
 {
     using RC = RankCfg<R>;
     using DC = DecodeCfg<RMAX>;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
     float *wpart = smem_f;
-    float *hpart = wpart + DC::WPART_FLOATS;
-    float *hfull = hpart + DC::HPART_FLOATS;
+    float *recv = wpart + DC::WPART_FLOATS + (nt & 1) * (kMaxCluster * TM * RMAX);
+    float *hfull = wpart + DC::WPART_FLOATS + DC::RECV_FLOATS;
     const __nv_bfloat16 *slotA = p.pool + (int64_t)tl.slot * p.slot_stride;
     const __nv_bfloat16 *slotB = slotA + p.b_offset;
 
@@ -448,36 +452,52 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float 
     if (tid == 0 && crank == 0 && !ok) report(p, r <= 0 ? kFlagSlotEmpty : kFlagBadRank);
     const int rank = ok ? r : 0;   // a rejected tile reads and writes no H
     const float scale = p.scales ? seg_scale : ctl.slot_scale;
+    bool h_ok = true;
 
     if constexpr (MODE != MODE_EXPAND) {
-        for (int e = tid; e < TM * R; e += kThreads) {
-            float sum = 0.f;
+        // This CTA's partial tile (summed over its warps) is pushed into every CTA of
+        // the cluster with st.async, which counts its bytes on the receiver's mbarrier:
+        // no cluster barrier with release semantics (which would first wait for the
+        // expand operands still in flight) stands between the shrink and the expand.
+        uint64_t *bar = &ctl.hbar[nt & 1];
+        if (tid == 0) mbar_arrive_expect_tx(bar, csize * TM * R * 4);
+        const uint32_t slot_s = smem_addr(recv + crank * TM * R);
+        const uint32_t bar_s = smem_addr(bar);
+        for (int e4 = tid; e4 < TM * R / 4; e4 += kThreads) {
+            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) sum += wpart[w * TM * R + e];
-            hpart[e] = sum;
+            for (int w = 0; w < kWarps; ++w) {
+                const float4 v = *reinterpret_cast<const float4 *>(wpart + w * TM * R + 4 * e4);
+                sum.x += v.x;
+                sum.y += v.y;
+                sum.z += v.z;
+                sum.w += v.w;
+            }
+            for (uint32_t c = 0; c < csize; ++c)
+                st_async_f32x4(map_to_rank(slot_s + 16u * e4, c), sum, map_to_rank(bar_s, c));
         }
-        // the cluster's partials, summed in CTA order through distributed shared memory
-        cluster_arrive_release();
-        cluster_wait_acquire();
-        const uint32_t hpart_s = smem_addr(hpart);
+        // the cluster's partials, summed in CTA order
+        const bool landed = mbar_wait_bounded(bar, (nt >> 1) & 1u, 1000000000ull);
+        if (!landed && tid == 0) report(p, kFlagTimeout);
         for (int e = tid; e < TM * R; e += kThreads) {
             const int i = e / R, j = e % R;
             if (MODE == MODE_SHRINK &&
-                ((uint32_t)i % csize != crank || i >= tl.nvalid || j >= rank || ctl.rows[i] < 0))
+                ((uint32_t)i % csize != crank || i >= tl.nvalid || j >= rank || ctl.rows[i] < 0 || !landed))
                 continue;
             float v[kMaxCluster];
 #pragma unroll
-            for (int c = 0; c < kMaxCluster; ++c)
-                v[c] = (c < (int)csize) ? ld_dsmem_f32(map_to_rank(hpart_s + 4u * e, c)) : 0.f;
+            for (int c = 0; c < kMaxCluster; ++c) v[c] = (c < (int)csize) ? recv[c * TM * R + e] : 0.f;
             float sum = 0.f;
 #pragma unroll
             for (int c = 0; c < kMaxCluster; ++c) sum += v[c];
+            if (!landed) sum = 0.f;   // (the tile's rows are then left alone)
             if constexpr (MODE == MODE_APPLY) {
                 hfull[i * DC::HPITCH + j] = sum;
             } else {
                 p.H[(int64_t)(tl.p0 + i) * p.ldh + j] = sum;
             }
         }
+        h_ok = landed;
         cluster_arrive_relaxed();   // paired with the wait at the end of the tile
     } else {
         for (int e = tid; e < TM * R; e += kThreads) {
@@ -506,7 +526,7 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float 
                 al[s][q] = pack_bf16x2(l0, l1);
             }
         }
-        const bool store = ok && row_ok;
+        const bool store = ok && row_ok && h_ok;
         for (int i = 0; i < ng; i += 2) {
             mma_expand_store<R>(e0, ah, al, scale, yrow, store, sl, warp + i * kWarps, t);
             if (i + 2 < ng) {
@@ -542,10 +562,21 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<RMAX>::MIN_BLOCKS)
     int tile = (int)cluster_index();
     // the next launch may start its CTAs now (they wait before touching our results)
     griddep_launch_dependents();
+    if constexpr (MODE != MODE_EXPAND) {
+        // receive barriers of the partial-H exchange, initialised before any peer pushes
+        if (tid == 0) {
+            mbar_init(&ctl.hbar[0], 1);
+            mbar_init(&ctl.hbar[1], 1);
+            fence_mbar_init();
+        }
+        cluster_arrive_release();
+        cluster_wait_acquire();
+    }
     if (p.early) prefetch_first_tile<RMAX, MODE>(p, tile, ctl, crank);
     griddep_wait();
     const int total = scan_tiles(p, tile, ctl, reporter);
-    for (; tile < total; tile += n_clusters) {
+    uint32_t nt = 0;   // tiles done by this CTA (parity of the exchange buffers and barriers)
+    for (; tile < total; tile += n_clusters, ++nt) {
         if (tile != (int)cluster_index()) scan_tiles(p, tile, ctl, false);
         // every CTA of the cluster reads the same metadata and reaches the same tile
         Tile tl;
@@ -565,16 +596,16 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<RMAX>::MIN_BLOCKS)
             if (R == 0 || R > RMAX) R = 8;   // rejected inside; moves rank-8 bytes
         }
         if (R == 8) {
-            run_tile<RMAX, MODE, 8>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize);
+            run_tile<RMAX, MODE, 8>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else if (R == 16) {
             if constexpr (RMAX >= 16)
-                run_tile<RMAX, MODE, 16>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize);
+                run_tile<RMAX, MODE, 16>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else if (R == 32) {
             if constexpr (RMAX >= 32)
-                run_tile<RMAX, MODE, 32>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize);
+                run_tile<RMAX, MODE, 32>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else {
             if constexpr (RMAX >= 64)
-                run_tile<RMAX, MODE, 64>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize);
+                run_tile<RMAX, MODE, 64>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         }
         __syncthreads();   // ctl and the H buffers are rewritten by the next tile
     }

@@ -499,6 +499,16 @@ __device__ __forceinline__ float ld_relaxed_f32(const float *p)
     return v;
 }
 
+// Store 16 bytes into shared memory of a CTA of this cluster (`remote_addr` and
+// `remote_bar` from map_to_rank); the bytes complete on that CTA's mbarrier.
+__device__ __forceinline__ void st_async_f32x4(uint32_t remote_addr, float4 v, uint32_t remote_bar)
+{
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+        ::"r"(remote_addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(remote_bar)
+        : "memory");
+}
+
 // Bring [p, p + bytes) into L2 (p 16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes)
 {
