@@ -21,14 +21,21 @@
 //
 // Expand (long_expand_kernel).  Warp-specialised and persistent: the (tile,
 // 128-column chunk) pairs of all long tiles are cut into one contiguous range per
-// CTA.  A producer warp streams each chunk's B rows (bulk copies) and Y0 rows (TMA
-// tile, or four-row gathers) into a ring of stages; an MMA warp multiplies
-// H_hi B^T + H_lo B^T (M=128, N=128) into one of two fp32 accumulators in tensor
-// memory; eight epilogue warps (two threads per row) add s * acc to Y0 in shared
-// memory and write the rows back -- one TMA tile store for a full tile of
-// consecutive rows, coalesced 16-byte stores otherwise -- and stage the next
-// unit's H as bf16 hi + lo parts (two buffers) ahead of its chunks.  The roles
-// meet only at mbarriers, so copies, tensor-core work and epilogue overlap.
+// CTA.  A producer warp streams each chunk's B rows (one 4-D TMA load: 128 columns
+// x all rank groups of the slot) and Y0 rows (TMA tile, or four-row gathers) into a
+// ring of stages; an MMA warp multiplies H_hi B^T + H_lo B^T (M=128, N=128) into
+// one of two fp32 accumulators in tensor memory; eight epilogue warps (two threads
+// per row) add s * acc to Y0 in shared memory and stage the next unit's H as bf16
+// hi + lo parts (two buffers) ahead of its chunks; a store warp writes full tiles
+// of consecutive rows back with TMA stores (the epilogue writes other tiles with
+// coalesced 16-byte stores) and releases the stages.  The roles meet only at
+// mbarriers, so copies, tensor-core work, epilogue and stores overlap.
+//
+// Which segments come here: those of at least 128 grouped positions whose rows are
+// consecutive in X and Y (prefill requests); see long_segment().  The shrink is
+// launched after the decode-shaped kernel and the expand after the shrink with
+// programmatic dependent launch, so each one's launch and set-up overlap the
+// kernel before it; the expand's epilogue waits for the shrink before reading H.
 //
 // Rank buckets: kernels are compiled for the pool's largest bucket and dispatch each
 // tile to code for its own bucket (bucket 8 runs as 16; its missing operand half is
