@@ -57,20 +57,20 @@ namespace mlora {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+constexpr int kMaxWarps = 8;     // CTAs of 256 threads, or 128 (see launch_rmax)
 constexpr int TM = kTileRows;   // 8
 constexpr int kMaxCluster = 8;
 
-template <int RMAX>
+template <int RMAX, int NT>
 struct DecodeCfg {
+    static constexpr int kWarps = NT / 32;
     static constexpr int WPART_FLOATS = kWarps * TM * RMAX;   // per-warp partial H
     // partial H tiles pushed by the cluster's CTAs, [tile parity][source CTA][TM * R]
     static constexpr int RECV_FLOATS = 2 * kMaxCluster * TM * RMAX;
     static constexpr int HPITCH = RMAX + 4;
     static constexpr int HFULL_FLOATS = TM * HPITCH;          // full H (after the cluster sum)
     static constexpr int SMEM = 4 * (WPART_FLOATS + RECV_FLOATS + HFULL_FLOATS);
-    static constexpr int MIN_BLOCKS = RMAX <= 16 ? 4 : 2;
+    static constexpr int MIN_BLOCKS = (RMAX <= 16 ? 4 : 2) * (256 / NT);
 };
 
 // Per-R register operands: one k32 block of the shrink, one 32-column group of the
@@ -99,7 +99,7 @@ struct ExpandOps {
 
 struct SharedCtl {
     uint64_t hbar[2];   // partial H tiles of the cluster landed (one per tile parity)
-    int scan[kWarps];
+    int scan[kMaxWarps];
     int rows[TM];       // original row of each tile position, -1 = absent or invalid
     int tile[5];        // segment, first position, end position, slot, rank from metadata
     float seg_scale;
@@ -130,9 +130,10 @@ __device__ __forceinline__ uint2 ldg_nc2(const void *p)
 // tile `want` exists, its segment and first position are left in ctl.tile.
 // SPEC: a speculative pass made before the grids this launch depends on have
 // finished (the metadata may still change): relaxed loads, nothing reported.
-template <bool SPEC = false>
+template <bool SPEC, int NT>
 __device__ int scan_tiles(const TileParams &p, int want, SharedCtl &ctl, bool reporter)
 {
+    constexpr int kThreads = NT, kWarps = NT / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid == 0) ctl.tile[0] = -1;
     __syncthreads();
@@ -310,10 +311,10 @@ __device__ __forceinline__ void mma_expand_store(const ExpandOps<R> &o, const ui
 // previous kernel.  The metadata read here may be stale; a wrong guess only costs
 // bandwidth (every address stays inside the pool), never correctness, since the
 // tile's real loads come after griddep_wait.
-template <int RMAX, int MODE>
+template <int RMAX, int MODE, int NT>
 __device__ void prefetch_first_tile(const TileParams &p, int want, SharedCtl &ctl, uint32_t crank)
 {
-    if (want >= scan_tiles<true>(p, want, ctl, false)) return;
+    if (want >= scan_tiles<true, NT>(p, want, ctl, false)) return;
     const int tid = threadIdx.x;
     const int slot = ctl.tile[3];
     if (slot < 0 || slot >= p.n_slots) return;
@@ -345,12 +346,13 @@ __device__ void prefetch_first_tile(const TileParams &p, int want, SharedCtl &ct
     }
 }
 
-template <int RMAX, int MODE, int R>
+template <int RMAX, int MODE, int R, int NT>
 __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float seg_scale,
                          SharedCtl &ctl, float *smem_f, uint32_t crank, uint32_t csize, uint32_t nt)
 {
+    constexpr int kThreads = NT, kWarps = NT / 32;
     using RC = RankCfg<R>;
-    using DC = DecodeCfg<RMAX>;
+    using DC = DecodeCfg<RMAX, NT>;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
     float *wpart = smem_f;
@@ -550,8 +552,8 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float 
     if constexpr (MODE != MODE_EXPAND) cluster_wait_acquire();
 }
 
-template <int RMAX, int MODE>
-__global__ void __launch_bounds__(kThreads, DecodeCfg<RMAX>::MIN_BLOCKS)
+template <int RMAX, int MODE, int NT>
+__global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
     lora_decode_kernel(const __grid_constant__ TileParams p)
 {
     extern __shared__ __align__(16) float smem_f[];
@@ -575,12 +577,12 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<RMAX>::MIN_BLOCKS)
         cluster_arrive_release();
         cluster_wait_acquire();
     }
-    if (p.early) prefetch_first_tile<RMAX, MODE>(p, tile, ctl, crank);
+    if (p.early) prefetch_first_tile<RMAX, MODE, NT>(p, tile, ctl, crank);
     griddep_wait();
-    const int total = scan_tiles(p, tile, ctl, reporter);
+    const int total = scan_tiles<false, NT>(p, tile, ctl, reporter);
     uint32_t nt = 0;   // tiles done by this CTA (parity of the exchange buffers and barriers)
     for (; tile < total; tile += n_clusters, ++nt) {
-        if (tile != (int)cluster_index()) scan_tiles(p, tile, ctl, false);
+        if (tile != (int)cluster_index()) scan_tiles<false, NT>(p, tile, ctl, false);
         // every CTA of the cluster reads the same metadata and reaches the same tile
         Tile tl;
         tl.seg = ctl.tile[0];
@@ -599,27 +601,57 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<RMAX>::MIN_BLOCKS)
             if (R == 0 || R > RMAX) R = 8;   // rejected inside; moves rank-8 bytes
         }
         if (R == 8) {
-            run_tile<RMAX, MODE, 8>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+            run_tile<RMAX, MODE, 8, NT>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else if (R == 16) {
             if constexpr (RMAX >= 16)
-                run_tile<RMAX, MODE, 16>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+                run_tile<RMAX, MODE, 16, NT>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else if (R == 32) {
             if constexpr (RMAX >= 32)
-                run_tile<RMAX, MODE, 32>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+                run_tile<RMAX, MODE, 32, NT>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else {
             if constexpr (RMAX >= 64)
-                run_tile<RMAX, MODE, 64>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+                run_tile<RMAX, MODE, 64, NT>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         }
         __syncthreads();   // ctl and the H buffers are rewritten by the next tile
     }
 }
 
-template <int RMAX, int MODE>
-cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, cudaStream_t stream)
+// Clusters of `cluster` CTAs of this kernel resident at once (cached per device).
+template <int RMAX, int MODE, int NT>
+cudaError_t active_clusters(int cluster, int &active)
+{
+    static std::mutex mu;
+    static int cached[64][kMaxCluster + 1] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    active = cached[dev][cluster];
+    if (active > 0) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cluster, 1, 1);
+    cfg.blockDim = dim3(NT, 1, 1);
+    cfg.dynamicSmemBytes = DecodeCfg<RMAX, NT>::SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&active, lora_decode_kernel<RMAX, MODE, NT>, &cfg);
+    if (e != cudaSuccess) return e;
+    if (active <= 0) return cudaErrorInvalidConfiguration;
+    cached[dev][cluster] = active;
+    return cudaSuccess;
+}
+
+template <int RMAX, int MODE, int NT>
+cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, int active,
+                       cudaStream_t stream)
 {
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = DecodeCfg<RMAX>::SMEM;
+    cfg.blockDim = dim3(NT, 1, 1);
+    cfg.dynamicSmemBytes = DecodeCfg<RMAX, NT>::SMEM;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -631,30 +663,30 @@ cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, cuda
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-
-    // clusters resident at once for this kernel and cluster size (cached per device)
-    static std::mutex mu;
-    static int cached[64][kMaxCluster + 1] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    int active;
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        active = cached[dev][cluster];
-        if (active == 0) {
-            cfg.gridDim = dim3((unsigned)cluster, 1, 1);
-            cudaError_t e =
-                cudaOccupancyMaxActiveClusters(&active, lora_decode_kernel<RMAX, MODE>, &cfg);
-            if (e != cudaSuccess) return e;
-            if (active <= 0) return cudaErrorInvalidConfiguration;
-            cached[dev][cluster] = active;
-        }
-    }
+    cfg.numAttrs = p.early ? 2 : 1;
     const int64_t n = max_tiles < active ? max_tiles : active;
     cfg.gridDim = dim3((unsigned)(n * cluster), 1, 1);
-    cfg.numAttrs = p.early ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, lora_decode_kernel<RMAX, MODE>, p);
+    return cudaLaunchKernelEx(&cfg, lora_decode_kernel<RMAX, MODE, NT>, p);
+}
+
+// CTA width.  256 threads keep each warp's operands in one round of loads; when the
+// batch has clearly more tiles than 256-thread clusters fit at once (many adapters or
+// long decode segments), 128-thread CTAs let twice as many tiles be in flight, which
+// hides more latency than their second round of loads costs (measured: a 4096 x 4096
+// batch of 60 tiles is 36% slower with 128 threads, batches of 300+ tiles 3-6% faster).
+template <int RMAX, int MODE>
+cudaError_t launch_mode(const TileParams &p, int cluster, int64_t max_tiles, cudaStream_t stream)
+{
+    int active = 0;
+    cudaError_t e = active_clusters<RMAX, MODE, 256>(cluster, active);
+    if (e != cudaSuccess) return e;
+    if (2 * max_tiles > 3 * (int64_t)active) {
+        int active128 = 0;
+        e = active_clusters<RMAX, MODE, 128>(cluster, active128);
+        if (e != cudaSuccess) return e;
+        return launch_one<RMAX, MODE, 128>(p, cluster, max_tiles, active128, stream);
+    }
+    return launch_one<RMAX, MODE, 256>(p, cluster, max_tiles, active, stream);
 }
 
 template <int RMAX>
@@ -662,9 +694,9 @@ cudaError_t launch_rmax(int mode, const TileParams &p, int cluster, int64_t max_
                         cudaStream_t stream)
 {
     switch (mode) {
-    case MODE_APPLY: return launch_one<RMAX, MODE_APPLY>(p, cluster, max_tiles, stream);
-    case MODE_SHRINK: return launch_one<RMAX, MODE_SHRINK>(p, cluster, max_tiles, stream);
-    case MODE_EXPAND: return launch_one<RMAX, MODE_EXPAND>(p, cluster, max_tiles, stream);
+    case MODE_APPLY: return launch_mode<RMAX, MODE_APPLY>(p, cluster, max_tiles, stream);
+    case MODE_SHRINK: return launch_mode<RMAX, MODE_SHRINK>(p, cluster, max_tiles, stream);
+    case MODE_EXPAND: return launch_mode<RMAX, MODE_EXPAND>(p, cluster, max_tiles, stream);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -672,18 +704,26 @@ cudaError_t launch_rmax(int mode, const TileParams &p, int cluster, int64_t max_
 // The shared-memory carveout is left to the driver: a preference for more L1
 // starves the kernel of resident CTAs, one for more shared memory shrinks the L1
 // through which its register operands stream (both measured slower).
+template <int RMAX, int NT>
+cudaError_t set_attrs_nt()
+{
+    cudaError_t e;
+    e = cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_APPLY, NT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX, NT>::SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_SHRINK, NT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX, NT>::SMEM);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_EXPAND, NT>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX, NT>::SMEM);
+}
+
 template <int RMAX>
 cudaError_t set_attrs()
 {
-    cudaError_t e;
-    e = cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_APPLY>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX>::SMEM);
+    cudaError_t e = set_attrs_nt<RMAX, 256>();
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_SHRINK>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX>::SMEM);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_EXPAND>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX>::SMEM);
+    return set_attrs_nt<RMAX, 128>();
 }
 
 // Repack: A [rank, d_in] -> [d_in/8][R][8]; B [d_out, rank] -> [R/8][d_out][8]; zero
