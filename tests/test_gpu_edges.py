@@ -112,6 +112,25 @@ def test_long_segments_consecutive_scattered_and_permuted():
         assert_close(Y, ref, name)
 
 
+def test_segment_mixing_scattered_rows_and_a_prefill_run():
+    """One adapter's segment = its scattered decode rows, then a prefill request of
+    consecutive rows (a mixed continuous batch): the chunks that are runs go to the
+    long-segment kernels, the others to the decode-shaped kernel."""
+    rng = np.random.default_rng(22)
+    W = wl.random_case(22, 760, 512, 384, 3, (16, 32), base_frac=0.0, r_max=32)
+    row_slot = np.empty(760, np.int32)
+    row_slot[:300] = np.where(rng.random(300) < 0.5, 1, 2)   # decode rows, slots 1 and 2
+    row_slot[300:] = 1                                       # a 460-row request on slot 1
+    W.row_slot = row_slot
+    proj = W.projection(0)
+    meta = _meta_from_oracle(W)
+    Y, flags, _ = run_apply(W, proj, meta=meta)
+    assert flags == 0
+    ref, f = _ref(W, proj, meta)
+    assert f == 0
+    assert_close(Y, ref, "mixed segment")
+
+
 def test_partial_coverage_and_empty_segments():
     W = wl.random_case(6, 90, 384, 256, 4, (16, 32), base_frac=0.0)
     proj = W.projection(0)
