@@ -57,7 +57,8 @@ typedef enum {
     MLORA_ERR_UNSUPPORTED = 2,     /* shape outside the supported limits, no sm_100 device */
     MLORA_ERR_OUT_OF_MEMORY = 3,   /* device allocation failed */
     MLORA_ERR_BAD_METADATA = 4,    /* mlora_pool_check: the device flagged bad metadata */
-    MLORA_ERR_CUDA = 5             /* a CUDA runtime call failed */
+    MLORA_ERR_CUDA = 5,            /* a CUDA runtime call failed */
+    MLORA_ERR_NO_SLOT = 6          /* mlora_slot_cache_acquire: every slot is pinned */
 } mlora_status;
 
 /* Device status bits reported by mlora_pool_check. */
@@ -67,6 +68,8 @@ typedef enum {
 #define MLORA_FLAG_BAD_ROW      8u   /* token_indices entry outside [0, n_rows) */
 #define MLORA_FLAG_SLOT_EMPTY  16u   /* segment refers to a slot with nothing loaded */
 #define MLORA_FLAG_TIMEOUT     32u   /* an internal wait gave up (results of that tile invalid) */
+#define MLORA_FLAG_STALE_SLOT  64u   /* the slot holds another generation than the batch was
+                                        built for (mlora_segments.generations) */
 
 /* Opaque adapter pool.  Owns its device slot buffer, slot table and status word. */
 typedef struct mlora_pool mlora_pool;
@@ -93,6 +96,12 @@ typedef struct {
     const float *scales;             /* [S] or NULL (then each slot's alpha / rank) */
     const int32_t *token_indices;    /* [n_tokens] grouped position -> original row, no
                                         duplicates; NULL = identity (p -> row p) */
+    const uint32_t *generations;     /* [S] or NULL: the generation of each adapter
+                                        segment's slot the batch was built for (see
+                                        mlora_pool_slot_generation); a segment whose slot
+                                        has since been reloaded or cleared is skipped and
+                                        flagged MLORA_FLAG_STALE_SLOT.  Base entries are
+                                        ignored. */
 } mlora_segments;
 
 /*
@@ -111,9 +120,12 @@ mlora_status mlora_pool_destroy(mlora_pool *pool);
  * Load an adapter into a slot: A is bf16 [rank, d_in] row-major, B is bf16
  * [d_out, rank] row-major (the PEFT layout of lora_A / lora_B), both in host
  * memory (src_is_device = 0) or device memory (1).  The slot is repacked into
- * the pool's internal layout and zero-filled up to its rank bucket.  The copy is
- * stream-ordered on `stream`; host sources may be reused when the call returns.
- * On any error the slot keeps its previous contents and rank.
+ * the pool's internal layout and zero-filled up to its rank bucket, and its
+ * generation advances by one.  The load is stream-ordered on `stream`: pageable host
+ * sources may be reused when the call returns; page-locked host sources are copied
+ * asynchronously and must stay unchanged until the stream has passed the load (so a
+ * load on one stream can overlap applies on another that use other slots).
+ * On any error the slot keeps its previous contents, rank and generation.
  */
 mlora_status mlora_pool_load_slot(mlora_pool *pool, int32_t slot, int32_t rank, float alpha,
                                   const void *A, const void *B, int32_t src_is_device,
@@ -121,6 +133,19 @@ mlora_status mlora_pool_load_slot(mlora_pool *pool, int32_t slot, int32_t rank, 
 
 /* Mark a slot empty (stream-ordered).  Segments that use it are then rejected. */
 mlora_status mlora_pool_clear_slot(mlora_pool *pool, int32_t slot, void *stream);
+
+/*
+ * Generation of a slot: 0 for a slot never loaded, then one more with every
+ * mlora_pool_load_slot and mlora_pool_clear_slot (host-side counter; the device copy
+ * the kernels compare with mlora_segments.generations is updated in stream order by
+ * the load or clear).  A serving loop records the generation when it builds a batch,
+ * so a batch that runs after its adapter was replaced is rejected rather than
+ * applied with the wrong weights (page "Multi-LoRA Serving: adapter batching",
+ * section "Eviction cannot look only at LRU": a replaced slot must not serve
+ * requests bound to the old adapter).  Loads that run concurrently with applies
+ * reading the same slot are the caller's to prevent (pin it, see mlora_slot_cache).
+ */
+mlora_status mlora_pool_slot_generation(const mlora_pool *pool, int32_t slot, uint32_t *generation);
 
 /* Host-side view of a slot: rank (0 if empty), alpha, and the parameter count
  * r (d_in + d_out) (page "Multi-LoRA Serving: adapter batching", section "LoRA on
@@ -207,6 +232,48 @@ mlora_status mlora_build_segments(const int32_t *row_slots, int32_t n_rows,
                                   int32_t *offsets, int32_t *slots, int32_t *token_indices,
                                   int32_t *n_segments, int32_t *max_segment_rows,
                                   const mlora_pool *pool, int32_t *ranks);
+
+/*
+ * Host-side adapter cache over the slots of a pool: which adapter (a caller-chosen
+ * 64-bit id) each slot holds, how many in-flight batches pin it, and least-recently
+ * used order among the unpinned ones (page "LoRA/QLoRA multi-tenant serving",
+ * section 2 on the adapter memory manager, and page "Multi-LoRA Serving: adapter
+ * batching", sections "Why the adapter cache needs tiers" and "Eviction cannot look
+ * only at LRU": pinned slots are never evicted).  No device memory, no CUDA calls;
+ * all functions are thread-safe.
+ */
+typedef struct mlora_slot_cache mlora_slot_cache;
+
+/* A cache of n_slots empty slots. */
+mlora_status mlora_slot_cache_create(int32_t n_slots, mlora_slot_cache **out);
+
+/* NULL is accepted. */
+mlora_status mlora_slot_cache_destroy(mlora_slot_cache *cache);
+
+/*
+ * Find or place adapter `adapter_id` and pin its slot (one more pin).  On a hit
+ * *needs_load = 0.  On a miss the slot is taken from the never-used slots first,
+ * then from the least recently released unpinned slot, whose adapter is forgotten
+ * (*evicted_id gets it, or UINT64_MAX if the slot was empty; evicted_id may be
+ * NULL); *needs_load = 1 and the caller loads the adapter (mlora_pool_load_slot)
+ * before using the slot.  MLORA_ERR_NO_SLOT if every slot is pinned.
+ */
+mlora_status mlora_slot_cache_acquire(mlora_slot_cache *cache, uint64_t adapter_id, int32_t *slot,
+                                      int32_t *needs_load, uint64_t *evicted_id);
+
+/* Drop one pin of a slot; with no pins left it becomes the most recently used
+ * candidate for eviction.  MLORA_ERR_INVALID_ARG if the slot is not pinned. */
+mlora_status mlora_slot_cache_release(mlora_slot_cache *cache, int32_t slot);
+
+/* Forget the adapter a slot holds (e.g. after its load failed); pins are kept. */
+mlora_status mlora_slot_cache_invalidate(mlora_slot_cache *cache, int32_t slot);
+
+/* Slot holding `adapter_id` (-1 if none), without pinning or touching the order. */
+mlora_status mlora_slot_cache_lookup(const mlora_slot_cache *cache, uint64_t adapter_id, int32_t *slot);
+
+/* Counters since creation: hits, misses, evictions of a held adapter.  NULL accepted. */
+mlora_status mlora_slot_cache_stats(const mlora_slot_cache *cache, int64_t *hits, int64_t *misses,
+                                    int64_t *evictions);
 
 /* Static description of a status code. */
 const char *mlora_status_string(mlora_status status);

@@ -23,16 +23,18 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmlora.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_OUT_OF_MEMORY, ERR_BAD_METADATA, ERR_CUDA = range(6)
-FLAG_BAD_OFFSETS, FLAG_BAD_SLOT, FLAG_BAD_RANK, FLAG_BAD_ROW, FLAG_SLOT_EMPTY, FLAG_TIMEOUT = (
-    1, 2, 4, 8, 16, 32)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_OUT_OF_MEMORY, ERR_BAD_METADATA, ERR_CUDA, ERR_NO_SLOT = range(7)
+(FLAG_BAD_OFFSETS, FLAG_BAD_SLOT, FLAG_BAD_RANK, FLAG_BAD_ROW, FLAG_SLOT_EMPTY, FLAG_TIMEOUT,
+ FLAG_STALE_SLOT) = (1, 2, 4, 8, 16, 32, 64)
 
 # Every function the header declares (checked by the CPU test suite).
 EXPORTS = ("mlora_pool_create", "mlora_pool_destroy", "mlora_pool_load_slot",
            "mlora_pool_clear_slot", "mlora_pool_slot_info", "mlora_pool_shape",
            "mlora_pool_check", "mlora_shrink", "mlora_expand", "mlora_apply",
            "mlora_apply_noalloc", "mlora_build_segments", "mlora_status_string",
-           "mlora_version")
+           "mlora_version", "mlora_pool_slot_generation", "mlora_slot_cache_create",
+           "mlora_slot_cache_destroy", "mlora_slot_cache_acquire", "mlora_slot_cache_release",
+           "mlora_slot_cache_invalidate", "mlora_slot_cache_lookup", "mlora_slot_cache_stats")
 
 
 class MloraError(RuntimeError):
@@ -46,7 +48,7 @@ class SegmentsStruct(ctypes.Structure):
                 ("n_tokens", ctypes.c_int32), ("max_segment_rows", ctypes.c_int32),
                 ("segment_offsets", ctypes.c_void_p), ("adapter_slots", ctypes.c_void_p),
                 ("ranks", ctypes.c_void_p), ("scales", ctypes.c_void_p),
-                ("token_indices", ctypes.c_void_p)]
+                ("token_indices", ctypes.c_void_p), ("generations", ctypes.c_void_p)]
 
 
 def _load():
@@ -69,6 +71,14 @@ def _load():
         "mlora_apply": [vp, seg_p, vp, i64, vp, i64, vp],
         "mlora_apply_noalloc": [vp, seg_p, vp, i64, vp, i64, vp],
         "mlora_build_segments": [vp, i32, vp, vp, vp, i32p, i32p, vp, vp],
+        "mlora_pool_slot_generation": [vp, i32, ctypes.POINTER(ctypes.c_uint32)],
+        "mlora_slot_cache_create": [i32, ctypes.POINTER(vp)],
+        "mlora_slot_cache_destroy": [vp],
+        "mlora_slot_cache_acquire": [vp, ctypes.c_uint64, i32p, i32p, ctypes.POINTER(ctypes.c_uint64)],
+        "mlora_slot_cache_release": [vp, i32],
+        "mlora_slot_cache_invalidate": [vp, i32],
+        "mlora_slot_cache_lookup": [vp, ctypes.c_uint64, i32p],
+        "mlora_slot_cache_stats": [vp, ctypes.POINTER(i64), ctypes.POINTER(i64), ctypes.POINTER(i64)],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -175,6 +185,13 @@ class Pool:
         _check(lib().mlora_pool_clear_slot(self.handle, slot, _stream_ptr(stream)),
                "mlora_pool_clear_slot")
 
+    def generation(self, slot: int) -> int:
+        """Generation of the slot's contents (mlora_pool_slot_generation)."""
+        g = ctypes.c_uint32()
+        _check(lib().mlora_pool_slot_generation(self.handle, slot, ctypes.byref(g)),
+               "mlora_pool_slot_generation")
+        return int(g.value)
+
     def slot_info(self, slot: int):
         r, a, n = ctypes.c_int32(), ctypes.c_float(), ctypes.c_int64()
         _check(lib().mlora_pool_slot_info(self.handle, slot, ctypes.byref(r), ctypes.byref(a),
@@ -226,7 +243,8 @@ def build_segments(row_slots: np.ndarray, pool: Optional[Pool] = None) -> dict:
 class DeviceSegments:
     """Segment metadata resident on the device, plus the C struct pointing at it."""
 
-    def __init__(self, meta: dict, n_rows: int, device, scales=None, identity_rows=False):
+    def __init__(self, meta: dict, n_rows: int, device, scales=None, identity_rows=False,
+                 generations=None):
         import torch
         dev = torch.device(device)
         self.offsets = torch.as_tensor(np.asarray(meta["offsets"], np.int32)).to(dev)
@@ -239,10 +257,13 @@ class DeviceSegments:
         self.token_indices = (None if (ti is None or identity_rows)
                               else torch.as_tensor(np.asarray(ti, np.int32)).to(dev))
         n_tokens = int(meta.get("n_tokens", self.offsets[-1].item() if ti is None else len(ti)))
+        gens = generations if generations is not None else meta.get("generations")
+        self.generations = None if gens is None else torch.as_tensor(
+            np.asarray(gens, np.uint32).view(np.int32)).to(dev)
         self.struct = SegmentsStruct(
             int(self.slots.numel()), int(n_rows), n_tokens, int(meta.get("max_segment_rows", 0)),
             _ptr(self.offsets), _ptr(self.slots), _ptr(self.ranks), _ptr(self.scales),
-            _ptr(self.token_indices))
+            _ptr(self.token_indices), _ptr(self.generations))
 
     @property
     def n_tokens(self) -> int:
@@ -272,6 +293,55 @@ def expand(pool: Pool, segs: DeviceSegments, H, Y, stream=None) -> None:
     """Y[t_p] = bf16(Y[t_p] + s H[p, :r] B^T) in place (mlora_expand)."""
     _check(lib().mlora_expand(pool.handle, ctypes.byref(segs.struct), _ptr(H), _ld(H, "H"),
                              _ptr(Y), _ld(Y, "Y"), _stream_ptr(stream)), "mlora_expand")
+
+
+class SlotCache:
+    """Host-side adapter cache over a pool's slots (mlora_slot_cache): LRU order among
+    unpinned slots, pin counts for in-flight batches.  Needs no GPU."""
+
+    NONE = 2 ** 64 - 1
+
+    def __init__(self, n_slots: int):
+        h = ctypes.c_void_p()
+        _check(lib().mlora_slot_cache_create(int(n_slots), ctypes.byref(h)), "mlora_slot_cache_create")
+        self.handle = h.value
+
+    def acquire(self, adapter_id: int):
+        """(slot, needs_load, evicted_id or None); pins the slot."""
+        s, nl, ev = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_uint64()
+        _check(lib().mlora_slot_cache_acquire(self.handle, ctypes.c_uint64(adapter_id), ctypes.byref(s),
+                                             ctypes.byref(nl), ctypes.byref(ev)),
+               "mlora_slot_cache_acquire")
+        return s.value, bool(nl.value), (None if ev.value == self.NONE else int(ev.value))
+
+    def release(self, slot: int) -> None:
+        _check(lib().mlora_slot_cache_release(self.handle, int(slot)), "mlora_slot_cache_release")
+
+    def invalidate(self, slot: int) -> None:
+        _check(lib().mlora_slot_cache_invalidate(self.handle, int(slot)), "mlora_slot_cache_invalidate")
+
+    def lookup(self, adapter_id: int) -> int:
+        s = ctypes.c_int32()
+        _check(lib().mlora_slot_cache_lookup(self.handle, ctypes.c_uint64(adapter_id), ctypes.byref(s)),
+               "mlora_slot_cache_lookup")
+        return s.value
+
+    def stats(self):
+        h, m, e = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        _check(lib().mlora_slot_cache_stats(self.handle, ctypes.byref(h), ctypes.byref(m), ctypes.byref(e)),
+               "mlora_slot_cache_stats")
+        return h.value, m.value, e.value
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            lib().mlora_slot_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def version() -> int:

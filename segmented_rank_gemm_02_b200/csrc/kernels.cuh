@@ -21,6 +21,7 @@ constexpr unsigned kFlagBadRank = 4u;
 constexpr unsigned kFlagBadRow = 8u;
 constexpr unsigned kFlagSlotEmpty = 16u;
 constexpr unsigned kFlagTimeout = 32u;
+constexpr unsigned kFlagStaleSlot = 64u;
 
 // Smallest rank bucket (8, 16, 32, 64) holding rank r; 0 if r is out of range.
 __host__ __device__ constexpr int rank_bucket(int r)
@@ -38,6 +39,7 @@ struct TileParams {
     int64_t b_offset;
     const int32_t *slot_rank;   // [n_slots], 0 = empty
     const float *slot_scale;    // [n_slots], alpha / rank
+    const uint32_t *slot_gen;   // [n_slots], generation of what the slot holds
     int32_t n_slots;
     unsigned int *status;       // device status word (MLORA_FLAG_* bits)
     int32_t d_in, d_out;
@@ -48,6 +50,7 @@ struct TileParams {
     const int32_t *ranks;       // may be null
     const float *scales;        // may be null
     const int32_t *token_indices;  // may be null (identity)
+    const uint32_t *generations;   // may be null: slot generation each segment expects
     // tensors
     const __nv_bfloat16 *X;
     int64_t ldx;
@@ -121,10 +124,17 @@ cudaError_t launch_tile_kernel(int mode, int rmax_bucket, const TileParams &p, i
 // Set per-kernel attributes (dynamic shared memory) on the current device.
 cudaError_t prepare_tile_kernels();
 
-// Repack one adapter from the PEFT layout into a pool slot and publish its rank/scale.
+// Repack one adapter from the PEFT layout into a pool slot and publish its rank, scale
+// and generation.
 cudaError_t launch_repack_slot(__nv_bfloat16 *slot_base, int64_t b_offset, int R, int rank,
                                int d_in, int d_out, const __nv_bfloat16 *A_src,
                                const __nv_bfloat16 *B_src, int32_t *slot_rank_entry,
-                               float *slot_scale_entry, float scale, cudaStream_t stream);
+                               float *slot_scale_entry, float scale, uint32_t *slot_gen_entry,
+                               uint32_t generation, cudaStream_t stream);
+
+// Publish a slot's rank, scale and generation without touching its weights (clear).
+cudaError_t launch_publish_slot(int32_t *slot_rank_entry, float *slot_scale_entry,
+                                uint32_t *slot_gen_entry, int rank, float scale,
+                                uint32_t generation, cudaStream_t stream);
 
 }  // namespace mlora

@@ -102,6 +102,7 @@ struct SharedCtl {
     int scan[kMaxWarps];
     int rows[TM];       // original row of each tile position, -1 = absent or invalid
     int tile[5];        // segment, first position, end position, slot, rank from metadata
+    int stale;          // the batch was built for an earlier generation of the slot
     float seg_scale;
     int slot_rank;
     float slot_scale;
@@ -190,6 +191,7 @@ __device__ int scan_tiles(const TileParams &p, int want, SharedCtl &ctl, bool re
             ctl.tile[3] = a;
             ctl.tile[4] = rk;
             ctl.seg_scale = sc;
+            if constexpr (!SPEC) ctl.stale = p.generations && p.slot_gen[a] != p.generations[g];
         }
         running += total;
         __syncthreads();   // ctl.scan is rewritten by the next chunk
@@ -380,6 +382,7 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float 
     if (tid == 0) {
         srank = p.slot_rank[tl.slot];
         sscale = p.slot_scale[tl.slot];
+        if (ctl.stale) srank = -1;   // rank -1 marks a stale generation
     }
     ShrinkOps<R> s0, s1;
     ExpandOps<R> e0, e1;
@@ -454,7 +457,8 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float 
     __syncthreads();
     const int r = ctl.slot_rank;
     const bool ok = r > 0 && (p.ranks == nullptr || r_meta == r) && rank_bucket(r) == R;
-    if (tid == 0 && crank == 0 && !ok) report(p, r <= 0 ? kFlagSlotEmpty : kFlagBadRank);
+    if (tid == 0 && crank == 0 && !ok)
+        report(p, r < 0 ? kFlagStaleSlot : r == 0 ? kFlagSlotEmpty : kFlagBadRank);
     const int rank = ok ? r : 0;   // a rejected tile reads and writes no H
     const float scale = p.scales ? seg_scale : ctl.slot_scale;
     bool h_ok = true;
@@ -731,7 +735,8 @@ cudaError_t set_attrs()
 __global__ void repack_slot_kernel(__nv_bfloat16 *slot, int64_t b_offset, int R, int rank,
                                    int d_in, int d_out, const __nv_bfloat16 *A,
                                    const __nv_bfloat16 *B, int32_t *rank_entry,
-                                   float *scale_entry, float scale)
+                                   float *scale_entry, float scale, uint32_t *gen_entry,
+                                   uint32_t generation)
 {
     const int na = R * (d_in / 8);    // 16-byte groups of the A block
     const int nb = (R / 8) * d_out;   // 16-byte groups of the B block
@@ -760,7 +765,16 @@ __global__ void repack_slot_kernel(__nv_bfloat16 *slot, int64_t b_offset, int R,
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         *rank_entry = rank;
         *scale_entry = scale;
+        *gen_entry = generation;
     }
+}
+
+__global__ void publish_slot_kernel(int32_t *rank_entry, float *scale_entry, uint32_t *gen_entry,
+                                    int rank, float scale, uint32_t generation)
+{
+    *rank_entry = rank;
+    *scale_entry = scale;
+    *gen_entry = generation;
 }
 
 }  // namespace
@@ -790,7 +804,8 @@ cudaError_t prepare_tile_kernels()
 cudaError_t launch_repack_slot(__nv_bfloat16 *slot_base, int64_t b_offset, int R, int rank,
                                int d_in, int d_out, const __nv_bfloat16 *A_src,
                                const __nv_bfloat16 *B_src, int32_t *slot_rank_entry,
-                               float *slot_scale_entry, float scale, cudaStream_t stream)
+                               float *slot_scale_entry, float scale, uint32_t *slot_gen_entry,
+                               uint32_t generation, cudaStream_t stream)
 {
     const int64_t groups = (int64_t)R * (d_in / 8) + (int64_t)(R / 8) * d_out;
     const int threads = 256;
@@ -798,7 +813,17 @@ cudaError_t launch_repack_slot(__nv_bfloat16 *slot_base, int64_t b_offset, int R
     const int blocks = (int)(blocks64 < 2048 ? blocks64 : 2048);
     repack_slot_kernel<<<blocks, threads, 0, stream>>>(slot_base, b_offset, R, rank, d_in, d_out,
                                                        A_src, B_src, slot_rank_entry,
-                                                       slot_scale_entry, scale);
+                                                       slot_scale_entry, scale, slot_gen_entry,
+                                                       generation);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_publish_slot(int32_t *slot_rank_entry, float *slot_scale_entry,
+                                uint32_t *slot_gen_entry, int rank, float scale,
+                                uint32_t generation, cudaStream_t stream)
+{
+    publish_slot_kernel<<<1, 1, 0, stream>>>(slot_rank_entry, slot_scale_entry, slot_gen_entry, rank,
+                                             scale, generation);
     return cudaGetLastError();
 }
 

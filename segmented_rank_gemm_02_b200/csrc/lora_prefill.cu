@@ -181,6 +181,8 @@ __device__ int tile_setup(const TileParams &p, LongCtl &ctl, int nvalid, bool re
     if (tid == 0) {
         ctl.slot_rank = p.slot_rank[slot];
         ctl.slot_scale = p.slot_scale[slot];
+        // a batch built for an earlier generation of the slot: rank -1 marks it stale
+        if (p.generations && p.slot_gen[slot] != p.generations[ctl.tile[0]]) ctl.slot_rank = -1;
     }
     __syncthreads();
     // consecutive rows, all present: one TMA tile covers the tile's X / Y rows
@@ -191,7 +193,8 @@ __device__ int tile_setup(const TileParams &p, LongCtl &ctl, int nvalid, bool re
     __syncthreads();
     const int r = ctl.slot_rank;
     ok = r > 0 && (p.ranks == nullptr || r_meta == r) && rank_bucket(r) != 0;
-    if (reporter && tid == 0 && !ok) report(p, r <= 0 ? kFlagSlotEmpty : kFlagBadRank);
+    if (reporter && tid == 0 && !ok)
+        report(p, r < 0 ? kFlagStaleSlot : r == 0 ? kFlagSlotEmpty : kFlagBadRank);
     rank = ok ? r : 0;
     return ok ? rank_bucket(r) : 0;
 }
@@ -463,6 +466,7 @@ constexpr int kEpiBar = 1;           // named barrier of the epilogue warps
 constexpr int kMaxUnits = 64;        // work units per CTA (the host sizes the grid)
 
 struct ExpUnit {
+    int seg;           // segment of the tile
     int p0, p1;        // first grouped position of the tile, end of its segment
     int slot, r_meta;  // slot and rank from the metadata (-1 if none)
     float seg_scale;   // scale from the metadata
@@ -484,6 +488,7 @@ struct ExpCtl {
 // Rank and scale of a unit's slot; every role derives the same values.
 struct UnitInfo {
     int nvalid, R, rank, ok, n_lo, n_hi, nch;
+    int slot_rank;   // as read (-1 if the segment's generation is stale)
     float scale;
 };
 
@@ -491,7 +496,10 @@ __device__ __forceinline__ UnitInfo unit_info(const TileParams &p, const ExpUnit
 {
     UnitInfo i;
     i.nvalid = min(PM, u.p1 - u.p0);
-    const int r = p.slot_rank[u.slot];
+    int r = p.slot_rank[u.slot];
+    // a batch built for an earlier generation of the slot: rank -1 marks it stale
+    if (p.generations && p.slot_gen[u.slot] != p.generations[u.seg]) r = -1;
+    i.slot_rank = r;
     i.ok = r > 0 && (p.ranks == nullptr || u.r_meta == r) && rank_bucket(r) != 0;
     i.rank = i.ok ? r : 0;
     i.R = i.ok ? rank_bucket(r) : 8;
@@ -559,6 +567,7 @@ __device__ int scan_units(const TileParams &p, ExpCtl &ctl, int want_lo, int wan
             const int t0 = max(lo, want_lo), t1 = min(lo + cnt - 1, want_hi);
             for (int t = t0; t <= t1; ++t) {
                 ExpUnit &e = ctl.unit[t - want_lo];
+                e.seg = g;
                 e.p0 = p0 + (t - lo) * PM;
                 e.p1 = p1;
                 e.slot = a;
@@ -751,7 +760,7 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
                 else if (MODE == MODE_EXPAND && u.c_begin == 0 && half == 0) report(p, kFlagBadRow);
             }
             if (MODE == MODE_EXPAND && u.c_begin == 0 && et == 0 && !ui.ok)
-                report(p, p.slot_rank[u.slot] <= 0 ? kFlagSlotEmpty : kFlagBadRank);
+                report(p, ui.slot_rank < 0 ? kFlagStaleSlot : ui.slot_rank == 0 ? kFlagSlotEmpty : kFlagBadRank);
             if (k >= 2 && !wait_all(&ctl.h_empty[hb], (uint32_t)((k >> 1) - 1) & 1u)) return false;
             if (half == 0) ctl.rows[hb][row] = t;
             const int RK = padded_rank(ui.R);

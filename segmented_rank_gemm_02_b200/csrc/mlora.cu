@@ -30,9 +30,11 @@ struct mlora_pool {
     __nv_bfloat16 *buf;
     int32_t *d_rank;
     float *d_scale;
+    uint32_t *d_gen;        // generation of each slot's contents (device copy)
     unsigned int *d_status;
     std::vector<int32_t> h_rank;
     std::vector<float> h_alpha;
+    std::vector<uint32_t> h_gen;
     float *ws;              // H partial sums of the long-segment kernels (grown on demand)
     size_t ws_bytes;
     std::mutex ws_mutex;
@@ -112,6 +114,7 @@ mlora::TileParams base_params(const mlora_pool *pool, const mlora_segments *s)
     p.b_offset = pool->b_offset;
     p.slot_rank = pool->d_rank;
     p.slot_scale = pool->d_scale;
+    p.slot_gen = pool->d_gen;
     p.n_slots = pool->n_slots;
     p.status = pool->d_status;
     p.d_in = pool->d_in;
@@ -124,6 +127,7 @@ mlora::TileParams base_params(const mlora_pool *pool, const mlora_segments *s)
     p.ranks = s->ranks;
     p.scales = s->scales;
     p.token_indices = s->token_indices;
+    p.generations = s->generations;
     for (int i = 0; i < 4; ++i) p.b_map[i] = pool->b_maps[i];
     return p;
 }
@@ -307,6 +311,7 @@ const char *mlora_status_string(mlora_status status)
     case MLORA_ERR_OUT_OF_MEMORY: return "out of device memory";
     case MLORA_ERR_BAD_METADATA: return "device flagged bad segment metadata";
     case MLORA_ERR_CUDA: return "CUDA runtime error";
+    case MLORA_ERR_NO_SLOT: return "every slot is pinned";
     }
     return "unknown status";
 }
@@ -344,20 +349,24 @@ mlora_status mlora_pool_create(int32_t d_in, int32_t d_out, int32_t n_slots, int
     pool->buf = nullptr;
     pool->d_rank = nullptr;
     pool->d_scale = nullptr;
+    pool->d_gen = nullptr;
     pool->d_status = nullptr;
     pool->ws = nullptr;
     pool->ws_bytes = 0;
     pool->h_rank.assign(n_slots, 0);
     pool->h_alpha.assign(n_slots, 0.f);
+    pool->h_gen.assign(n_slots, 0u);
 
     mlora_status st = MLORA_OK;
     if (cudaMalloc(&pool->buf, (size_t)stride * 2 * n_slots) != cudaSuccess ||
         cudaMalloc(&pool->d_rank, sizeof(int32_t) * n_slots) != cudaSuccess ||
         cudaMalloc(&pool->d_scale, sizeof(float) * n_slots) != cudaSuccess ||
+        cudaMalloc(&pool->d_gen, sizeof(uint32_t) * n_slots) != cudaSuccess ||
         cudaMalloc(&pool->d_status, sizeof(unsigned int)) != cudaSuccess) {
         st = MLORA_ERR_OUT_OF_MEMORY;
     } else if (cudaMemset(pool->d_rank, 0, sizeof(int32_t) * n_slots) != cudaSuccess ||
                cudaMemset(pool->d_scale, 0, sizeof(float) * n_slots) != cudaSuccess ||
+               cudaMemset(pool->d_gen, 0, sizeof(uint32_t) * n_slots) != cudaSuccess ||
                cudaMemset(pool->d_status, 0, sizeof(unsigned int)) != cudaSuccess ||
                cudaDeviceSynchronize() != cudaSuccess) {
         st = MLORA_ERR_CUDA;
@@ -386,6 +395,7 @@ mlora_status mlora_pool_destroy(mlora_pool *pool)
     if (pool->buf) cudaFree(pool->buf);
     if (pool->d_rank) cudaFree(pool->d_rank);
     if (pool->d_scale) cudaFree(pool->d_scale);
+    if (pool->d_gen) cudaFree(pool->d_gen);
     if (pool->d_status) cudaFree(pool->d_status);
     if (pool->ws) cudaFree(pool->ws);
     delete pool;
@@ -439,14 +449,16 @@ mlora_status mlora_pool_load_slot(mlora_pool *pool, int32_t slot, int32_t rank, 
         b_src = staging + a_elems;
     }
     const float scale = alpha / (float)rank;
+    const uint32_t gen = pool->h_gen[slot] + 1;
     cudaError_t e = mlora::launch_repack_slot(pool->buf + (int64_t)slot * pool->slot_stride,
                                               pool->b_offset, R, rank, pool->d_in, pool->d_out,
                                               a_src, b_src, pool->d_rank + slot,
-                                              pool->d_scale + slot, scale, st);
+                                              pool->d_scale + slot, scale, pool->d_gen + slot, gen, st);
     if (staging) cudaFreeAsync(staging, st);
     if (e != cudaSuccess) return MLORA_ERR_CUDA;
     pool->h_rank[slot] = rank;
     pool->h_alpha[slot] = alpha;
+    pool->h_gen[slot] = gen;
     return MLORA_OK;
 }
 
@@ -455,11 +467,21 @@ mlora_status mlora_pool_clear_slot(mlora_pool *pool, int32_t slot, void *stream)
     if (pool == nullptr || slot < 0 || slot >= pool->n_slots) return MLORA_ERR_INVALID_ARG;
     DeviceGuard guard(pool->device);
     if (!guard.ok) return MLORA_ERR_CUDA;
-    if (cudaMemsetAsync(pool->d_rank + slot, 0, sizeof(int32_t),
-                        static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    const uint32_t gen = pool->h_gen[slot] + 1;
+    if (mlora::launch_publish_slot(pool->d_rank + slot, pool->d_scale + slot, pool->d_gen + slot, 0, 0.f,
+                                   gen, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return MLORA_ERR_CUDA;
     pool->h_rank[slot] = 0;
     pool->h_alpha[slot] = 0.f;
+    pool->h_gen[slot] = gen;
+    return MLORA_OK;
+}
+
+mlora_status mlora_pool_slot_generation(const mlora_pool *pool, int32_t slot, uint32_t *generation)
+{
+    if (pool == nullptr || generation == nullptr || slot < 0 || slot >= pool->n_slots)
+        return MLORA_ERR_INVALID_ARG;
+    *generation = pool->h_gen[slot];
     return MLORA_OK;
 }
 
