@@ -539,6 +539,81 @@ def run_e2e(args, W, projs, meta0, entries, dev, stream, world: int = 1):
                         "over copy-in, compute and copy-out streams with two buffer sets"}
 
 
+# --------------------------------------------------------------------------- slot loads
+
+def run_slot_load(args):
+    """Adapter loads (mlora_pool_load_slot from page-locked host memory: H2D copy and
+    repack) for every adapter the workload references, and how much they slow down
+    applies running meanwhile on another stream (loads go to slots the batch does not
+    use)."""
+    import torch
+    import segmented_rank_gemm_02_b200 as mlora
+    import workloads as wl
+    from segmented_rank_gemm_02_b200 import staging
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    W = wl.make(args.config)
+    proj = W.projection(0)
+    slots = sorted(proj.A)
+    host = {s: (torch.from_numpy(proj.A[s].view(np.int16)).pin_memory(),
+                torch.from_numpy(proj.B[s].view(np.int16)).pin_memory()) for s in slots}
+    nbytes = sum(proj.A[s].nbytes + proj.B[s].nbytes for s in slots)
+    spare = [s for s in range(W.n_slots) if s not in proj.A]
+    pool = mlora.Pool(proj.d_in, proj.d_out, W.n_slots, W.r_max)
+    s_load, s_apply = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+
+    def load_all(targets):
+        for s, t in zip(slots, targets):
+            pool.load_slot(t, int(W.slot_rank[s]), float(W.slot_alpha[s]), host[s][0], host[s][1],
+                           stream=s_load)
+
+    load_all(slots)
+    torch.cuda.synchronize()
+    reps = 20
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_load)
+    for _ in range(reps):
+        load_all(slots)
+    e1.record(s_load)
+    torch.cuda.synchronize()
+    load_ms = e0.elapsed_time(e1) / reps
+
+    st = staging.upload(W, proj, dev, pool=pool)
+    k = 200
+
+    def applies():
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(s_apply)
+        for _ in range(k):
+            mlora.apply(pool, st["segs"], st["X"], st["Y"], stream=s_apply)
+        a1.record(s_apply)
+        return a0, a1
+
+    a0, a1 = applies()
+    torch.cuda.synchronize()
+    a0, a1 = applies()
+    torch.cuda.synchronize()
+    alone_us = a0.elapsed_time(a1) * 1e3 / k
+    # the same applies while adapters stream into the spare slots on the other stream
+    targets = [spare[i % len(spare)] for i in range(len(slots))] if spare else None
+    with_us = None
+    if targets:
+        a0, a1 = applies()
+        for _ in range(reps):
+            load_all(targets)
+        torch.cuda.synchronize()
+        with_us = a0.elapsed_time(a1) * 1e3 / k
+    assert pool.check() == 0
+    return {"metric": "adapter slot loads from page-locked host memory (H2D + repack)",
+            "value": nbytes / (load_ms / 1e3) / 1e9, "unit": "GB/s", "higher_is_better": True,
+            "config": {"workload": W.name, "adapters": len(slots), "bytes_per_round": nbytes,
+                       "rank": sorted(set(int(W.slot_rank[s]) for s in slots))},
+            "us_per_adapter": load_ms * 1e3 / len(slots),
+            "apply_us_alone": alone_us, "apply_us_with_concurrent_loads": with_us,
+            "note": "applies (eager launches) on one stream, loads into spare slots on another"}
+
+
 # --------------------------------------------------------------------------- reference arm
 
 def run_reference(args, rank: int, world: int):
@@ -573,6 +648,8 @@ def main(argv=None) -> int:
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--e2e-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--slot-load", action="store_true",
+                    help="measure adapter slot loads instead of the apply step (one GPU)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -580,6 +657,10 @@ def main(argv=None) -> int:
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.slot_load:
+        print(json.dumps(run_slot_load(args)), flush=True)
+        return 0
 
     if args.impl == "reference":
         if rank != 0:
