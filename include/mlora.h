@@ -87,7 +87,9 @@ typedef struct {
                                         (== segment_offsets[S] for well-formed metadata);
                                         rows of H in mlora_shrink / mlora_expand */
     int32_t max_segment_rows;        /* host hint: an upper bound on the length of any
-                                        adapter segment, or 0 if unknown.  Only steers
+                                        adapter segment whose rows are consecutive in X
+                                        and Y (the only segments the tensor-memory
+                                        kernels take), or 0 if unknown.  Only steers
                                         kernel choice; a wrong hint never changes results. */
     const int32_t *segment_offsets;  /* [S+1], non-decreasing, offsets[0] >= 0 */
     const int32_t *adapter_slots;    /* [S], -1 = base model only, else 0..n_slots-1 */
@@ -224,7 +226,8 @@ mlora_status mlora_apply_noalloc(mlora_pool *pool, const mlora_segments *segs, c
  * Segments come in the order their slot first appears; rows keep their original
  * order inside a segment.  Outputs are HOST arrays the caller sizes:
  * offsets[n_rows + 1], slots[n_rows], token_indices[n_rows].  *n_segments gets S,
- * *max_segment_rows (may be NULL) the longest adapter segment.  If pool and
+ * *max_segment_rows (may be NULL) the longest adapter segment whose rows are
+ * consecutive (the mlora_segments hint).  If pool and
  * ranks are both non-NULL, ranks[n_rows] gets each segment's slot rank (0 for
  * base).  Slots are not range-checked here (the device checks them).
  */

@@ -598,13 +598,16 @@ mlora_status mlora_build_segments(const int32_t *row_slots, int32_t n_rows, int3
     const int32_t S = (int32_t)counts.size();
     // Pass 2: offsets; pass 3: stable scatter of rows to grouped positions.
     offsets[0] = 0;
-    int32_t longest = 0;
-    for (int32_t g = 0; g < S; ++g) {
-        offsets[g + 1] = offsets[g] + counts[g];
-        if (slots[g] >= 0) longest = std::max(longest, counts[g]);
-    }
+    for (int32_t g = 0; g < S; ++g) offsets[g + 1] = offsets[g] + counts[g];
     std::vector<int32_t> cursor(offsets, offsets + S);
     for (int32_t t = 0; t < n_rows; ++t) token_indices[cursor[row_seg[t]]++] = t;
+    // the longest adapter segment whose rows are consecutive (rows keep their order, so
+    // first and last decide): only such segments can go to the tensor-memory kernels
+    int32_t longest = 0;
+    for (int32_t g = 0; g < S; ++g)
+        if (slots[g] >= 0 && counts[g] > 0 &&
+            token_indices[offsets[g + 1] - 1] - token_indices[offsets[g]] == counts[g] - 1)
+            longest = std::max(longest, counts[g]);
     *n_segments = S;
     if (max_segment_rows) *max_segment_rows = longest;
     if (pool != nullptr && ranks != nullptr) {
