@@ -37,12 +37,12 @@
 // hi + lo parts and both are multiplied on the tensor cores, so H enters the
 // product with about 2^-17 relative error instead of bf16's 2^-9.
 //
-// Back-to-back launches.  For batches without long segments the kernel is launched
-// with programmatic dependent launch: its CTAs may start while the previous kernel
-// in the stream finishes, bring their first tile's adapter slices into L2 from a
-// speculative read of the metadata (adapter weights only change through
-// load_slot), and wait (griddepcontrol.wait) before reading the metadata, X or Y
-// for real.  A stale guess costs bandwidth, never correctness.
+// Back-to-back launches.  For batches without long segments and about one wave of
+// tiles, the kernel is launched with programmatic dependent launch: its CTAs may
+// start while the previous kernel in the stream finishes, bring their first tile's
+// adapter slices into L2 from a speculative read of the metadata (adapter weights
+// only change through load_slot), and wait (griddepcontrol.wait) before reading the
+// metadata, X or Y for real.  A stale guess costs bandwidth, never correctness.
 //
 // Invalid metadata never traps: bad segments and rows are skipped and flagged in
 // the status word; every CTA of a cluster reaches the same decisions, so cluster
