@@ -181,11 +181,11 @@ bool encode_b_map(CUtensorMap *map, const mlora_pool *pool, int R)
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Make the pool's workspace hold `bytes`; growing it is not possible while the stream
-// is being captured into a graph.
+// Make the pool's workspace hold `bytes` (the caller holds pool->ws_mutex and keeps it
+// until the kernels that use the workspace are launched, so that no other thread frees
+// it in between); growing it is not possible while the stream is being captured.
 mlora_status ensure_workspace(mlora_pool *pool, size_t bytes, cudaStream_t stream)
 {
-    std::lock_guard<std::mutex> lock(pool->ws_mutex);
     if (pool->ws_bytes >= bytes) return MLORA_OK;
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return MLORA_ERR_CUDA;
@@ -251,13 +251,16 @@ mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::
         if ((size_t)s->n_tokens * rk * sizeof(float) > ext_ws_bytes) return MLORA_ERR_UNSUPPORTED;
         p.ws = ext_ws;
         p.ws_ld = rk;
-    } else if (mode == mlora::MODE_APPLY) {
+    }
+    std::unique_lock<std::mutex> ws_lock(pool->ws_mutex, std::defer_lock);
+    if (mode == mlora::MODE_APPLY && ext_ws == nullptr) {
+        ws_lock.lock();   // held until the long kernels are launched
         const size_t bytes = (size_t)s->n_tokens * rk * sizeof(float);
         st = ensure_workspace(pool, bytes, stream);
         if (st != MLORA_OK) return st;
         p.ws = pool->ws;
         p.ws_ld = rk;
-    } else {
+    } else if (mode != mlora::MODE_APPLY) {
         p.ws = p.H;
         p.ws_ld = p.ldh;
     }

@@ -131,6 +131,46 @@ def test_segment_mixing_scattered_rows_and_a_prefill_run():
     assert_close(Y, ref, "mixed segment")
 
 
+def test_apply_from_two_host_threads_on_one_pool():
+    """Two host threads share a pool and a stream; their batches have long segments of
+    different sizes, so the pool's workspace grows while the other thread launches."""
+    import threading
+    W = wl.random_case(23, 900, 512, 256, 2, (16,), base_frac=0.0, shuffle=False)
+    proj = W.projection(0)
+    pool = staging.make_pool(512, 256, W.n_slots, W.r_max, W.slot_rank, W.slot_alpha, proj.A, proj.B)
+    stream = torch.cuda.Stream()
+    ref = oracle.reference(W, proj)
+    results, errors = {}, []
+
+    def worker(n):
+        try:
+            meta = mlora.build_segments(W.row_slot[:n], pool)
+            segs = mlora.DeviceSegments(meta, n, DEVICE)
+            X = mlora.as_bf16_tensor(proj.X[:n], DEVICE)
+            Y0 = mlora.as_bf16_tensor(proj.Y0[:n], DEVICE)
+            Y = Y0.clone()
+            torch.cuda.synchronize()
+            for _ in range(5):
+                with torch.cuda.stream(stream):
+                    Y.copy_(Y0)
+                    mlora.apply(pool, segs, X, Y, stream=stream)
+            stream.synchronize()
+            results[n] = mlora.bf16_bits(Y)
+        except Exception as e:  # pragma: no cover
+            errors.append(e)
+
+    ts = [threading.Thread(target=worker, args=(n,)) for n in (300, 900)]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    assert not errors, errors
+    assert pool.check() == 0
+    for n, Y in results.items():
+        # a prefix of the batch: each row gets the same delta as in the whole batch
+        assert_close(Y, ref[:n], f"{n} rows")
+
+
 def test_partial_coverage_and_empty_segments():
     W = wl.random_case(6, 90, 384, 256, 4, (16, 32), base_frac=0.0)
     proj = W.projection(0)
