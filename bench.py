@@ -14,6 +14,10 @@ Default workload: the Llama-3-8B q_proj decode batch (d 4096, 64 rank-16 slots,
 256 rows, Zipf(1.1) adapters, 10% base-only).  --config selects the others:
 1 tiny, 2 qproj_decode, 3 qkv_prefill, 4 mixed_mlp, 5 block70b.
 
+--fused applies the projections of a layer that read the same input rows (q, k
+and v; gate and up) with one mlora_apply_multi call each, those projections then
+sharing one X; the algorithmic bytes count that X once.
+
 Under torchrun each rank runs its own batch of the same shape (independent
 problems, no collective on the data path); value = all ranks' tokens / the
 slowest rank's time.  --impl reference times the fp64 CPU oracle instead.
@@ -21,6 +25,7 @@ slowest rank's time.  --impl reference times the fp64 CPU oracle instead.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -50,8 +55,37 @@ BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
 
 # --------------------------------------------------------------------------- workload facts
 
-def workload_facts(W) -> dict:
-    """Algorithmic bytes and flops of one step (every projection once)."""
+# Projections of one layer that read the same input rows.
+FUSION_SETS = ({"q_proj", "k_proj", "v_proj"}, {"gate_proj", "up_proj"})
+
+
+def fusion_groups(W, fused: bool):
+    """Projection indices applied together: with ``fused``, the members of each fusion
+    set with a common d_in form one group (at its first member's place); otherwise
+    every projection alone."""
+    n = len(W.proj_shapes)
+    if not fused:
+        return [[j] for j in range(n)]
+    groups, taken = [], set()
+    for j, (name, d_in, _) in enumerate(W.proj_shapes):
+        if j in taken:
+            continue
+        fam = next((f for f in FUSION_SETS if name in f), None)
+        g = [j] if fam is None else [i for i, (nm, di, _) in enumerate(W.proj_shapes)
+                                     if i not in taken and nm in fam and di == d_in]
+        taken.update(g)
+        groups.append(g)
+    return groups
+
+
+def group_leaders(groups):
+    """Projection -> the projection whose X it reads (the first of its group)."""
+    return {j: g[0] for g in groups for j in g}
+
+
+def workload_facts(W, groups=None) -> dict:
+    """Algorithmic bytes and flops of one step (every projection once; X once per group)."""
+    leader = group_leaders(groups or [[j] for j in range(len(W.proj_shapes))])
     adapter = W.row_slot >= 0
     n_l = int(adapter.sum())
     distinct = W.referenced_slots
@@ -59,9 +93,9 @@ def workload_facts(W) -> dict:
     total_bytes = 0
     flops = 0
     per_proj = []
-    for name, d_in, d_out in W.proj_shapes:
+    for j, (name, d_in, d_out) in enumerate(W.proj_shapes):
         w_bytes = int(sum(int(W.slot_rank[s]) * (d_in + d_out) * 2 for s in distinct))
-        x_bytes = n_l * d_in * 2
+        x_bytes = n_l * d_in * 2 if leader[j] == j else 0
         y_bytes = n_l * d_out * 2 * 2
         b = w_bytes + x_bytes + y_bytes
         per_proj.append({"name": name, "d_in": d_in, "d_out": d_out, "bytes": b,
@@ -256,8 +290,13 @@ def run_ours(args, rank: int, world: int, device_index: int):
     torch.cuda.set_device(device_index)
     dev = torch.device("cuda", device_index)
     W = wl.make(args.config)
-    facts = workload_facts(W)
+    groups = fusion_groups(W, args.fused)
+    leader = group_leaders(groups)
+    facts = workload_facts(W, groups)
     projs = [W.projection(j) for j in range(len(W.proj_shapes))]
+    # the members of a fused group read their leader's X
+    projs = [p if leader[j] == j else dataclasses.replace(p, X=projs[leader[j]].X)
+             for j, p in enumerate(projs)]
     meta = mlora.build_segments(W.row_slot)
     n_proj = len(projs)
 
@@ -276,13 +315,15 @@ def run_ours(args, rank: int, world: int, device_index: int):
             m = dict(meta)
             m["ranks"] = np.array([0 if s < 0 else W.slot_rank[s] for s in meta["slots"]], np.int32)
             segs = mlora.DeviceSegments(m, W.n_rows, dev)
-            out.append({"pool": pool, "segs": segs, "X": X0[j].clone(), "Y": Y0[j].clone()})
+            X = X0[j].clone() if leader[j] == j else out[leader[j]]["X"]
+            out.append({"pool": pool, "segs": segs, "X": X, "Y": Y0[j].clone()})
         return out
 
     rb = next(b for b in (8, 16, 32, 64) if b >= W.r_max)
     pool_bytes = sum(W.n_slots * 2 * (((rb * (p.d_in + p.d_out) + 127) // 128) * 128)
                      for p in projs)
-    act_bytes = sum(W.n_rows * (p.d_in + p.d_out) * 2 for p in projs)
+    act_bytes = sum(W.n_rows * ((p.d_in if leader[j] == j else 0) + p.d_out) * 2
+                    for j, p in enumerate(projs))
     set_bytes = pool_bytes + act_bytes
     try:
         l2 = int(torch.cuda.get_device_properties(dev).L2_cache_size)
@@ -296,23 +337,32 @@ def run_ours(args, rank: int, world: int, device_index: int):
     rows = np.unique(np.concatenate([meta["token_indices"][meta["offsets"][:-1]],
                                      np.nonzero(W.row_slot >= 0)[0][:8]]))
     rows = rows[W.row_slot[rows] >= 0][:48]
+    def apply_group(entries, g, stream=None, segs=None):
+        if len(g) == 1:
+            e = entries[g[0]]
+            mlora.apply(e["pool"], segs or e["segs"], e["X"], e["Y"], stream=stream)
+        else:
+            e0 = entries[g[0]]
+            mlora.apply_multi([entries[j]["pool"] for j in g], segs or e0["segs"], e0["X"],
+                              [entries[j]["Y"] for j in g], stream=stream)
+
     worst = 0.0
-    for j, p in enumerate(projs):
-        e = sets[0][j]
-        mlora.apply(e["pool"], e["segs"], e["X"], e["Y"])
-        assert e["pool"].check() == 0
-        got = oracle.bf16_to_f64(mlora.bf16_bits(e["Y"][torch.as_tensor(rows, device=dev)]))
-        ref = oracle.reference(W, p, rows=rows)
-        worst = max(worst, float(np.max(np.abs(got - ref) / (1e-2 * (1 + np.abs(ref))))))
-        e["Y"].copy_(Y0[j])
+    for g in groups:
+        apply_group(sets[0], g)
+        for j in g:
+            e, p = sets[0][j], projs[j]
+            assert e["pool"].check() == 0
+            got = oracle.bf16_to_f64(mlora.bf16_bits(e["Y"][torch.as_tensor(rows, device=dev)]))
+            ref = oracle.reference(W, p, rows=rows)
+            worst = max(worst, float(np.max(np.abs(got - ref) / (1e-2 * (1 + np.abs(ref))))))
+            e["Y"].copy_(Y0[j])
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream(device=dev)
 
     def step(k):
-        for j in range(n_proj):
-            e = sets[k % n_sets][j]
-            mlora.apply(e["pool"], e["segs"], e["X"], e["Y"], stream=stream)
+        for g in groups:
+            apply_group(sets[k % n_sets], g, stream=stream)
 
     # warm-up steps (eager), then capture exactly K steps into one graph
     with torch.cuda.stream(stream):
@@ -328,10 +378,11 @@ def run_ours(args, rank: int, world: int, device_index: int):
     with torch.cuda.stream(stream):
         graph.replay()   # first replay uploads the graph; not timed
     stream.synchronize()
-    per_apply = (launches / (args.steps * n_proj)) if launches else None
-    kernel_desc = ("mlora_apply: lora_decode_kernel" if per_apply == 1 else
-                   "mlora_apply: lora_decode_kernel + long_shrink_kernel + long_expand_kernel"
-                   if per_apply == 3 else "mlora_apply")
+    per_apply = (launches / (args.steps * len(groups))) if launches else None
+    call = "mlora_apply_multi / mlora_apply" if args.fused else "mlora_apply"
+    kernel_desc = (f"{call}: lora_decode_kernel" if per_apply == 1 else
+                   f"{call}: lora_decode_kernel + long_shrink_kernel + long_expand_kernel"
+                   if per_apply == 3 else call)
 
     dist = None
     if world > 1:
@@ -369,7 +420,7 @@ def run_ours(args, rank: int, world: int, device_index: int):
 
     # end to end through the public API with host buffers: host grouping, H2D of the
     # metadata, X and Y0 from pinned memory, mlora_apply, D2H of Y
-    e2e = run_e2e(args, W, projs, meta, sets[0], dev, stream, world)
+    e2e = run_e2e(args, W, projs, meta, sets[0], dev, stream, world, groups, apply_group)
 
     tokens = facts["adapter_rows"]
     steps = args.steps
@@ -378,7 +429,7 @@ def run_ours(args, rank: int, world: int, device_index: int):
     per_launch_s = (ms / 1e3) / steps
     peaks = measured_peaks()
     achieved = facts["bytes"] / per_launch_s / 1e9
-    traffic = recorded_traffic(W.name)
+    traffic = recorded_traffic(W.name + ("_fused" if args.fused else ""))
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": ms_max / steps, "higher_is_better": True,
@@ -393,6 +444,7 @@ def run_ours(args, rank: int, world: int, device_index: int):
             "l2": f"rotating {n_sets} buffer set(s) of {set_bytes / 2**20:.0f} MiB "
                   f"({n_sets * set_bytes / 2**20:.0f} MiB > 2x {l2 / 2**20:.0f} MiB L2)",
             "timing": "one CUDA graph of exactly K steps, CUDA events on its stream",
+            "fused": [[W.proj_shapes[j][0] for j in g] for g in groups if len(g) > 1],
         },
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -417,7 +469,7 @@ def run_ours(args, rank: int, world: int, device_index: int):
     return result
 
 
-def run_e2e(args, W, projs, meta0, entries, dev, stream, world: int = 1):
+def run_e2e(args, W, projs, meta0, entries, dev, stream, world, groups, apply_group):
     """The same step through the public API with host buffers, pipelined the way a
     serving loop would run it: step k's host grouping and H2D copies (copy-in
     stream) overlap step k-1's apply (compute stream) and step k-2's D2H copy
@@ -442,9 +494,13 @@ def run_e2e(args, W, projs, meta0, entries, dev, stream, world: int = 1):
         y_off.append(off)
         off += al(p.Y0.nbytes)
     y_end = off
-    for p in projs:
-        x_off.append(off)
-        off += al(p.X.nbytes)
+    leader = group_leaders(groups)
+    for j, p in enumerate(projs):
+        if leader[j] == j:   # a fused group's members read their leader's X
+            x_off.append(off)
+            off += al(p.X.nbytes)
+        else:
+            x_off.append(x_off[leader[j]])
     arena_bytes = off
     host = [torch.empty(arena_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
     devb = [torch.empty(arena_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
@@ -494,8 +550,9 @@ def run_e2e(args, W, projs, meta0, entries, dev, stream, world: int = 1):
         holder = type("S", (), {})()
         holder.struct = segs
         s_comp.wait_event(ev_in)
-        for j, e in enumerate(entries):
-            mlora.apply(e["pool"], holder, Xd[b][j], Yd[b][j], stream=s_comp)
+        views = [{"pool": e["pool"], "X": Xd[b][j], "Y": Yd[b][j]} for j, e in enumerate(entries)]
+        for g in groups:
+            apply_group(views, g, stream=s_comp, segs=holder)
         ev_comp = torch.cuda.Event()
         ev_comp.record(s_comp)
         with torch.cuda.stream(s_out):
@@ -535,7 +592,7 @@ def run_e2e(args, W, projs, meta0, entries, dev, stream, world: int = 1):
             "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": ms / steps,
             "includes": "host grouping (mlora_build_segments), one H2D copy of metadata+X+Y0 "
-                        "from pinned memory, mlora_apply, one D2H copy of Y; steps pipelined "
+                        "from pinned memory, the apply calls, one D2H copy of Y; steps pipelined "
                         "over copy-in, compute and copy-out streams with two buffer sets"}
 
 
@@ -648,6 +705,8 @@ def main(argv=None) -> int:
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--e2e-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fused", action="store_true",
+                    help="one mlora_apply_multi per group of projections reading the same X")
     ap.add_argument("--slot-load", action="store_true",
                     help="measure adapter slot loads instead of the apply step (one GPU)")
     args = ap.parse_args(argv)

@@ -198,6 +198,41 @@ mlora_status mlora_expand(mlora_pool *pool, const mlora_segments *segs, const fl
 mlora_status mlora_apply(mlora_pool *pool, const mlora_segments *segs, const void *X,
                          int64_t ldx, void *Y, int64_t ldy, void *stream);
 
+/* Projections one mlora_apply_multi call may cover. */
+#define MLORA_MAX_FUSED 4
+
+/*
+ * mlora_apply over several projections of one layer that read the same input rows
+ * -- q_proj, k_proj and v_proj, or gate_proj and up_proj -- in one pass over X.
+ * An adapter covers several target modules of a layer, each with its own A and B
+ * (page "Multi-LoRA Serving: adapter batching", section "An adapter is not one
+ * contiguous weight"); with one pool per module, slot a of every pool holds the
+ * same adapter's weights for that module, so one batch's segments serve them all.
+ *
+ *   For k = 0 .. n_proj-1:  Y_k[t, :] = bf16(Y_k[t, :] + s (X[t, :] A_{a,k}^T) B_{a,k}^T)
+ *
+ * with the same results as n_proj mlora_apply calls on (pools[k], Y[k]).
+ * pools[n_proj]: distinct pools with equal d_in and n_slots (d_out, r_max may
+ * differ); the rank and scale come from each pool's slot (segs->ranks, when given,
+ * must match every pool; segs->scales, when given, applies to all;
+ * segs->generations, when given, must match the slot's generation in every pool,
+ * which holds when an adapter is always loaded into all the pools together).  X: device bf16
+ * [n_rows, d_in], shared; Y[k]: device bf16 [n_rows, d_out of pools[k]] with row
+ * stride ldy[k], distinct, non-overlapping buffers.  1 <= n_proj <= MLORA_MAX_FUSED.
+ * Short segments run in one launch whose work items are (tile, projection) with a
+ * tile's projections side by side, so its X rows are read from HBM once; long
+ * segments run the long-segment kernels once per projection, each with its pool's
+ * workspace (grown as in mlora_apply, all before anything is launched).
+ * Errors: host-side as mlora_apply (plus a repeated pool or output, different
+ * d_in / n_slots / device: MLORA_ERR_INVALID_ARG).  Device-side: metadata problems
+ * found while scanning the segments (bad offsets or slots) go to pools[0]'s status
+ * word; problems of one projection's tile (bad row, empty slot, rank or generation
+ * mismatch) to that projection's pool.
+ */
+mlora_status mlora_apply_multi(mlora_pool *const *pools, int32_t n_proj,
+                               const mlora_segments *segs, const void *X, int64_t ldx,
+                               void *const *Y, const int64_t *ldy, void *stream);
+
 /*
  * mlora_apply for callers that cannot allocate device memory.  The paper has no
  * counterpart: this entry point is an interface choice of this library.

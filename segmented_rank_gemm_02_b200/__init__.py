@@ -31,7 +31,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_OUT_OF_MEMORY, ERR_BAD_METADATA, ERR_C
 EXPORTS = ("mlora_pool_create", "mlora_pool_destroy", "mlora_pool_load_slot",
            "mlora_pool_clear_slot", "mlora_pool_slot_info", "mlora_pool_shape",
            "mlora_pool_check", "mlora_shrink", "mlora_expand", "mlora_apply",
-           "mlora_apply_noalloc", "mlora_build_segments", "mlora_status_string",
+           "mlora_apply_noalloc", "mlora_apply_multi", "mlora_build_segments", "mlora_status_string",
            "mlora_version", "mlora_pool_slot_generation", "mlora_slot_cache_create",
            "mlora_slot_cache_destroy", "mlora_slot_cache_acquire", "mlora_slot_cache_release",
            "mlora_slot_cache_invalidate", "mlora_slot_cache_lookup", "mlora_slot_cache_stats")
@@ -70,6 +70,8 @@ def _load():
         "mlora_expand": [vp, seg_p, vp, i64, vp, i64, vp],
         "mlora_apply": [vp, seg_p, vp, i64, vp, i64, vp],
         "mlora_apply_noalloc": [vp, seg_p, vp, i64, vp, i64, vp],
+        "mlora_apply_multi": [ctypes.POINTER(vp), i32, seg_p, vp, i64, ctypes.POINTER(vp),
+                              ctypes.POINTER(i64), vp],
         "mlora_build_segments": [vp, i32, vp, vp, vp, i32p, i32p, vp, vp],
         "mlora_pool_slot_generation": [vp, i32, ctypes.POINTER(ctypes.c_uint32)],
         "mlora_slot_cache_create": [i32, ctypes.POINTER(vp)],
@@ -281,6 +283,23 @@ def apply_noalloc(pool: Pool, segs: DeviceSegments, X, Y, stream=None) -> None:
     (mlora_apply_noalloc): allocates nothing; concurrent calls on the GPU race."""
     _check(lib().mlora_apply_noalloc(pool.handle, ctypes.byref(segs.struct), _ptr(X), _ld(X, "X"),
                                      _ptr(Y), _ld(Y, "Y"), _stream_ptr(stream)), "mlora_apply_noalloc")
+
+
+MAX_FUSED = 4
+
+
+def apply_multi(pools, segs: DeviceSegments, X, Ys, stream=None) -> None:
+    """mlora_apply over several projections sharing X and the segments (q/k/v,
+    gate/up): Ys[k] += delta of pools[k], in one pass over X (mlora_apply_multi)."""
+    pools, Ys = list(pools), list(Ys)
+    if len(pools) != len(Ys):
+        raise ValueError("one output per pool")
+    n = len(pools)
+    handles = (ctypes.c_void_p * max(n, 1))(*[p.handle for p in pools])
+    outs = (ctypes.c_void_p * max(n, 1))(*[_ptr(Y) for Y in Ys])
+    lds = (ctypes.c_int64 * max(n, 1))(*[_ld(Y, "Y") for Y in Ys])
+    _check(lib().mlora_apply_multi(handles, n, ctypes.byref(segs.struct), _ptr(X), _ld(X, "X"),
+                                   outs, lds, _stream_ptr(stream)), "mlora_apply_multi")
 
 
 def shrink(pool: Pool, segs: DeviceSegments, X, H, stream=None) -> None:

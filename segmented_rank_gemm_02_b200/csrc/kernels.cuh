@@ -29,6 +29,25 @@ __host__ __device__ constexpr int rank_bucket(int r)
     return r <= 0 ? 0 : r <= 8 ? 8 : r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : 0;
 }
 
+// Projections one fused launch of the decode-shaped kernel may cover.
+constexpr int kMaxFused = 4;
+
+// What differs between the projections of a fused launch: each has its own pool
+// (same d_in and slot numbering, its own d_out) and its own output.  Entry 0 repeats
+// the single-projection fields of TileParams.
+struct ProjView {
+    const __nv_bfloat16 *pool;
+    int64_t slot_stride;
+    int64_t b_offset;
+    const int32_t *slot_rank;
+    const float *slot_scale;
+    const uint32_t *slot_gen;
+    unsigned int *status;       // this projection's status word (its slot problems)
+    int32_t d_out, n_slice;
+    __nv_bfloat16 *Y;
+    int64_t ldy;
+};
+
 // Everything one launch of the segmented tile kernel needs.  Passed by value.
 struct TileParams {
     // adapter pool: slot a's A block starts at pool + a * slot_stride and holds
@@ -82,6 +101,10 @@ struct TileParams {
     // TMA views of the pool's B blocks, one per rank bucket 8, 16, 32, 64: a box is
     // one 128-column chunk of one slot's B (all its rank groups)
     CUtensorMap b_map[4];
+    // decode-shaped kernel: the projections it applies (1 unless fused; all share X,
+    // d_in, the segment metadata and the slot numbering)
+    int32_t n_proj;
+    ProjView proj[kMaxFused];
 };
 
 // A segment [p0, p1) goes to the long-segment kernels when it holds at least
@@ -120,6 +143,11 @@ int long_shrink_split(int rmax_bucket, int d_in, int64_t tiles);
 // can be resident at once, but no more than `max_tiles` (each loops over tiles).
 cudaError_t launch_tile_kernel(int mode, int rmax_bucket, const TileParams &p, int cluster,
                                int64_t max_tiles, cudaStream_t stream);
+
+// Fused launch over p.n_proj projections (MODE_APPLY): a work item is one tile of one
+// projection, and the items of a tile are adjacent so its X rows come from HBM once.
+cudaError_t launch_tile_kernel_fused(int rmax_bucket, const TileParams &p, int cluster,
+                                     int64_t max_items, cudaStream_t stream);
 
 // Set per-kernel attributes (dynamic shared memory) on the current device.
 cudaError_t prepare_tile_kernels();

@@ -117,6 +117,11 @@ __device__ __forceinline__ void report(const TileParams &p, unsigned flag)
     atomicOr(p.status, flag);
 }
 
+__device__ __forceinline__ void report(const ProjView &v, unsigned flag)
+{
+    atomicOr(v.status, flag);
+}
+
 __device__ __forceinline__ uint4 ldg_nc(const void *p)
 {
     return __ldg(reinterpret_cast<const uint4 *>(p));
@@ -131,8 +136,10 @@ __device__ __forceinline__ uint2 ldg_nc2(const void *p)
 // tile `want` exists, its segment and first position are left in ctl.tile.
 // SPEC: a speculative pass made before the grids this launch depends on have
 // finished (the metadata may still change): relaxed loads, nothing reported.
+// slot_gen: generations of the pool the tile will read (ctl.stale).
 template <bool SPEC, int NT>
-__device__ int scan_tiles(const TileParams &p, int want, SharedCtl &ctl, bool reporter)
+__device__ int scan_tiles(const TileParams &p, const uint32_t *slot_gen, int want, SharedCtl &ctl,
+                          bool reporter)
 {
     constexpr int kThreads = NT, kWarps = NT / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -191,7 +198,7 @@ __device__ int scan_tiles(const TileParams &p, int want, SharedCtl &ctl, bool re
             ctl.tile[3] = a;
             ctl.tile[4] = rk;
             ctl.seg_scale = sc;
-            if constexpr (!SPEC) ctl.stale = p.generations && p.slot_gen[a] != p.generations[g];
+            if constexpr (!SPEC) ctl.stale = p.generations && slot_gen[a] != p.generations[g];
         }
         running += total;
         __syncthreads();   // ctl.scan is rewritten by the next chunk
@@ -314,19 +321,20 @@ __device__ __forceinline__ void mma_expand_store(const ExpandOps<R> &o, const ui
 // bandwidth (every address stays inside the pool), never correctness, since the
 // tile's real loads come after griddep_wait.
 template <int RMAX, int MODE, int NT>
-__device__ void prefetch_first_tile(const TileParams &p, int want, SharedCtl &ctl, uint32_t crank)
+__device__ void prefetch_first_tile(const TileParams &p, const ProjView &v, int want, SharedCtl &ctl,
+                                    uint32_t crank)
 {
-    if (want >= scan_tiles<true, NT>(p, want, ctl, false)) return;
+    if (want >= scan_tiles<true, NT>(p, v.slot_gen, want, ctl, false)) return;
     const int tid = threadIdx.x;
     const int slot = ctl.tile[3];
     if (slot < 0 || slot >= p.n_slots) return;
     int R = rank_bucket(ctl.tile[4]);
-    if (p.ranks == nullptr || R == 0 || R > RMAX) R = rank_bucket(ld_relaxed_s32(p.slot_rank + slot));
+    if (p.ranks == nullptr || R == 0 || R > RMAX) R = rank_bucket(ld_relaxed_s32(v.slot_rank + slot));
     if (R == 0 || R > RMAX) return;
     const int p0 = ctl.tile[1];
     if (tid == 32 && p.token_indices != nullptr && p0 >= 0 && p0 < p.n_tokens)
         prefetch_l2_line(p.token_indices + p0);
-    const char *slotA = reinterpret_cast<const char *>(p.pool + (int64_t)slot * p.slot_stride);
+    const char *slotA = reinterpret_cast<const char *>(v.pool + (int64_t)slot * v.slot_stride);
     constexpr uint32_t kChunk = 16384;
     if (MODE != MODE_EXPAND && tid < 8) {
         // A block [d_in/8][R][8]: the slice [k_begin, k_end) is one contiguous run
@@ -339,9 +347,9 @@ __device__ void prefetch_first_tile(const TileParams &p, int want, SharedCtl &ct
     if (MODE != MODE_SHRINK && tid >= 64 && tid < 64 + R / 8) {
         // B block [R/8][d_out][8]: rows [n_begin, n_end) of rank group j, contiguous
         const int j = tid - 64;
-        const int n0 = min(p.d_out, (int)crank * p.n_slice);
-        const int n1 = min(p.d_out, n0 + p.n_slice);
-        const char *b = slotA + (p.b_offset + ((int64_t)j * p.d_out + n0) * 8) * 2;
+        const int n0 = min(v.d_out, (int)crank * v.n_slice);
+        const int n1 = min(v.d_out, n0 + v.n_slice);
+        const char *b = slotA + (v.b_offset + ((int64_t)j * v.d_out + n0) * 8) * 2;
         const int64_t len = (int64_t)(n1 - n0) * 16;
         for (int64_t off = 0; off < len; off += kChunk)
             prefetch_l2_bulk(b + off, (uint32_t)(len - off < kChunk ? len - off : kChunk));
@@ -349,8 +357,9 @@ __device__ void prefetch_first_tile(const TileParams &p, int want, SharedCtl &ct
 }
 
 template <int RMAX, int MODE, int R, int NT>
-__device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float seg_scale,
-                         SharedCtl &ctl, float *smem_f, uint32_t crank, uint32_t csize, uint32_t nt)
+__device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl, int r_meta,
+                         float seg_scale, SharedCtl &ctl, float *smem_f, uint32_t crank,
+                         uint32_t csize, uint32_t nt)
 {
     constexpr int kThreads = NT, kWarps = NT / 32;
     using RC = RankCfg<R>;
@@ -360,15 +369,15 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float 
     float *wpart = smem_f;
     float *recv = wpart + DC::WPART_FLOATS + (nt & 1) * (kMaxCluster * TM * RMAX);
     float *hfull = wpart + DC::WPART_FLOATS + DC::RECV_FLOATS;
-    const __nv_bfloat16 *slotA = p.pool + (int64_t)tl.slot * p.slot_stride;
-    const __nv_bfloat16 *slotB = slotA + p.b_offset;
+    const __nv_bfloat16 *slotA = v.pool + (int64_t)tl.slot * v.slot_stride;
+    const __nv_bfloat16 *slotB = slotA + v.b_offset;
 
     Slices sl;
     sl.k_begin = min(p.d_in, (int)crank * p.k_slice);
     sl.k_end = min(p.d_in, sl.k_begin + p.k_slice);
     sl.nblk = (MODE == MODE_EXPAND) ? 0 : (sl.k_end - sl.k_begin + 31) / 32;
-    sl.n_begin = min(p.d_out, (int)crank * p.n_slice);
-    sl.n_end = min(p.d_out, sl.n_begin + p.n_slice);
+    sl.n_begin = min(v.d_out, (int)crank * v.n_slice);
+    sl.n_end = min(v.d_out, sl.n_begin + v.n_slice);
     sl.ngrp = (MODE == MODE_SHRINK) ? 0 : (sl.n_end - sl.n_begin + 31) / 32;
     // blocks w, w + 8, ... and groups w, w + 8, ... of this warp, as local indices 0, 1, ...
     const int nb = sl.nblk > warp ? (sl.nblk - warp + kWarps - 1) / kWarps : 0;
@@ -380,8 +389,8 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float 
     int srank = 0;
     float sscale = 0.f;
     if (tid == 0) {
-        srank = p.slot_rank[tl.slot];
-        sscale = p.slot_scale[tl.slot];
+        srank = v.slot_rank[tl.slot];
+        sscale = v.slot_scale[tl.slot];
         if (ctl.stale) srank = -1;   // rank -1 marks a stale generation
     }
     ShrinkOps<R> s0, s1;
@@ -390,16 +399,16 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float 
         load_a<R>(s0, slotA, sl, warp, g, t);
         load_a<R>(s1, slotA, sl, warp + kWarps, g, t);
     }
-    if constexpr (MODE != MODE_SHRINK && RC::EARLY_EXPAND) load_b<R>(e0, slotB, p.d_out, sl, warp, g, t);
+    if constexpr (MODE != MODE_SHRINK && RC::EARLY_EXPAND) load_b<R>(e0, slotB, v.d_out, sl, warp, g, t);
 
     // ---- requests that need the row
     if (g < tl.nvalid && (row_g < 0 || row_g >= p.n_rows)) {
-        if (crank == 0 && warp == 0 && t == 0) report(p, kFlagBadRow);
+        if (crank == 0 && warp == 0 && t == 0) report(v, kFlagBadRow);
         row_g = -1;
     }
     const bool row_ok = row_g >= 0;
     const __nv_bfloat16 *xrow = p.X + (int64_t)(row_ok ? row_g : 0) * p.ldx;
-    __nv_bfloat16 *yrow = p.Y + (int64_t)(row_ok ? row_g : 0) * p.ldy;
+    __nv_bfloat16 *yrow = v.Y + (int64_t)(row_ok ? row_g : 0) * v.ldy;
     if constexpr (MODE != MODE_EXPAND) {
         load_x<R>(s0, xrow, row_ok, sl, warp, t);
         load_x<R>(s1, xrow, row_ok, sl, warp + kWarps, t);
@@ -430,10 +439,10 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float 
         if constexpr (MODE != MODE_SHRINK) {
             // the expand's first groups travel while the cluster sums H
             if constexpr (!RC::EARLY_EXPAND) {
-                load_b<R>(e0, slotB, p.d_out, sl, warp, g, t);
+                load_b<R>(e0, slotB, v.d_out, sl, warp, g, t);
                 load_y<R>(e0, yrow, row_ok, sl, warp, t);
             }
-            load_b<R>(e1, slotB, p.d_out, sl, warp + kWarps, g, t);
+            load_b<R>(e1, slotB, v.d_out, sl, warp + kWarps, g, t);
             load_y<R>(e1, yrow, row_ok, sl, warp + kWarps, t);
         }
 #pragma unroll
@@ -442,10 +451,10 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float 
             wpart[(warp * TM + g) * R + n * 8 + 2 * t + 1] = acc[n][1];
         }
     } else {
-        load_b<R>(e1, slotB, p.d_out, sl, warp + kWarps, g, t);
+        load_b<R>(e1, slotB, v.d_out, sl, warp + kWarps, g, t);
         load_y<R>(e1, yrow, row_ok, sl, warp + kWarps, t);
         if constexpr (!RC::EARLY_EXPAND) {
-            load_b<R>(e0, slotB, p.d_out, sl, warp, g, t);
+            load_b<R>(e0, slotB, v.d_out, sl, warp, g, t);
             load_y<R>(e0, yrow, row_ok, sl, warp, t);
         }
     }
@@ -458,7 +467,7 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float 
     const int r = ctl.slot_rank;
     const bool ok = r > 0 && (p.ranks == nullptr || r_meta == r) && rank_bucket(r) == R;
     if (tid == 0 && crank == 0 && !ok)
-        report(p, r < 0 ? kFlagStaleSlot : r == 0 ? kFlagSlotEmpty : kFlagBadRank);
+        report(v, r < 0 ? kFlagStaleSlot : r == 0 ? kFlagSlotEmpty : kFlagBadRank);
     const int rank = ok ? r : 0;   // a rejected tile reads and writes no H
     const float scale = p.scales ? seg_scale : ctl.slot_scale;
     bool h_ok = true;
@@ -487,7 +496,7 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float 
         }
         // the cluster's partials, summed in CTA order
         const bool landed = mbar_wait_bounded(bar, (nt >> 1) & 1u, 1000000000ull);
-        if (!landed && tid == 0) report(p, kFlagTimeout);
+        if (!landed && tid == 0) report(v, kFlagTimeout);
         for (int e = tid; e < TM * R; e += kThreads) {
             const int i = e / R, j = e % R;
             if (MODE == MODE_SHRINK &&
@@ -540,14 +549,14 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float 
             mma_expand_store<R>(e0, ah, al, scale, yrow, store, sl, warp + i * kWarps, t);
             if (i + 2 < ng) {
                 const int q = warp + (i + 2) * kWarps;
-                load_b<R>(e0, slotB, p.d_out, sl, q, g, t);
+                load_b<R>(e0, slotB, v.d_out, sl, q, g, t);
                 load_y<R>(e0, yrow, row_ok, sl, q, t);
             }
             if (i + 1 < ng) {
                 mma_expand_store<R>(e1, ah, al, scale, yrow, store, sl, warp + (i + 1) * kWarps, t);
                 if (i + 3 < ng) {
                     const int q = warp + (i + 3) * kWarps;
-                    load_b<R>(e1, slotB, p.d_out, sl, q, g, t);
+                    load_b<R>(e1, slotB, v.d_out, sl, q, g, t);
                     load_y<R>(e1, yrow, row_ok, sl, q, t);
                 }
             }
@@ -556,7 +565,11 @@ __device__ void run_tile(const TileParams &p, const Tile &tl, int r_meta, float 
     if constexpr (MODE != MODE_EXPAND) cluster_wait_acquire();
 }
 
-template <int RMAX, int MODE, int NT>
+// FUSED: the launch applies p.n_proj projections that share X and the metadata.  A
+// work item is (tile, projection), projection fastest, so the clusters working on one
+// tile's projections run side by side and its X rows come from HBM once (the later
+// reads hit L2).  Otherwise the only projection is p.proj[0].
+template <int RMAX, int MODE, int NT, bool FUSED>
 __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
     lora_decode_kernel(const __grid_constant__ TileParams p)
 {
@@ -567,8 +580,11 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
     const uint32_t csize = cluster_size();
     const int n_clusters = (int)(gridDim.x / csize);
     const bool reporter = blockIdx.x == 0;
+    const int np = FUSED ? p.n_proj : 1;
 
-    int tile = (int)cluster_index();
+    int item = (int)cluster_index();
+    int tile = FUSED ? item / np : item;
+    int k = FUSED ? item - tile * np : 0;
     // the next launch may start its CTAs now (they wait before touching our results)
     griddep_launch_dependents();
     if constexpr (MODE != MODE_EXPAND) {
@@ -581,12 +597,19 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
         cluster_arrive_release();
         cluster_wait_acquire();
     }
-    if (p.early) prefetch_first_tile<RMAX, MODE, NT>(p, tile, ctl, crank);
+    if (p.early) prefetch_first_tile<RMAX, MODE, NT>(p, p.proj[k], tile, ctl, crank);
     griddep_wait();
-    const int total = scan_tiles<false, NT>(p, tile, ctl, reporter);
+    const int total = scan_tiles<false, NT>(p, p.proj[k].slot_gen, tile, ctl, reporter) * np;
     uint32_t nt = 0;   // tiles done by this CTA (parity of the exchange buffers and barriers)
-    for (; tile < total; tile += n_clusters, ++nt) {
-        if (tile != (int)cluster_index()) scan_tiles<false, NT>(p, tile, ctl, false);
+    for (; item < total; item += n_clusters, ++nt) {
+        if constexpr (FUSED) {
+            tile = item / np;
+            k = item - tile * np;
+        } else {
+            tile = item;
+        }
+        const ProjView &v = p.proj[k];
+        if (item != (int)cluster_index()) scan_tiles<false, NT>(p, v.slot_gen, tile, ctl, false);
         // every CTA of the cluster reads the same metadata and reaches the same tile
         Tile tl;
         tl.seg = ctl.tile[0];
@@ -599,29 +622,29 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
         int R = rank_bucket(r_meta);
         if (p.ranks == nullptr || R == 0 || R > RMAX) {
             __syncthreads();
-            if (tid == 0) ctl.slot_rank = p.slot_rank[tl.slot];
+            if (tid == 0) ctl.slot_rank = v.slot_rank[tl.slot];
             __syncthreads();
             R = rank_bucket(ctl.slot_rank);
             if (R == 0 || R > RMAX) R = 8;   // rejected inside; moves rank-8 bytes
         }
         if (R == 8) {
-            run_tile<RMAX, MODE, 8, NT>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+            run_tile<RMAX, MODE, 8, NT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else if (R == 16) {
             if constexpr (RMAX >= 16)
-                run_tile<RMAX, MODE, 16, NT>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+                run_tile<RMAX, MODE, 16, NT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else if (R == 32) {
             if constexpr (RMAX >= 32)
-                run_tile<RMAX, MODE, 32, NT>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+                run_tile<RMAX, MODE, 32, NT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else {
             if constexpr (RMAX >= 64)
-                run_tile<RMAX, MODE, 64, NT>(p, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+                run_tile<RMAX, MODE, 64, NT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         }
         __syncthreads();   // ctl and the H buffers are rewritten by the next tile
     }
 }
 
 // Clusters of `cluster` CTAs of this kernel resident at once (cached per device).
-template <int RMAX, int MODE, int NT>
+template <int RMAX, int MODE, int NT, bool FUSED>
 cudaError_t active_clusters(int cluster, int &active)
 {
     static std::mutex mu;
@@ -642,14 +665,14 @@ cudaError_t active_clusters(int cluster, int &active)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaOccupancyMaxActiveClusters(&active, lora_decode_kernel<RMAX, MODE, NT>, &cfg);
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&active, lora_decode_kernel<RMAX, MODE, NT, FUSED>, &cfg);
     if (e != cudaSuccess) return e;
     if (active <= 0) return cudaErrorInvalidConfiguration;
     cached[dev][cluster] = active;
     return cudaSuccess;
 }
 
-template <int RMAX, int MODE, int NT>
+template <int RMAX, int MODE, int NT, bool FUSED>
 cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, int active,
                        cudaStream_t stream)
 {
@@ -670,7 +693,7 @@ cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, int 
     cfg.numAttrs = p.early ? 2 : 1;
     const int64_t n = max_tiles < active ? max_tiles : active;
     cfg.gridDim = dim3((unsigned)(n * cluster), 1, 1);
-    return cudaLaunchKernelEx(&cfg, lora_decode_kernel<RMAX, MODE, NT>, p);
+    return cudaLaunchKernelEx(&cfg, lora_decode_kernel<RMAX, MODE, NT, FUSED>, p);
 }
 
 // CTA width.  256 threads keep each warp's operands in one round of loads; when the
@@ -678,24 +701,24 @@ cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, int 
 // long decode segments), 128-thread CTAs let twice as many tiles be in flight, which
 // hides more latency than their second round of loads costs (measured: a 4096 x 4096
 // batch of 60 tiles is 36% slower with 128 threads, batches of 300+ tiles 3-6% faster).
-template <int RMAX, int MODE>
+template <int RMAX, int MODE, bool FUSED = false>
 cudaError_t launch_mode(const TileParams &p, int cluster, int64_t max_tiles, cudaStream_t stream)
 {
     int active = 0;
-    cudaError_t e = active_clusters<RMAX, MODE, 256>(cluster, active);
+    cudaError_t e = active_clusters<RMAX, MODE, 256, FUSED>(cluster, active);
     if (e != cudaSuccess) return e;
     if (2 * max_tiles > 3 * (int64_t)active) {
         int active128 = 0;
-        e = active_clusters<RMAX, MODE, 128>(cluster, active128);
+        e = active_clusters<RMAX, MODE, 128, FUSED>(cluster, active128);
         if (e != cudaSuccess) return e;
         // Early launch with adapter prefetch only pays for batches of about one wave of
         // tiles: with many more, the prefetched slices thrash L2 and the early CTAs
         // hold slots (measured 16% slower on 2048 decode rows over 128 adapters).
         TileParams q = p;
         q.early = 0;
-        return launch_one<RMAX, MODE, 128>(q, cluster, max_tiles, active128, stream);
+        return launch_one<RMAX, MODE, 128, FUSED>(q, cluster, max_tiles, active128, stream);
     }
-    return launch_one<RMAX, MODE, 256>(p, cluster, max_tiles, active, stream);
+    return launch_one<RMAX, MODE, 256, FUSED>(p, cluster, max_tiles, active, stream);
 }
 
 template <int RMAX>
@@ -717,13 +740,16 @@ template <int RMAX, int NT>
 cudaError_t set_attrs_nt()
 {
     cudaError_t e;
-    e = cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_APPLY, NT>,
+    e = cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_APPLY, NT, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX, NT>::SMEM);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_SHRINK, NT>,
+    e = cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_APPLY, NT, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX, NT>::SMEM);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_EXPAND, NT>,
+    e = cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_SHRINK, NT, false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX, NT>::SMEM);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_EXPAND, NT, false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX, NT>::SMEM);
 }
 
@@ -793,6 +819,20 @@ cudaError_t launch_tile_kernel(int mode, int rmax_bucket, const TileParams &p, i
     case 16: return launch_rmax<16>(mode, p, cluster, max_tiles, stream);
     case 32: return launch_rmax<32>(mode, p, cluster, max_tiles, stream);
     case 64: return launch_rmax<64>(mode, p, cluster, max_tiles, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_tile_kernel_fused(int rmax_bucket, const TileParams &p, int cluster,
+                                     int64_t max_items, cudaStream_t stream)
+{
+    if (cluster < 1 || cluster > kMaxCluster || max_items < 1) return cudaErrorInvalidValue;
+    if (p.n_proj < 1 || p.n_proj > kMaxFused) return cudaErrorInvalidValue;
+    switch (rmax_bucket) {
+    case 8: return launch_mode<8, MODE_APPLY, true>(p, cluster, max_items, stream);
+    case 16: return launch_mode<16, MODE_APPLY, true>(p, cluster, max_items, stream);
+    case 32: return launch_mode<32, MODE_APPLY, true>(p, cluster, max_items, stream);
+    case 64: return launch_mode<64, MODE_APPLY, true>(p, cluster, max_items, stream);
     default: return cudaErrorInvalidValue;
     }
 }

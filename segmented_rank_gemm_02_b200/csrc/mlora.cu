@@ -205,6 +205,25 @@ mlora_status ensure_workspace(mlora_pool *pool, size_t bytes, cudaStream_t strea
     return MLORA_OK;
 }
 
+// Whether the batch may hold long segments for the tensor-memory kernels: only if some
+// segment may reach kLongRows (the host's hint, when given, rules them out).
+bool long_path(const mlora_pool *pool, const mlora_segments *s)
+{
+    return s->n_tokens >= kLongRows && pool->d_in % 64 == 0 &&
+           (s->max_segment_rows <= 0 || s->max_segment_rows >= kLongRows) && pool->b_maps_ok;
+}
+
+// The single projection of a launch as entry 0 of the per-projection table.
+void set_single_projection(mlora::TileParams &p)
+{
+    p.n_proj = 1;
+    p.proj[0] = mlora::ProjView{p.pool, p.slot_stride, p.b_offset, p.slot_rank, p.slot_scale, p.slot_gen,
+                                p.status, p.d_out, p.n_slice, p.Y, p.ldy};
+}
+
+mlora_status launch_long(mlora_pool *pool, const mlora_segments *s, int mode, mlora::TileParams &p,
+                         cudaStream_t stream, float *ext_ws, size_t ext_ws_bytes);
+
 // `ext_ws` (optional): caller-provided memory of `ext_ws_bytes` for the long-segment H
 // workspace, used instead of the pool's own (which is then never grown).
 mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::TileParams &p,
@@ -214,11 +233,9 @@ mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::
     const int c = choose_cluster(pool->d_in, pool->d_out);
     p.k_slice = (int32_t)round_up((pool->d_in + c - 1) / c, 32);
     p.n_slice = (int32_t)round_up((pool->d_out + c - 1) / c, 8);
-    // Long segments exist only if some segment may reach kLongRows (the host's hint,
-    // when given, rules them out); the decode kernel then leaves them alone.
-    const bool use_long = s->n_tokens >= kLongRows && pool->d_in % 64 == 0 &&
-                          (s->max_segment_rows <= 0 || s->max_segment_rows >= kLongRows) &&
-                          pool->b_maps_ok;
+    set_single_projection(p);
+    // the decode kernel leaves the long segments alone when the long kernels run
+    const bool use_long = long_path(pool, s);
     p.long_rows = use_long ? kLongRows : 0x7fffffff;
     p.early = use_long ? 0 : 1;
     mlora_status st = prepare_device(pool->device);
@@ -228,7 +245,17 @@ mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::
     cudaError_t e = mlora::launch_tile_kernel(mode, pool->r_bucket_max, p, c, tiles, stream);
     if (e != cudaSuccess) return MLORA_ERR_CUDA;
     if (!use_long) return MLORA_OK;
+    return launch_long(pool, s, mode, p, stream, ext_ws, ext_ws_bytes);
+}
 
+// The long-segment kernels (shrink, then expand) of one projection.
+mlora_status launch_long(mlora_pool *pool, const mlora_segments *s, int mode, mlora::TileParams &p,
+                         cudaStream_t stream, float *ext_ws, size_t ext_ws_bytes)
+{
+    mlora_status st = MLORA_OK;
+    cudaError_t e = cudaSuccess;
+    p.long_rows = kLongRows;
+    p.early = 0;
     const int64_t long_tiles = (int64_t)s->n_tokens / mlora::kLongTileRows + s->n_tokens / kLongRows + 1;
     const int64_t est_tiles = std::max<int64_t>(1, (s->n_tokens + mlora::kLongTileRows - 1) / mlora::kLongTileRows);
     const int rk = std::max(16, pool->r_bucket_max);
@@ -531,6 +558,84 @@ mlora_status mlora_apply(mlora_pool *pool, const mlora_segments *segs, const voi
     p.Y = static_cast<__nv_bfloat16 *>(Y);
     p.ldy = ldy;
     return launch(pool, segs, mlora::MODE_APPLY, p, stream);
+}
+
+mlora_status mlora_apply_multi(mlora_pool *const *pools, int32_t n_proj, const mlora_segments *segs,
+                               const void *X, int64_t ldx, void *const *Y, const int64_t *ldy,
+                               void *stream)
+{
+    if (pools == nullptr || Y == nullptr || ldy == nullptr) return MLORA_ERR_INVALID_ARG;
+    if (n_proj < 1 || n_proj > MLORA_MAX_FUSED) return MLORA_ERR_INVALID_ARG;
+    mlora_pool *const p0 = pools[0];
+    mlora_status st = check_segments(p0, segs);
+    if (st != MLORA_OK) return st;
+    for (int k = 0; k < n_proj; ++k) {
+        const mlora_pool *q = pools[k];
+        if (q == nullptr || q->device != p0->device || q->d_in != p0->d_in || q->n_slots != p0->n_slots)
+            return MLORA_ERR_INVALID_ARG;
+        for (int j = 0; j < k; ++j)
+            if (pools[j] == q || Y[j] == Y[k]) return MLORA_ERR_INVALID_ARG;
+    }
+    if (segs->n_segments == 0 || segs->n_tokens == 0) return MLORA_OK;
+    if (X == nullptr || !aligned16(X) || ldx < p0->d_in || ldx % 8 != 0) return MLORA_ERR_INVALID_ARG;
+    for (int k = 0; k < n_proj; ++k)
+        if (Y[k] == nullptr || !aligned16(Y[k]) || ldy[k] < pools[k]->d_out || ldy[k] % 8 != 0)
+            return MLORA_ERR_INVALID_ARG;
+    DeviceGuard guard(p0->device);
+    if (!guard.ok) return MLORA_ERR_CUDA;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+
+    // one cluster shape for all projections: d_in is shared, each d_out is sliced alike
+    int c = 8, rmax = 8;
+    bool use_long = true;
+    for (int k = 0; k < n_proj; ++k) {
+        c = std::min(c, choose_cluster(p0->d_in, pools[k]->d_out));
+        rmax = std::max(rmax, pools[k]->r_bucket_max);
+        use_long = use_long && long_path(pools[k], segs);
+    }
+    st = prepare_device(p0->device);
+    if (st != MLORA_OK) return st;
+    if (use_long) {
+        // every projection's long-segment workspace first, so that a failure launches nothing
+        const size_t bytes = (size_t)segs->n_tokens * std::max(16, rmax) * sizeof(float);
+        for (int k = 0; k < n_proj; ++k) {
+            std::lock_guard<std::mutex> lock(pools[k]->ws_mutex);
+            st = ensure_workspace(pools[k], bytes, cs);
+            if (st != MLORA_OK) return st;
+        }
+    }
+
+    mlora::TileParams p = base_params(p0, segs);
+    p.X = static_cast<const __nv_bfloat16 *>(X);
+    p.ldx = ldx;
+    p.Y = static_cast<__nv_bfloat16 *>(Y[0]);
+    p.ldy = ldy[0];
+    p.k_slice = (int32_t)round_up((p0->d_in + c - 1) / c, 32);
+    p.n_slice = (int32_t)round_up((p0->d_out + c - 1) / c, 8);
+    p.n_proj = n_proj;
+    for (int k = 0; k < n_proj; ++k) {
+        const mlora_pool *q = pools[k];
+        p.proj[k] = mlora::ProjView{q->buf, q->slot_stride, q->b_offset, q->d_rank, q->d_scale, q->d_gen,
+                                    q->d_status, q->d_out,
+                                    (int32_t)round_up((q->d_out + c - 1) / c, 8),
+                                    static_cast<__nv_bfloat16 *>(Y[k]), ldy[k]};
+    }
+    p.long_rows = use_long ? kLongRows : 0x7fffffff;
+    p.early = use_long ? 0 : 1;
+    const int64_t tiles = (int64_t)segs->n_segments + (int64_t)segs->n_tokens / mlora::kTileRows + 1;
+    if (mlora::launch_tile_kernel_fused(rmax, p, c, tiles * n_proj, cs) != cudaSuccess)
+        return MLORA_ERR_CUDA;
+    if (!use_long) return MLORA_OK;
+    for (int k = 0; k < n_proj; ++k) {
+        mlora::TileParams q = base_params(pools[k], segs);
+        q.X = p.X;
+        q.ldx = ldx;
+        q.Y = static_cast<__nv_bfloat16 *>(Y[k]);
+        q.ldy = ldy[k];
+        st = launch_long(pools[k], segs, mlora::MODE_APPLY, q, cs, nullptr, 0);
+        if (st != MLORA_OK) return st;
+    }
+    return MLORA_OK;
 }
 
 mlora_status mlora_shrink(mlora_pool *pool, const mlora_segments *segs, const void *X,

@@ -35,6 +35,14 @@ def test_header_functions_match_binding(mlora):
     assert _declared_functions() == sorted(mlora.EXPORTS)
 
 
+def test_header_constants_match_binding(mlora):
+    text = open(HEADER).read()
+    defines = dict(re.findall(r"#define (MLORA_\w+)\s+(\d+)u?", text))
+    assert int(defines["MLORA_MAX_FUSED"]) == mlora.MAX_FUSED
+    for name in ("BAD_OFFSETS", "BAD_SLOT", "BAD_RANK", "BAD_ROW", "SLOT_EMPTY", "TIMEOUT", "STALE_SLOT"):
+        assert int(defines["MLORA_FLAG_" + name]) == getattr(mlora, "FLAG_" + name)
+
+
 def test_library_exports_every_declared_symbol(mlora):
     out = subprocess.run(["nm", "-D", "--defined-only", mlora.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
@@ -61,6 +69,13 @@ def test_null_arguments_rejected_without_gpu(mlora):
     assert L.mlora_pool_check(None, None, None) == mlora.ERR_INVALID_ARG
     assert L.mlora_pool_slot_info(None, 0, None, None, None) == mlora.ERR_INVALID_ARG
     assert L.mlora_pool_destroy(None) == mlora.OK
+    # fused apply: no pool list, no pools, too many, or a null pool in the list
+    null2 = (ctypes.c_void_p * 2)(None, None)
+    lds = (ctypes.c_int64 * 2)(0, 0)
+    assert L.mlora_apply_multi(None, 1, ctypes.byref(seg), None, 0, null2, lds, None) == mlora.ERR_INVALID_ARG
+    for n in (0, mlora.MAX_FUSED + 1, 2):
+        assert L.mlora_apply_multi(null2, n, ctypes.byref(seg), None, 0, null2, lds, None) == \
+            mlora.ERR_INVALID_ARG
     h = ctypes.c_void_p()
     assert L.mlora_pool_create(0, 16, 1, 8, ctypes.byref(h)) == mlora.ERR_INVALID_ARG
     assert L.mlora_pool_create(12, 16, 1, 8, ctypes.byref(h)) == mlora.ERR_UNSUPPORTED
