@@ -354,6 +354,28 @@ __device__ void prefetch_first_tile(const TileParams &p, const ProjView &v, int 
         for (int64_t off = 0; off < len; off += kChunk)
             prefetch_l2_bulk(b + off, (uint32_t)(len - off < kChunk ? len - off : kChunk));
     }
+    // the tile's rows from a speculative read of token_indices (checked against n_rows,
+    // so a stale guess still stays inside X and Y): this CTA's slices of their X and
+    // Y0 rows.  L2 is the point of coherence, so lines the previous kernel is still
+    // writing are never served stale.
+    if (tid >= 96 && tid < 96 + TM) {
+        const int pos = p0 + (tid - 96);
+        if (pos >= 0 && pos < ctl.tile[2] && pos < p.n_tokens) {
+            const int row = p.token_indices ? ld_relaxed_s32(p.token_indices + pos) : pos;
+            if (row >= 0 && row < p.n_rows) {
+                if (MODE != MODE_EXPAND) {
+                    const int k0 = min(p.d_in, (int)crank * p.k_slice);
+                    const int k1 = min(p.d_in, k0 + p.k_slice);
+                    if (k1 > k0) prefetch_l2_bulk(p.X + (int64_t)row * p.ldx + k0, (uint32_t)(k1 - k0) * 2);
+                }
+                if (MODE != MODE_SHRINK) {
+                    const int n0 = min(v.d_out, (int)crank * v.n_slice);
+                    const int n1 = min(v.d_out, n0 + v.n_slice);
+                    if (n1 > n0) prefetch_l2_bulk(v.Y + (int64_t)row * v.ldy + n0, (uint32_t)(n1 - n0) * 2);
+                }
+            }
+        }
+    }
 }
 
 template <int RMAX, int MODE, int R, int NT>
