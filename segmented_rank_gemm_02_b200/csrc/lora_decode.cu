@@ -41,12 +41,20 @@
 // tiles, the kernel is launched with programmatic dependent launch: its CTAs may
 // start while the previous kernel in the stream finishes, bring their first tile's
 // adapter slices into L2 from a speculative read of the metadata (adapter weights
-// only change through load_slot), and wait (griddepcontrol.wait) before reading the
-// metadata, X or Y for real.  A stale guess costs bandwidth, never correctness.
+// only change through load_slot) and their rows' X and Y0 slices, and wait
+// (griddepcontrol.wait) before reading the metadata, X or Y for real.  A stale
+// guess costs bandwidth, never correctness.  In such launches a cluster with a
+// second tile also prefetches that tile's adapter slices while it runs the first.
+//
+// Fused projections.  With FUSED, one launch applies several projections that share
+// X and the metadata (q/k/v, gate/up), each with its own pool and output; a work
+// item is (tile, projection), projection fastest, so a tile's X rows are read from
+// HBM once.
 //
 // Invalid metadata never traps: bad segments and rows are skipped and flagged in
 // the status word; every CTA of a cluster reaches the same decisions, so cluster
-// barriers always match.  The kernel has no spin-waits.
+// barriers always match.  Its one wait on other CTAs (the partial-H exchange) is
+// bounded: on expiry it flags a timeout and leaves the tile's rows alone.
 #include <climits>
 #include <mutex>
 
@@ -132,14 +140,46 @@ __device__ __forceinline__ uint2 ldg_nc2(const void *p)
     return __ldg(reinterpret_cast<const uint2 *>(p));
 }
 
+// L2 prefetch, by one thread, of this CTA's slices of an adapter's A and B blocks
+// (slot, rank bucket R): every address stays inside the pool.
+template <int MODE>
+__device__ __forceinline__ void prefetch_slices_one(const TileParams &p, const ProjView &v, int slot, int R,
+                                                    uint32_t crank)
+{
+    constexpr uint32_t kChunk = 32768;
+    const char *slotA = reinterpret_cast<const char *>(v.pool + (int64_t)slot * v.slot_stride);
+    if (MODE != MODE_EXPAND) {
+        const int k0 = min(p.d_in, (int)crank * p.k_slice);
+        const int k1 = min(p.d_in, k0 + p.k_slice);
+        const int64_t beg = (int64_t)k0 * R * 2, len = (int64_t)(k1 - k0) * R * 2;
+        for (int64_t off = 0; off < len; off += kChunk)
+            prefetch_l2_bulk(slotA + beg + off, (uint32_t)(len - off < kChunk ? len - off : kChunk));
+    }
+    if (MODE != MODE_SHRINK) {
+        const int n0 = min(v.d_out, (int)crank * v.n_slice);
+        const int n1 = min(v.d_out, n0 + v.n_slice);
+        const int64_t len = (int64_t)(n1 - n0) * 16;
+        for (int j = 0; j < R / 8; ++j) {
+            const char *b = slotA + (v.b_offset + ((int64_t)j * v.d_out + n0) * 8) * 2;
+            for (int64_t off = 0; off < len; off += kChunk)
+                prefetch_l2_bulk(b + off, (uint32_t)(len - off < kChunk ? len - off : kChunk));
+        }
+    }
+}
+
 // Block-wide scan of per-segment tile counts.  Returns the number of tiles; if
 // tile `want` exists, its segment and first position are left in ctl.tile.
 // SPEC: a speculative pass made before the grids this launch depends on have
 // finished (the metadata may still change): relaxed loads, nothing reported.
 // slot_gen: generations of the pool the tile will read (ctl.stale).
-template <bool SPEC, int NT>
-__device__ int scan_tiles(const TileParams &p, const uint32_t *slot_gen, int want, SharedCtl &ctl,
-                          bool reporter)
+// want2 (-1: none): the cluster's next tile, of projection v2.  In early launches
+// (batches of about one wave of tiles) the thread that finds it prefetches this CTA's
+// slices of that tile's adapter into L2, so that they travel while the current tile
+// runs.  Batches of several waves skip it: there the prefetches thrashed L2
+// (measured 11% slower on 2048 decode rows of 8192-wide projections).
+template <bool SPEC, int NT, int MODE, int RMAX>
+__device__ int scan_tiles(const TileParams &p, const uint32_t *slot_gen, int want, int want2,
+                          const ProjView &v2, SharedCtl &ctl, bool reporter)
 {
     constexpr int kThreads = NT, kWarps = NT / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -199,6 +239,12 @@ __device__ int scan_tiles(const TileParams &p, const uint32_t *slot_gen, int wan
             ctl.tile[4] = rk;
             ctl.seg_scale = sc;
             if constexpr (!SPEC) ctl.stale = p.generations && slot_gen[a] != p.generations[g];
+        }
+        if constexpr (RMAX <= 16) {   // (larger pools: more register spills than it saved)
+            if (p.early && cnt > 0 && want2 >= lo && want2 < running + incl && p.ranks != nullptr) {
+                const int R2 = rank_bucket(rk);
+                if (R2 > 0 && R2 <= RMAX) prefetch_slices_one<MODE>(p, v2, a, R2, cluster_rank());
+            }
         }
         running += total;
         __syncthreads();   // ctl.scan is rewritten by the next chunk
@@ -320,18 +366,14 @@ __device__ __forceinline__ void mma_expand_store(const ExpandOps<R> &o, const ui
 // previous kernel.  The metadata read here may be stale; a wrong guess only costs
 // bandwidth (every address stays inside the pool), never correctness, since the
 // tile's real loads come after griddep_wait.
-template <int RMAX, int MODE, int NT>
-__device__ void prefetch_first_tile(const TileParams &p, const ProjView &v, int want, SharedCtl &ctl,
-                                    uint32_t crank)
+// L2 prefetch of this CTA's slices of one tile's adapter (slot, rank bucket R) and
+// of the line of token_indices at its first position: every address is inside the
+// pool or the metadata whatever the values, so the caller may pass a guess.
+template <int MODE>
+__device__ void prefetch_slices(const TileParams &p, const ProjView &v, int slot, int R, int p0,
+                                uint32_t crank)
 {
-    if (want >= scan_tiles<true, NT>(p, v.slot_gen, want, ctl, false)) return;
     const int tid = threadIdx.x;
-    const int slot = ctl.tile[3];
-    if (slot < 0 || slot >= p.n_slots) return;
-    int R = rank_bucket(ctl.tile[4]);
-    if (p.ranks == nullptr || R == 0 || R > RMAX) R = rank_bucket(ld_relaxed_s32(v.slot_rank + slot));
-    if (R == 0 || R > RMAX) return;
-    const int p0 = ctl.tile[1];
     if (tid == 32 && p.token_indices != nullptr && p0 >= 0 && p0 < p.n_tokens)
         prefetch_l2_line(p.token_indices + p0);
     const char *slotA = reinterpret_cast<const char *>(v.pool + (int64_t)slot * v.slot_stride);
@@ -354,6 +396,21 @@ __device__ void prefetch_first_tile(const TileParams &p, const ProjView &v, int 
         for (int64_t off = 0; off < len; off += kChunk)
             prefetch_l2_bulk(b + off, (uint32_t)(len - off < kChunk ? len - off : kChunk));
     }
+}
+
+template <int RMAX, int MODE, int NT>
+__device__ void prefetch_first_tile(const TileParams &p, const ProjView &v, int want, SharedCtl &ctl,
+                                    uint32_t crank)
+{
+    if (want >= scan_tiles<true, NT, MODE, RMAX>(p, v.slot_gen, want, -1, v, ctl, false)) return;
+    const int tid = threadIdx.x;
+    const int slot = ctl.tile[3];
+    if (slot < 0 || slot >= p.n_slots) return;
+    int R = rank_bucket(ctl.tile[4]);
+    if (p.ranks == nullptr || R == 0 || R > RMAX) R = rank_bucket(ld_relaxed_s32(v.slot_rank + slot));
+    if (R == 0 || R > RMAX) return;
+    const int p0 = ctl.tile[1];
+    prefetch_slices<MODE>(p, v, slot, R, p0, crank);
     // the tile's rows from a speculative read of token_indices (checked against n_rows,
     // so a stale guess still stays inside X and Y): this CTA's slices of their X and
     // Y0 rows.  L2 is the point of coherence, so lines the previous kernel is still
@@ -621,7 +678,10 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
     }
     if (p.early) prefetch_first_tile<RMAX, MODE, NT>(p, p.proj[k], tile, ctl, crank);
     griddep_wait();
-    const int total = scan_tiles<false, NT>(p, p.proj[k].slot_gen, tile, ctl, reporter) * np;
+    const int item2 = item + n_clusters;   // this cluster's next work item
+    const int total = scan_tiles<false, NT, MODE, RMAX>(p, p.proj[k].slot_gen, tile, item2 / np,
+                                                        p.proj[FUSED ? item2 % np : 0], ctl, reporter) *
+                      np;
     uint32_t nt = 0;   // tiles done by this CTA (parity of the exchange buffers and barriers)
     for (; item < total; item += n_clusters, ++nt) {
         if constexpr (FUSED) {
@@ -631,7 +691,11 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
             tile = item;
         }
         const ProjView &v = p.proj[k];
-        if (item != (int)cluster_index()) scan_tiles<false, NT>(p, v.slot_gen, tile, ctl, false);
+        if (item != (int)cluster_index()) {
+            const int next = item + n_clusters;
+            scan_tiles<false, NT, MODE, RMAX>(p, v.slot_gen, tile, next / np, p.proj[FUSED ? next % np : 0],
+                                              ctl, false);
+        }
         // every CTA of the cluster reads the same metadata and reaches the same tile
         Tile tl;
         tl.seg = ctl.tile[0];
