@@ -4,23 +4,31 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
 
 A step applies the LoRA delta of one batch to every projection the workload names
-(mlora_apply per projection, inputs resident in HBM).  The timed region replays a
-CUDA graph holding exactly K steps that cycle through enough independent buffer
-sets (pool, X, Y) to exceed twice the L2 cache, bracketed by CUDA events on the
-launching stream.  Metric: LoRA delta tokens/s (adapter rows per second), plus
-achieved HBM GB/s of the kernel against the measured copy peak.
+(inputs resident in HBM).  Each timed region replays a CUDA graph holding exactly K
+steps that cycle through enough independent buffer sets (pools, X, Y) to exceed
+twice the L2 cache, bracketed by CUDA events on the launching stream; the region is
+taken R times (R >= 5) and the line reports the median, with the spread.  Metric:
+LoRA delta tokens/s (adapter rows per second), plus achieved HBM GB/s of the step
+against the measured copy peak.
 
-Default workload: the Llama-3-8B q_proj decode batch (d 4096, 64 rank-16 slots,
-256 rows, Zipf(1.1) adapters, 10% base-only).  --config selects the others:
-1 tiny, 2 qproj_decode, 3 qkv_prefill, 4 mixed_mlp, 5 block70b.
+Default workload: the 70B-shaped decoder block (d 8192, 2048 decode rows over 128
+rank-16 adapters, all seven projections), the largest single-GPU configuration,
+with the projections that read the same input rows (q/k/v, gate/up) applied by one
+mlora_apply_multi call each.  --config selects another workload for the headline:
+1 tiny, 2 qproj_decode, 3 qkv_prefill, 4 mixed_mlp, 5 block70b; --no-fused applies
+every projection with its own mlora_apply.  With the default headline the line
+also carries ``per_config``: the same measurement for workloads 2, 3 and 4 (and a
+parity-only entry for 1), so one run covers every workload.
 
---fused applies the projections of a layer that read the same input rows (q, k
-and v; gate and up) with one mlora_apply_multi call each, those projections then
-sharing one X; the algorithmic bytes count that X once.
+Next to the steady-state step (consecutive steps overlap only as far as programmatic
+dependent launch lets the next step's kernels start early) the line reports the
+isolated step (one step after an L2 flush, nothing to overlap with) and the first
+step of the process.
 
-Under torchrun each rank runs its own batch of the same shape (independent
-problems, no collective on the data path); value = all ranks' tokens / the
-slowest rank's time.  --impl reference times the fp64 CPU oracle instead.
+With --gpus N > 1 outside torchrun the script relaunches itself under
+torch.distributed.run with N ranks.  Each rank runs its own batch of the same shape
+(independent problems, no collective on the data path); value = all ranks' tokens /
+the slowest rank's time.  --impl reference times the fp64 CPU oracle instead.
 """
 from __future__ import annotations
 
@@ -43,7 +51,8 @@ import numpy as np
 
 METRIC = "LoRA delta tokens/s and achieved HBM GB/s (% roofline), decode & prefill"
 UNIT = "delta tokens/s"
-DEFAULT_CONFIG = 2
+DEFAULT_CONFIG = 5
+PER_CONFIG = (1, 2, 3, 4)
 L2_FALLBACK = 126 * 2**20
 
 REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -104,6 +113,21 @@ def workload_facts(W, groups=None) -> dict:
         flops += int(2 * r_rows.sum() * (d_in + d_out))
     return {"adapter_rows": n_l, "distinct_adapters": int(distinct.size),
             "bytes": total_bytes, "flops": flops, "per_projection": per_proj}
+
+
+def workload_config(W, facts, groups, world: int) -> dict:
+    """The ``config`` object of a bench line: the workload and how it is applied."""
+    tokens = facts["adapter_rows"]
+    return {
+        "workload": W.name, "projections": [p[0] for p in W.proj_shapes],
+        "shapes": [[p[1], p[2]] for p in W.proj_shapes], "rows": W.n_rows,
+        "adapter_rows": tokens, "slots": W.n_slots,
+        "distinct_adapters": facts["distinct_adapters"],
+        "ranks": sorted(set(int(r) for r in W.slot_rank[W.referenced_slots])),
+        "global_batch": tokens * world,
+        "parallelism": f"replicas x{world} (independent batches)",
+        "fused": [[W.proj_shapes[j][0] for j in g] for g in groups if len(g) > 1],
+    }
 
 
 def max_over_ranks(x: float, device=None) -> float:
@@ -244,16 +268,18 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- CPU oracle
 
-def cpu_oracle_rate(W, seconds: float, steps: int = 0):
-    """Time the fp64 oracle on a bounded sample of the workload (tokens/s)."""
+def cpu_oracle_rate(W, seconds: float, steps: int = 0, n_threads: int = 0):
+    """Time the fp64 oracle on a bounded sample of the workload (tokens/s).
+    ``n_threads`` 0 = every host core (OpenMP's default)."""
     import oracle
+    threads = n_threads or oracle.max_threads()
     projs = [W.projection(j) for j in range(len(W.proj_shapes))]
     adapter_rows = np.nonzero(W.row_slot >= 0)[0]
     # per-row cost estimate on a small sample
     probe = adapter_rows[: min(16, adapter_rows.size)]
     t = time.perf_counter()
     for p in projs:
-        oracle.reference(W, p, rows=probe)
+        oracle.reference(W, p, rows=probe, n_threads=threads)
     per_row = (time.perf_counter() - t) / max(1, probe.size)
     budget = seconds / max(1, steps) if steps else seconds
     n_rows = int(max(1, min(adapter_rows.size, budget / max(per_row, 1e-9))))
@@ -263,7 +289,7 @@ def cpu_oracle_rate(W, seconds: float, steps: int = 0):
     reps = 0
     while True:
         for p in projs:
-            oracle.reference(W, p, rows=rows)
+            oracle.reference(W, p, rows=rows, n_threads=threads)
         done += rows.size
         reps += 1
         el = time.perf_counter() - t0
@@ -275,22 +301,43 @@ def cpu_oracle_rate(W, seconds: float, steps: int = 0):
     el = time.perf_counter() - t0
     sample = (f"first {rows.size} of {adapter_rows.size} adapter rows of {W.name}, all "
               f"{len(projs)} projection(s), {reps} pass(es)")
-    return done / el, el, sample, oracle.max_threads()
+    return done / el, el, sample, threads
 
 
 # --------------------------------------------------------------------------- GPU arm
 
-def run_ours(args, rank: int, world: int, device_index: int):
+class Repeated:
+    """Median and spread of R timings of the same region (milliseconds)."""
+
+    def __init__(self, ms):
+        self.ms = sorted(float(m) for m in ms)
+
+    @property
+    def median(self) -> float:
+        return statistics.median(self.ms)
+
+    def summary(self, per: int = 1) -> dict:
+        return {"median": self.median / per, "min": self.ms[0] / per, "max": self.ms[-1] / per,
+                "n": len(self.ms)}
+
+
+def flush_l2(buf) -> None:
+    """Overwrite a buffer larger than L2 on the current stream (evicts cached lines)."""
+    buf.add_(1)
+
+
+def measure(args, cfg: int, fused: bool, rank: int, world: int, device_index: int,
+            e2e_seconds: float, repeats: int, cpu: bool) -> dict:
+    """One workload: parity on sampled rows, then the steady-state K-step graph R
+    times, the isolated step, the first step, and the end-to-end leg."""
     import torch
     import oracle
     import segmented_rank_gemm_02_b200 as mlora
     import workloads as wl
-    from segmented_rank_gemm_02_b200 import staging
 
-    torch.cuda.set_device(device_index)
     dev = torch.device("cuda", device_index)
-    W = wl.make(args.config)
-    groups = fusion_groups(W, args.fused)
+    W = wl.make(cfg)
+    groups = fusion_groups(W, fused)
     leader = group_leaders(groups)
     facts = workload_facts(W, groups)
     projs = [W.projection(j) for j in range(len(W.proj_shapes))]
@@ -298,7 +345,6 @@ def run_ours(args, rank: int, world: int, device_index: int):
     projs = [p if leader[j] == j else dataclasses.replace(p, X=projs[leader[j]].X)
              for j, p in enumerate(projs)]
     meta = mlora.build_segments(W.row_slot)
-    n_proj = len(projs)
 
     # device copies of the adapters, used to fill every pool of the ring
     dA = [{s: mlora.as_bf16_tensor(p.A[s], dev) for s in p.A} for p in projs]
@@ -331,12 +377,10 @@ def run_ours(args, rank: int, world: int, device_index: int):
         l2 = L2_FALLBACK
     n_sets = max(1, math.ceil(2 * l2 / set_bytes))
     sets = [new_set() for _ in range(n_sets)]
+    flush_buf = torch.zeros(2 * l2 // 4, dtype=torch.float32, device=dev)
     torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device=dev)
 
-    # parity on sampled rows of a fresh set (outside any timed region)
-    rows = np.unique(np.concatenate([meta["token_indices"][meta["offsets"][:-1]],
-                                     np.nonzero(W.row_slot >= 0)[0][:8]]))
-    rows = rows[W.row_slot[rows] >= 0][:48]
     def apply_group(entries, g, stream=None, segs=None):
         if len(g) == 1:
             e = entries[g[0]]
@@ -346,6 +390,28 @@ def run_ours(args, rank: int, world: int, device_index: int):
             mlora.apply_multi([entries[j]["pool"] for j in g], segs or e0["segs"], e0["X"],
                               [entries[j]["Y"] for j in g], stream=stream)
 
+    def step(k):
+        for g in groups:
+            apply_group(sets[k % n_sets], g, stream=stream)
+
+    # the first step of the process on this workload (cold caches, first launches)
+    with torch.cuda.stream(stream):
+        flush_l2(flush_buf)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step(0)
+        e1.record(stream)
+    stream.synchronize()
+    first_ms = e0.elapsed_time(e1)
+    for j in range(len(projs)):
+        sets[0][j]["Y"].copy_(Y0[j])
+    torch.cuda.synchronize()
+
+    # parity on sampled rows of a fresh set (outside any timed region)
+    rows = np.unique(np.concatenate([meta["token_indices"][meta["offsets"][:-1]],
+                                     np.nonzero(W.row_slot >= 0)[0][:8],
+                                     meta["token_indices"][np.maximum(meta["offsets"][1:] - 1, 0)]]))
+    rows = rows[W.row_slot[rows] >= 0][:96]
     worst = 0.0
     for g in groups:
         apply_group(sets[0], g)
@@ -357,12 +423,6 @@ def run_ours(args, rank: int, world: int, device_index: int):
             worst = max(worst, float(np.max(np.abs(got - ref) / (1e-2 * (1 + np.abs(ref))))))
             e["Y"].copy_(Y0[j])
     torch.cuda.synchronize()
-
-    stream = torch.cuda.Stream(device=dev)
-
-    def step(k):
-        for g in groups:
-            apply_group(sets[k % n_sets], g, stream=stream)
 
     # warm-up steps (eager), then capture exactly K steps into one graph
     with torch.cuda.stream(stream):
@@ -379,79 +439,98 @@ def run_ours(args, rank: int, world: int, device_index: int):
         graph.replay()   # first replay uploads the graph; not timed
     stream.synchronize()
     per_apply = (launches / (args.steps * len(groups))) if launches else None
-    call = "mlora_apply_multi / mlora_apply" if args.fused else "mlora_apply"
+    call = "mlora_apply_multi / mlora_apply" if fused and any(len(g) > 1 for g in groups) \
+        else "mlora_apply"
     kernel_desc = (f"{call}: lora_decode_kernel" if per_apply == 1 else
                    f"{call}: lora_decode_kernel + long_shrink_kernel + long_expand_kernel"
-                   if per_apply == 3 else call)
+                   if per_apply and per_apply >= 3 else call)
 
     dist = None
     if world > 1:
         import torch.distributed as dist
 
-    def timed():
+    def timed_once():
         start = torch.cuda.Event(enable_timing=True)
         end = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            graph.replay()
+            end.record(stream)
+        stream.synchronize()
+        return start.elapsed_time(end)
+
+    def timed_region():
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
         torch.cuda.synchronize()
         t0 = time.perf_counter()
-        with torch.cuda.stream(stream):
-            start.record(stream)
-            graph.replay()
-            end.record(stream)
-        torch.cuda.synchronize()
+        ms = [timed_once() for _ in range(repeats)]
         t1 = time.perf_counter()
         if dist:
             dist.barrier()
-        return start.elapsed_time(end), t0, t1
+        return Repeated(ms), t0, t1
 
     with ClockSampler(device_index) as clk:
-        ms, t0, t1 = timed()
+        rep, t0, t1 = timed_region()
     clocks = clk.summary(t0, t1)
     if set(clocks.get("reasons", [])) & BAD_REASONS:
         with ClockSampler(device_index) as clk:
-            ms, t0, t1 = timed()
+            rep, t0, t1 = timed_region()
         clocks = clk.summary(t0, t1)
         clocks["remeasured"] = True
-
-    ms_max = max_over_ranks(ms, dev)
+    ms_med = max_over_ranks(rep.median, dev)
     del graph
 
-    # end to end through the public API with host buffers: host grouping, H2D of the
-    # metadata, X and Y0 from pinned memory, mlora_apply, D2H of Y
-    e2e = run_e2e(args, W, projs, meta, sets[0], dev, stream, world, groups, apply_group)
+    # the isolated step: one step after an L2 flush (no earlier step to overlap with);
+    # the flush kernel in front keeps the host's launch time out of the interval
+    g1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1, stream=stream):
+        step(0)
+    iso = []
+    for _ in range(max(5, repeats)):
+        with torch.cuda.stream(stream):
+            flush_l2(flush_buf)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g1.replay()
+            b.record(stream)
+        stream.synchronize()
+        iso.append(a.elapsed_time(b))
+    del g1
+    iso = Repeated(iso)
+    iso_med = max_over_ranks(iso.median, dev)
+
+    e2e = run_e2e(args, W, projs, meta, sets[0], dev, stream, world, groups, apply_group,
+                  e2e_seconds) if e2e_seconds > 0 else None
 
     tokens = facts["adapter_rows"]
     steps = args.steps
-    sec = ms_max / 1e3
+    sec = ms_med / 1e3
     value = whole_job_rate(tokens, steps, world, sec)
-    per_launch_s = (ms / 1e3) / steps
+    per_step_s = (rep.median / 1e3) / steps
     peaks = measured_peaks()
-    achieved = facts["bytes"] / per_launch_s / 1e9
-    traffic = recorded_traffic(W.name + ("_fused" if args.fused else ""))
-    result = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
-        "warmup": args.warmup, "ms_per_step": ms_max / steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {
-            "workload": W.name, "projections": [p[0] for p in W.proj_shapes],
-            "shapes": [[p[1], p[2]] for p in W.proj_shapes], "rows": W.n_rows,
-            "adapter_rows": tokens, "slots": W.n_slots,
-            "distinct_adapters": facts["distinct_adapters"],
-            "ranks": sorted(set(int(r) for r in W.slot_rank[W.referenced_slots])),
-            "global_batch": tokens * world, "parallelism": f"replicas x{world} (independent batches)",
+    achieved = facts["bytes"] / per_step_s / 1e9
+    traffic = recorded_traffic(W.name + ("_fused" if fused and any(len(g) > 1 for g in groups)
+                                         else ""))
+    out = {
+        "workload": W.name, "value": value, "unit": UNIT, "ms_per_step": ms_med / steps,
+        "us_per_step": rep.summary(steps / 1e3),
+        "isolated_us_per_step": iso_med * 1e3,
+        "isolated_spread_us": iso.summary(1 / 1e3),
+        "first_step_us": first_ms * 1e3,
+        "config": dict(workload_config(W, facts, groups, world), **{
             "l2": f"rotating {n_sets} buffer set(s) of {set_bytes / 2**20:.0f} MiB "
                   f"({n_sets * set_bytes / 2**20:.0f} MiB > 2x {l2 / 2**20:.0f} MiB L2)",
-            "timing": "one CUDA graph of exactly K steps, CUDA events on its stream",
-            "fused": [[W.proj_shapes[j][0] for j in g] for g in groups if len(g) > 1],
-        },
+            "timing": f"one CUDA graph of exactly K steps, CUDA events on its stream, "
+                      f"taken {repeats} times: median (spread in us_per_step)"}),
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
             "peak_source": peaks["source"], "algorithmic_bytes_per_step": facts["bytes"],
             "flops_per_step": facts["flops"],
-            "tensor_frac": facts["flops"] / per_launch_s / 1e12 / peaks["bf16_tflops"],
+            "tensor_frac": facts["flops"] / per_step_s / 1e12 / peaks["bf16_tflops"],
+            "isolated_frac": facts["bytes"] / (iso.median / 1e3) / 1e9 / peaks["hbm_gbs"],
             "kernel": kernel_desc,
         },
         "e2e": e2e,
@@ -459,17 +538,87 @@ def run_ours(args, rank: int, world: int, device_index: int):
         "clocks": clocks,
         "parity": {"rows_checked": int(rows.size), "max_err_over_tolerance": worst},
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if cpu:
         rate, el, sample, cores = cpu_oracle_rate(W, args.cpu_seconds)
-        result["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                  "sample": sample, "seconds": el}
+        out["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": sample, "seconds": el}
     for s in sets:
         for e in s:
             e["pool"].close()
+    del sets, flush_buf
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
+def parity_only(cfg: int, device_index: int) -> dict:
+    """Every row of a small workload against the oracle, plus the oracle's one-thread
+    rate on it (the workload is far too small to time the GPU meaningfully)."""
+    import torch
+    import oracle
+    import segmented_rank_gemm_02_b200 as mlora
+    import workloads as wl
+    from segmented_rank_gemm_02_b200 import staging
+    dev = torch.device("cuda", device_index)
+    W = wl.make(cfg)
+    worst = 0.0
+    for j in range(len(W.proj_shapes)):
+        p = W.projection(j)
+        st = staging.upload(W, p, dev)
+        mlora.apply(st["pool"], st["segs"], st["X"], st["Y"])
+        assert st["pool"].check() == 0
+        got = oracle.bf16_to_f64(mlora.bf16_bits(st["Y"]))
+        ref = oracle.reference(W, p)
+        worst = max(worst, float(np.max(np.abs(got - ref) / (1e-2 * (1 + np.abs(ref))))))
+        base = W.row_slot < 0
+        assert np.array_equal(mlora.bf16_bits(st["Y"])[base], p.Y0[base])
+        st["pool"].close()
+    return {"workload": W.name, "parity": {"rows_checked": W.n_rows, "max_err_over_tolerance": worst}}
+
+
+def run_ours(args, rank: int, world: int, device_index: int):
+    import torch
+    torch.cuda.set_device(device_index)
+    cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    head = measure(args, args.config, args.fused, rank, world, device_index, args.e2e_seconds,
+                   args.repeats, cpu)
+    result = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": head["config"], "roofline": head["roofline"],
+        "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+        "parity": head["parity"], "us_per_step": head["us_per_step"],
+        "isolated_us_per_step": head["isolated_us_per_step"],
+        "isolated_spread_us": head["isolated_spread_us"], "first_step_us": head["first_step_us"],
+    }
+    if "cpu_baseline" in head:
+        result["cpu_baseline"] = head["cpu_baseline"]
+    if args.per_config and world == 1:
+        per = {}
+        for cfg in PER_CONFIG:
+            if cfg == args.config:
+                continue
+            if cfg == 1:
+                e = parity_only(cfg, device_index)
+            else:
+                e = measure(args, cfg, args.fused, rank, world, device_index,
+                            args.per_config_e2e_seconds, args.repeats, False)
+                for k in ("config", "clocks"):
+                    e.pop(k)
+            if cfg in (1, 2) and rank == 0 and not args.no_cpu_baseline:
+                import workloads as wl
+                rate, el, sample, cores = cpu_oracle_rate(wl.make(cfg), min(args.cpu_seconds, 3.0),
+                                                          n_threads=1)
+                e["cpu_one_thread"] = {"value": rate, "unit": UNIT, "cores": cores,
+                                       "kind": "oracle", "sample": sample, "seconds": el}
+            per[str(cfg)] = e
+        result["per_config"] = per
     return result
 
 
-def run_e2e(args, W, projs, meta0, entries, dev, stream, world, groups, apply_group):
+def run_e2e(args, W, projs, meta0, entries, dev, stream, world, groups, apply_group,
+            e2e_seconds):
     """The same step through the public API with host buffers, pipelined the way a
     serving loop would run it: step k's host grouping and H2D copies (copy-in
     stream) overlap step k-1's apply (compute stream) and step k-2's D2H copy
@@ -570,7 +719,7 @@ def run_e2e(args, W, projs, meta0, entries, dev, stream, world, groups, apply_gr
         one_step()
     torch.cuda.synchronize()
     est = (time.perf_counter() - t) / 4
-    steps = int(max(3, min(args.steps, args.e2e_seconds / max(est, 1e-6))))
+    steps = int(max(3, min(args.steps, e2e_seconds / max(est, 1e-6))))
     steps = int(max_over_ranks(steps, dev))   # the same count on every rank
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
@@ -676,7 +825,8 @@ def run_slot_load(args):
 def run_reference(args, rank: int, world: int):
     import workloads as wl
     W = wl.make(args.config)
-    facts = workload_facts(W)
+    groups = fusion_groups(W, args.fused)
+    facts = workload_facts(W, groups)
     budget = float(args.cpu_seconds) if args.cpu_seconds else 60.0
     # warm-up passes are bounded samples too (not timed)
     if args.warmup:
@@ -687,33 +837,64 @@ def run_reference(args, rank: int, world: int):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el * 1e3 / max(1, args.steps), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": W.name, "adapter_rows": facts["adapter_rows"],
-                   "projections": [p[0] for p in W.proj_shapes]},
+        "config": workload_config(W, facts, groups, world),
         "cpu_baseline": {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
+def relaunch(argv, gpus: int) -> int:
+    """Run this script under torch.distributed.run with ``gpus`` ranks on this node."""
+    import socket
+    import subprocess
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={gpus}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
 def main(argv=None) -> int:
+    argv = list(sys.argv[1:] if argv is None else argv)
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--repeats", type=int, default=7,
+                    help="timed K-step regions per measurement (median reported); at least 5")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--e2e-seconds", type=float, default=5.0)
+    ap.add_argument("--e2e-seconds", type=float, default=3.0)
+    ap.add_argument("--per-config-e2e-seconds", type=float, default=1.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--fused", action="store_true",
-                    help="one mlora_apply_multi per group of projections reading the same X")
+    ap.add_argument("--fused", action=argparse.BooleanOptionalAction, default=True,
+                    help="one mlora_apply_multi per group of projections reading the same X "
+                         "(default); --no-fused: one mlora_apply per projection")
+    ap.add_argument("--per-config", action=argparse.BooleanOptionalAction, default=None,
+                    help="also measure the other workloads (default: with the default headline)")
     ap.add_argument("--slot-load", action="store_true",
                     help="measure adapter slot loads instead of the apply step (one GPU)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.repeats < 5:
+        ap.error("--repeats must be at least 5")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    if args.per_config is None:
+        args.per_config = "--config" not in " ".join(argv)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is None and args.gpus > 1:
+        return relaunch(argv, args.gpus)
+    world = int(env_world or "1")
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+        return 2
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 

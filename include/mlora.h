@@ -108,9 +108,16 @@ typedef struct {
 
 /*
  * Create a pool of n_slots adapter slots for one projection (d_in -> d_out) with
- * ranks up to r_max (1..64).  Allocates n_slots * bucket(r_max) * (d_in + d_out)
- * bf16 elements of device memory on the current device; all slots start empty.
- * Returns MLORA_ERR_OUT_OF_MEMORY if the allocation fails.
+ * ranks up to r_max (1..64): one pre-allocated buffer of fixed-size slots, so a
+ * slot's address is base + slot * stride (page "LoRA/QLoRA multi-tenant serving",
+ * ybb.press, section 1.1 on the adapter pool and unified size alignment; page
+ * "Multi-LoRA Serving: adapter batching", section "Why the adapter cache needs
+ * tiers", on keeping hot adapters resident in GPU memory).  Allocates
+ * n_slots * bucket(r_max) * (d_in + d_out) bf16 elements of device memory on the
+ * current device; all slots start empty.  It also reserves, once per device, the
+ * scratch array of mlora_apply_noalloc.  Returns MLORA_ERR_OUT_OF_MEMORY if an
+ * allocation fails, MLORA_ERR_UNSUPPORTED without an sm_100 device or for r_max > 64
+ * or d_in, d_out not multiples of 8.
  */
 mlora_status mlora_pool_create(int32_t d_in, int32_t d_out, int32_t n_slots, int32_t r_max,
                                mlora_pool **out);
@@ -167,7 +174,10 @@ mlora_status mlora_pool_shape(const mlora_pool *pool, int32_t *d_in, int32_t *d_
 mlora_status mlora_pool_check(mlora_pool *pool, void *stream, uint32_t *flags);
 
 /*
- * Shrink alone: H[p, 0:r] = X[t_p, :] A_a^T for every grouped position p of every
+ * Shrink alone (page "Multi-LoRA Serving: adapter batching", section "What metadata
+ * a segmented kernel needs", the shrink step; page "S-LoRA deep dive", section 3 on
+ * the segmented gather + GEMM):
+ * H[p, 0:r] = X[t_p, :] A_a^T for every grouped position p of every
  * adapter segment, fp32, grouped order (row stride ldh >= r).  X is device bf16
  * [n_rows, d_in] (row stride ldx); H is device fp32 [n_tokens, ldh].  Entries of
  * base or rejected segments and columns >= r are not written.
@@ -176,7 +186,10 @@ mlora_status mlora_shrink(mlora_pool *pool, const mlora_segments *segs, const vo
                           int64_t ldx, float *H, int64_t ldh, void *stream);
 
 /*
- * Expand alone: Y[t_p, :] = bf16(Y[t_p, :] + s_g H[p, 0:r] B_a^T) for every grouped
+ * Expand alone (page "Multi-LoRA Serving: adapter batching", section "What metadata
+ * a segmented kernel needs", the expand and scatter-add steps, with s = alpha / r
+ * from section "LoRA on one Linear layer"):
+ * Y[t_p, :] = bf16(Y[t_p, :] + s_g H[p, 0:r] B_a^T) for every grouped
  * position p of every adapter segment.  H is device fp32 [n_tokens, ldh] in
  * grouped order; Y is device bf16 [n_rows, d_out] (row stride ldy), updated in
  * place.
@@ -246,13 +259,16 @@ mlora_status mlora_apply_multi(mlora_pool *const *pools, int32_t n_proj,
  * hit the device-wide synchronisation a cudaMalloc / cudaFree can cause.  This
  * variant takes the workspace from a fixed scratch array in the library's own device
  * memory instead, and calls no cudaMalloc, cudaFree or other allocating routine.
- *   - The scratch array is 4 MiB; every GPU that loads the library holds it until
- *     the process exits.  A batch needs n_tokens * max(16, bucket(r_max)) * 4 bytes
- *     (up to 16384 grouped rows for a rank-64 pool, 65536 for r_max <= 16); larger
- *     batches return MLORA_ERR_UNSUPPORTED with nothing launched.
- *   - The first call on a device looks up the array's device address (with the
- *     pool's device current) and keeps it; make that first call before any stream
- *     capture.
+ *   - The scratch array is 4 MiB.  It is reserved on a device when the first pool
+ *     is created there (mlora_pool_create looks up its address, which under CUDA's
+ *     lazy module loading is what brings it onto the device), so the first
+ *     mlora_apply_noalloc call finds it in place; every GPU that has held a pool keeps
+ *     it until the process exits.
+ *   - Only batches that take the long-segment kernels use it: n_tokens >= 128, d_in a
+ *     multiple of 64, and segs->max_segment_rows either 0 (unknown) or >= 128.  Such
+ *     a batch needs n_tokens * max(16, bucket(r_max)) * 4 bytes (up to 16384 grouped
+ *     rows for a rank-64 pool, 65536 for r_max <= 16); a larger one returns
+ *     MLORA_ERR_UNSUPPORTED with nothing launched.  Other batches have no size limit.
  *   - Every call shares the one array, which keeps the last call's contents (no
  *     part of it needs to start at zero: each call writes the H values it reads).
  *     Calls whose kernels overlap on the GPU -- on different streams, from several
@@ -267,7 +283,7 @@ mlora_status mlora_apply_noalloc(mlora_pool *pool, const mlora_segments *segs, c
  * order inside a segment.  Outputs are HOST arrays the caller sizes:
  * offsets[n_rows + 1], slots[n_rows], token_indices[n_rows].  *n_segments gets S,
  * *max_segment_rows (may be NULL) the longest adapter segment whose rows are
- * consecutive (the mlora_segments hint).  If pool and
+ * consecutive (the mlora_segments hint), at least 1 (0 would read as "unknown").  If pool and
  * ranks are both non-NULL, ranks[n_rows] gets each segment's slot rank (0 for
  * base).  Slots are not range-checked here (the device checks them).
  */

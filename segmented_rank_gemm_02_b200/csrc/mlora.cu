@@ -20,6 +20,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include "internal.h"
 #include "kernels.cuh"
 
 struct mlora_pool {
@@ -312,7 +313,9 @@ mlora_status mlora_apply_with_workspace(mlora_pool *pool, const mlora_segments *
 {
     mlora_status st = check_segments(pool, segs);
     if (st != MLORA_OK) return st;
-    if ((size_t)segs->n_tokens * std::max(16, pool->r_bucket_max) * sizeof(float) > ws_bytes)
+    // only batches that take the long-segment kernels use the workspace
+    if (long_path(pool, segs) &&
+        (size_t)segs->n_tokens * std::max(16, pool->r_bucket_max) * sizeof(float) > ws_bytes)
         return MLORA_ERR_UNSUPPORTED;
     if (segs->n_segments == 0 || segs->n_tokens == 0) return MLORA_OK;
     if (X == nullptr || Y == nullptr || !aligned16(X) || !aligned16(Y)) return MLORA_ERR_INVALID_ARG;
@@ -403,6 +406,9 @@ mlora_status mlora_pool_create(int32_t d_in, int32_t d_out, int32_t n_slots, int
     } else {
         st = prepare_device(dev);
     }
+    // the no-allocation entry point's scratch array is reserved here, with the pool's
+    // device current, rather than by its first call
+    if (st == MLORA_OK) st = mlora_noalloc_reserve(dev);
     if (st == MLORA_OK) {
         pool->b_maps_ok = tensor_map_encoder() != nullptr;
         for (int i = 0; i < 4 && pool->b_maps_ok; ++i)
@@ -717,7 +723,9 @@ mlora_status mlora_build_segments(const int32_t *row_slots, int32_t n_rows, int3
             token_indices[offsets[g + 1] - 1] - token_indices[offsets[g]] == counts[g] - 1)
             longest = std::max(longest, counts[g]);
     *n_segments = S;
-    if (max_segment_rows) *max_segment_rows = longest;
+    // at least 1: in mlora_segments a hint of 0 means "unknown", which would send a
+    // batch without any run of consecutive rows to the long-segment kernels
+    if (max_segment_rows) *max_segment_rows = std::max(longest, 1);
     if (pool != nullptr && ranks != nullptr) {
         for (int32_t g = 0; g < S; ++g) {
             const int32_t a = slots[g];

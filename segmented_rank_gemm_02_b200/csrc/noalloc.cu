@@ -6,11 +6,20 @@
 // allocate device memory: a serving engine that reserves nearly all of HBM up front
 // and serves every buffer from its own allocator, or a loop that must not meet the
 // device-wide synchronisation of a cudaMalloc / cudaFree.  For them this entry point
-// takes the workspace from a fixed array in the library's own device memory,
-// reserved when the library is loaded (every GPU that loads the library holds it
-// until the process exits), so a call allocates nothing.  The array keeps the last
-// call's contents; each call writes every H value it later reads, so nothing needs
-// clearing.  Calls whose kernels overlap on the GPU race on the one array.
+// takes the workspace from a fixed array in the library's own device memory, so a
+// call allocates nothing.
+//
+// When the array is reserved.  Each .cu file of the library is its own module, and
+// CUDA loads modules lazily: this file's module (and the array with it) is brought
+// onto a device the first time its symbol is looked up there.  mlora_pool_create does
+// that look-up for its device (mlora_noalloc_reserve), so the array is reserved when
+// the first pool is created on a device -- a call that allocates anyway -- and a later
+// mlora_apply_noalloc finds the address cached.  Every GPU that has held a pool keeps
+// the array until the process exits.
+//
+// The array keeps the last call's contents; each call writes every H value it later
+// reads, so nothing needs clearing.  Calls whose kernels overlap on the GPU race on
+// the one array.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -48,6 +57,12 @@ mlora_status scratch_address(int dev, float **out)
 }
 
 }  // namespace
+
+mlora_status mlora_noalloc_reserve(int dev)
+{
+    float *unused = nullptr;
+    return scratch_address(dev, &unused);
+}
 
 extern "C" mlora_status mlora_apply_noalloc(mlora_pool *pool, const mlora_segments *segs,
                                             const void *X, int64_t ldx, void *Y, int64_t ldy,

@@ -111,8 +111,9 @@ def test_build_segments_matches_oracle_grouping(mlora, seed, n, hi):
     assert np.array_equal(meta["offsets"], off)
     assert np.array_equal(meta["slots"], slots)
     assert np.array_equal(meta["token_indices"], ti)
-    # the hint: the longest adapter segment whose rows are consecutive
-    want = 0
+    # the hint: the longest adapter segment whose rows are consecutive, at least 1
+    # (0 means "unknown" in mlora_segments)
+    want = 1
     for g in range(len(slots)):
         a, b = off[g], off[g + 1]
         if slots[g] >= 0 and b > a and ti[b - 1] - ti[a] == b - a - 1:

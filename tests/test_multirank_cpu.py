@@ -68,14 +68,40 @@ def test_reference_arm_only_rank0_prints(monkeypatch, capsys):
     monkeypatch.setenv("WORLD_SIZE", "2")
     monkeypatch.setenv("RANK", "1")
     monkeypatch.setenv("LOCAL_RANK", "1")
-    assert bench.main(["--impl", "reference", "--config", "1", "--steps", "1", "--warmup", "3",
-                       "--cpu-seconds", "0.2"]) == 0
+    assert bench.main(["--gpus", "2", "--impl", "reference", "--config", "1", "--steps", "1",
+                       "--warmup", "3", "--cpu-seconds", "0.2"]) == 0
     assert capsys.readouterr().out == ""
     monkeypatch.setenv("RANK", "0")
     monkeypatch.setenv("LOCAL_RANK", "0")
-    assert bench.main(["--impl", "reference", "--config", "1", "--steps", "1", "--warmup", "3",
-                       "--cpu-seconds", "0.2"]) == 0
+    assert bench.main(["--gpus", "2", "--impl", "reference", "--config", "1", "--steps", "1",
+                       "--warmup", "3", "--cpu-seconds", "0.2"]) == 0
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_gpus_must_match_the_launch(monkeypatch):
+    """A multi-GPU request never runs (or reports) as a 1-GPU job: under a launcher
+    whose world size differs from --gpus the script refuses."""
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setenv("RANK", "0")
+    assert bench.main(["--gpus", "2", "--impl", "reference", "--config", "1", "--steps", "1",
+                       "--warmup", "3", "--cpu-seconds", "0.2"]) == 2
+
+
+def test_gpus_n_outside_a_launcher_spawns_n_ranks(monkeypatch, capfd):
+    """--gpus 2 without torchrun relaunches the script with two ranks (here the reference
+    arm, which needs no GPU): exactly one JSON line, from rank 0, saying n_gpus 2."""
+    sys.path.insert(0, ROOT)
+    import bench
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "LOCAL_WORLD_SIZE", "MASTER_ADDR", "MASTER_PORT"):
+        monkeypatch.delenv(k, raising=False)
+    assert bench.main(["--gpus", "2", "--impl", "reference", "--config", "1", "--steps", "1",
+                       "--warmup", "3", "--cpu-seconds", "0.2"]) == 0
+    lines = [l for l in capfd.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
