@@ -424,9 +424,10 @@ def measure(args, cfg: int, fused: bool, rank: int, world: int, device_index: in
             e["Y"].copy_(Y0[j])
     torch.cuda.synchronize()
 
-    # warm-up steps (eager), then capture exactly K steps into one graph
+    # warm-up steps (eager; at least one per buffer set, which sizes every pool's
+    # workspace before capture), then capture exactly K steps into one graph
     with torch.cuda.stream(stream):
-        for k in range(args.warmup):
+        for k in range(max(args.warmup, n_sets)):
             step(k)
     stream.synchronize()
     graph = torch.cuda.CUDAGraph(keep_graph=True)   # kept so its kernel nodes can be counted

@@ -201,9 +201,10 @@ mlora_status mlora_expand(mlora_pool *pool, const mlora_segments *segs, const fl
  * Fused shrink + expand: Y[t, :] = bf16(Y0[t, :] + s_g (X[t, :] A_a^T) B_a^T) in
  * place on the caller's base output Y (= Y0 = X W^T on entry).  For short segments
  * the rank-r intermediate stays on chip; for segments of 128 or more consecutive
- * rows it passes through an fp32 workspace the pool owns (grown with cudaMalloc
- * when a batch needs more, which is not possible during stream capture:
- * MLORA_ERR_UNSUPPORTED).  Calls on one pool whose kernels overlap on the GPU
+ * rows it passes through an fp32 workspace the pool owns (grown, stream-ordered on
+ * `stream` with no device-wide synchronisation, when a batch needs more; growth is
+ * not possible during stream capture: MLORA_ERR_UNSUPPORTED, so run the largest
+ * batch once before capturing).  Calls on one pool whose kernels overlap on the GPU
  * (several streams) share that workspace and race on it: serialise them, give each
  * stream its own pool, or use mlora_shrink / mlora_expand with caller-owned H.
  * X: device bf16 [n_rows, d_in]; Y: device bf16 [n_rows, d_out].

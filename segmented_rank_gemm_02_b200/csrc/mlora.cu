@@ -184,7 +184,9 @@ bool encode_b_map(CUtensorMap *map, const mlora_pool *pool, int R)
 
 // Make the pool's workspace hold `bytes` (the caller holds pool->ws_mutex and keeps it
 // until the kernels that use the workspace are launched, so that no other thread frees
-// it in between); growing it is not possible while the stream is being captured.
+// it in between).  Growth is stream-ordered (the old buffer is freed, and the new one
+// allocated, on `stream`: no device-wide synchronisation); it is not possible while
+// the stream is being captured.
 mlora_status ensure_workspace(mlora_pool *pool, size_t bytes, cudaStream_t stream)
 {
     if (pool->ws_bytes >= bytes) return MLORA_OK;
@@ -192,14 +194,15 @@ mlora_status ensure_workspace(mlora_pool *pool, size_t bytes, cudaStream_t strea
     if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return MLORA_ERR_CUDA;
     if (cs != cudaStreamCaptureStatusNone) return MLORA_ERR_UNSUPPORTED;
     if (pool->ws) {
-        if (cudaDeviceSynchronize() != cudaSuccess) return MLORA_ERR_CUDA;
-        cudaFree(pool->ws);
+        if (cudaFreeAsync(pool->ws, stream) != cudaSuccess) return MLORA_ERR_CUDA;
         pool->ws = nullptr;
         pool->ws_bytes = 0;
     }
-    const size_t want = std::max<size_t>(bytes, (size_t)1 << 20);
-    if (cudaMalloc(&pool->ws, want) != cudaSuccess) {
+    // some headroom, so that a slowly growing batch does not reallocate every call
+    const size_t want = std::max<size_t>(bytes + bytes / 4, (size_t)1 << 20);
+    if (cudaMallocAsync(reinterpret_cast<void **>(&pool->ws), want, stream) != cudaSuccess) {
         cudaGetLastError();
+        pool->ws = nullptr;
         return MLORA_ERR_OUT_OF_MEMORY;
     }
     pool->ws_bytes = want;
@@ -433,7 +436,10 @@ mlora_status mlora_pool_destroy(mlora_pool *pool)
     if (pool->d_scale) cudaFree(pool->d_scale);
     if (pool->d_gen) cudaFree(pool->d_gen);
     if (pool->d_status) cudaFree(pool->d_status);
-    if (pool->ws) cudaFree(pool->ws);
+    if (pool->ws) {   // stream-ordered allocation: freed the same way, then waited for
+        cudaFreeAsync(pool->ws, nullptr);
+        cudaDeviceSynchronize();
+    }
     delete pool;
     return MLORA_OK;
 }
