@@ -61,6 +61,10 @@ def _declare(lib):
     lib.orc_apply_rows.argtypes = [
         ctypes.c_int, ctypes.c_int, ctypes.c_int, _u16p, ctypes.c_int64, _f64p, ctypes.c_int64,
         _i32p, _f64p, ctypes.c_int, _i32p, _f64p, _u16pp, _u16pp, ctypes.c_int]
+    lib.orc_apply_rows_xf64.restype = ctypes.c_int
+    lib.orc_apply_rows_xf64.argtypes = [
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, _f64p, ctypes.c_int64, _f64p, ctypes.c_int64,
+        _i32p, _f64p, ctypes.c_int, _i32p, _f64p, _u16pp, _u16pp, ctypes.c_int]
     lib.orc_shrink.restype = ctypes.c_int
     lib.orc_shrink.argtypes = [
         ctypes.c_int, ctypes.c_int, _u16p, ctypes.c_int64,
@@ -206,6 +210,48 @@ def apply_rows(X: np.ndarray, Y0: np.ndarray, row_slot, row_scale, slot_rank, sl
         _p(slot_alpha, _f64p), ta, tb, int(n_threads))
     del ka, kb
     return Y, int(flags)
+
+
+def apply_rows_xf64(X: np.ndarray, Y0: np.ndarray, row_slot, row_scale, slot_rank, slot_alpha,
+                    A: Dict[int, np.ndarray], B: Dict[int, np.ndarray],
+                    n_threads: int = 0) -> Tuple[np.ndarray, int]:
+    """Per-row formulation with the activation given as fp64 values (``X`` float64) and
+    ``Y0`` as float64 values: the reference at a quantized base model's dtype boundary,
+    where X is an FP8 code times its scale and Y0 an fp16 or fp32 base output."""
+    lib = load()
+    X = np.array(X, dtype=np.float64, order="C")
+    Y = np.array(Y0, dtype=np.float64, order="C")
+    n_rows, d_in = X.shape
+    d_out = Y.shape[1]
+    row_slot, row_scale = _i32(row_slot), _f64(row_scale)
+    slot_rank, slot_alpha = _i32(slot_rank), _f64(slot_alpha)
+    n_slots = slot_rank.shape[0]
+    ta, ka = _ptr_table(A, n_slots)
+    tb, kb = _ptr_table(B, n_slots)
+    flags = lib.orc_apply_rows_xf64(
+        n_rows, d_in, d_out, _p(X, _f64p), d_in, _p(Y, _f64p), d_out,
+        _p(row_slot, _i32p), _p(row_scale, _f64p), n_slots, _p(slot_rank, _i32p),
+        _p(slot_alpha, _f64p), ta, tb, int(n_threads))
+    del ka, kb
+    return Y, int(flags)
+
+
+def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
+    """Exact values of FP8 e4m3 codes (1 sign bit, 4 exponent bits with bias 7, 3
+    mantissa bits; exponent field 0 is subnormal, 2^-6 * m/8; S.1111.111 is NaN and
+    there is no infinity), as float64."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    val = np.where((e == 0xF) & ((c & 0x7) == 0x7), np.nan, val)
+    return sign * val
+
+
+def f16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact values of IEEE binary16 bit patterns as float64."""
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
 
 
 def shrink(X: np.ndarray, offsets, slots, ranks, token_indices, slot_rank,

@@ -87,6 +87,28 @@ static void lora_row(int d_in, int d_out, int r, const uint16_t *x, double *y, d
     }
 }
 
+/* The same row with the activation given as fp64 values rather than bf16 bits -- an
+ * activation whose exact value is known by other means, such as an FP8 code times its
+ * scale at the dtype boundary of a quantized base model (page "Multi-LoRA Serving:
+ * adapter batching", section "The dtype boundary between a quantized base model and
+ * LoRA").  Same loop order. */
+static void lora_row_xf64(int d_in, int d_out, int r, const double *x, double *y, double s,
+                          const uint16_t *A, const uint16_t *B, double *h)
+{
+    for (int j = 0; j < r; ++j) {
+        double dot = 0.0;
+        const uint16_t *arow_j = A + (size_t)d_in * j;
+        for (int k = 0; k < d_in; ++k) dot += x[k] * bf16_value(arow_j[k]);
+        h[j] = dot;
+    }
+    for (int o = 0; o < d_out; ++o) {
+        double dot = 0.0;
+        const uint16_t *brow_o = B + (size_t)r * o;
+        for (int j = 0; j < r; ++j) dot += h[j] * bf16_value(brow_o[j]);
+        y[o] = y[o] + s * dot;
+    }
+}
+
 static void set_threads(int n_threads)
 {
 #ifdef _OPENMP
@@ -161,6 +183,33 @@ int orc_apply_rows(int n_rows, int d_in, int d_out,
         double s = row_scale ? row_scale[t] : slot_alpha[a] / (double)r;
         double h[ORC_MAX_RANK];
         lora_row(d_in, d_out, r, X + (size_t)t * ldx, Y + (size_t)t * ldy, s, A[a], B[a], h);
+    }
+    return flags;
+}
+
+/*
+ * Per-row formulation with the activation as fp64 values (X fp64 [n_rows, ldx]); the
+ * rest as orc_apply_rows.
+ */
+int orc_apply_rows_xf64(int n_rows, int d_in, int d_out,
+                        const double *X, int64_t ldx, double *Y, int64_t ldy,
+                        const int32_t *row_slot, const double *row_scale,
+                        int n_slots, const int32_t *slot_rank, const double *slot_alpha,
+                        const uint16_t *const *A, const uint16_t *const *B, int n_threads)
+{
+    int flags = 0;
+    set_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : flags)
+    for (int t = 0; t < n_rows; ++t) {
+        int a = row_slot[t];
+        if (a == -1) continue;
+        if (a < -1 || a >= n_slots) { flags |= ORC_BAD_SLOT; continue; }
+        int r = slot_rank[a];
+        if (r <= 0) { flags |= ORC_SLOT_EMPTY; continue; }
+        if (r > ORC_MAX_RANK) { flags |= ORC_BAD_RANK; continue; }
+        double s = row_scale ? row_scale[t] : slot_alpha[a] / (double)r;
+        double h[ORC_MAX_RANK];
+        lora_row_xf64(d_in, d_out, r, X + (size_t)t * ldx, Y + (size_t)t * ldy, s, A[a], B[a], h);
     }
     return flags;
 }

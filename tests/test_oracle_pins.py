@@ -347,6 +347,10 @@ MUTANTS = {
     "A_row_stride": ("A + (size_t)j * d_in;", "A + (size_t)j;", 1),
     "x_index": ("acc += bf16_value(x[k]) * bf16_value(a_row[k])",
                 "acc += bf16_value(x[j]) * bf16_value(a_row[k])", 1),
+    # the fp64-activation row (dtype boundary of a quantized base model)
+    "xf64_x_index": ("dot += x[k] * bf16_value(arow_j[k])", "dot += x[j] * bf16_value(arow_j[k])", 1),
+    "xf64_dropped_scale": ("y[o] = y[o] + s * dot;", "y[o] = y[o] + dot;", 1),
+    "xf64_A_row_stride": ("A + (size_t)d_in * j;", "A + (size_t)j;", 1),
 }
 
 
@@ -375,9 +379,88 @@ def test_planted_mistake_is_caught(name, tmp_path):
     lib = oracle.load(so)
     failed = []
     with _swapped_oracle(lib):
-        for check in PIN_CHECKS:
+        for check in MUTANT_CHECKS:
             try:
                 check()
             except AssertionError:
                 failed.append(check.__name__)
     assert failed, f"mutant {name} passed every pin"
+
+
+# ---------------------------------------------------------------------------
+# the dtype boundary of a quantized base model: FP8 e4m3 activation codes and
+# fp16 / fp32 base outputs (page "Multi-LoRA Serving: adapter batching", section
+# "The dtype boundary between a quantized base model and LoRA")
+# ---------------------------------------------------------------------------
+
+def test_e4m3_decoding_closed_forms():
+    # the format: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, subnormals at
+    # exponent field 0, S.1111.111 NaN, no infinity
+    v = oracle.e4m3_to_f64(np.array([0x38, 0x3C, 0x7E, 0x08, 0x01, 0x07, 0x00, 0xB8, 0xFE, 0x40], np.uint8))
+    assert v.tolist() == [1.0, 1.5, 448.0, 2.0 ** -6, 2.0 ** -9, 7 * 2.0 ** -9, 0.0, -1.0, -448.0, 2.0]
+    assert np.isnan(oracle.e4m3_to_f64(np.array([0x7F, 0xFF], np.uint8))).all()
+
+
+def test_e4m3_decoding_matches_library_conversion():
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_to_f64(codes)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    both_nan = np.isnan(ours) & np.isnan(lib)
+    assert np.array_equal(ours[~both_nan], lib[~both_nan]) and np.isnan(ours).sum() == np.isnan(lib).sum() == 2
+
+
+def test_f16_decoding_closed_forms():
+    v = oracle.f16_to_f64(np.array([0x3C00, 0x7BFF, 0x0001, 0xC000, 0x3555], np.uint16))
+    assert v.tolist() == [1.0, 65504.0, 2.0 ** -24, -2.0, 0.333251953125]
+
+
+def test_fp64_activation_entry_equals_bf16_entry():
+    # the same activation values given as fp64 instead of bf16 bits: identical results
+    P = _small_problem(seed=31)
+    Yb, fb = oracle.apply_rows(P["X"], P["Y0"], P["row_slot"], None, P["slot_rank"], P["slot_alpha"],
+                               P["A"], P["B"])
+    Yx, fx = oracle.apply_rows_xf64(oracle.bf16_to_f64(P["X"]), oracle.bf16_to_f64(P["Y0"]), P["row_slot"],
+                                    None, P["slot_rank"], P["slot_alpha"], P["A"], P["B"])
+    assert fb == fx == 0
+    assert np.array_equal(Yb, Yx)
+
+
+def test_fp64_activation_merged_weight_identity_with_fp8_codes():
+    # X = code * scale (FP8 activation), Y0 = X W^T in fp64: the result must equal
+    # X (W + s B A)^T for adapter rows and X W^T for base rows
+    rng = np.random.default_rng(5)
+    P = _small_problem(seed=32, d_in=48, d_out=40)
+    codes = rng.integers(0, 256, P["X"].shape).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x38            # no NaN codes
+    scale = 0.0625
+    X = oracle.e4m3_to_f64(codes) * scale
+    W = rng.normal(0, 0.5, (40, 48))
+    Y0 = X @ W.T
+    Y, flags = oracle.apply_rows_xf64(X, Y0, P["row_slot"], None, P["slot_rank"], P["slot_alpha"], P["A"], P["B"])
+    assert flags == 0
+    for t in range(X.shape[0]):
+        a = int(P["row_slot"][t])
+        Wt = W.copy()
+        if a >= 0:
+            s = P["slot_alpha"][a] / P["slot_rank"][a]
+            Wt = W + s * oracle.bf16_to_f64(P["B"][a]) @ oracle.bf16_to_f64(P["A"][a])
+        want = X[t] @ Wt.T
+        assert np.allclose(Y[t], want, rtol=1e-12, atol=1e-12), t
+
+
+def test_fp64_activation_is_linear_in_the_activation():
+    # doubling X doubles the delta, exactly (powers of two scale fp64 sums exactly)
+    P = _small_problem(seed=33)
+    X = oracle.bf16_to_f64(P["X"])
+    Y0 = np.zeros((X.shape[0], P["Y0"].shape[1]))
+    Y1, _ = oracle.apply_rows_xf64(X, Y0, P["row_slot"], None, P["slot_rank"], P["slot_alpha"], P["A"], P["B"])
+    Y2, _ = oracle.apply_rows_xf64(4 * X, Y0, P["row_slot"], None, P["slot_rank"], P["slot_alpha"], P["A"], P["B"])
+    assert np.array_equal(Y2, 4 * Y1)
+    assert np.abs(Y1).max() > 0
+
+
+# the planted mistakes are judged by every pin, the fp64-activation ones included
+MUTANT_CHECKS = PIN_CHECKS + [test_fp64_activation_entry_equals_bf16_entry,
+                              test_fp64_activation_merged_weight_identity_with_fp8_codes,
+                              test_fp64_activation_is_linear_in_the_activation]
