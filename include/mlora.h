@@ -212,6 +212,38 @@ mlora_status mlora_expand(mlora_pool *pool, const mlora_segments *segs, const fl
 mlora_status mlora_apply(mlora_pool *pool, const mlora_segments *segs, const void *X,
                          int64_t ldx, void *Y, int64_t ldy, void *stream);
 
+/* Element types at the dtype boundary of a quantized base model (mlora_apply_ex). */
+#define MLORA_DTYPE_BF16      0
+#define MLORA_DTYPE_FP16      1
+#define MLORA_DTYPE_FP32      2
+#define MLORA_DTYPE_FP8_E4M3  3
+
+/*
+ * mlora_apply at the dtype boundary of a quantized base model (page "Multi-LoRA
+ * Serving: adapter batching", section "The dtype boundary between a quantized base
+ * model and LoRA": the base GEMM's accumulation and output dtype, whether the LoRA
+ * branch reuses the activation from before quantization, the dtype and scale of A and
+ * B, and where the two paths add).  The answers this entry point gives:
+ *   - A and B stay bf16 in the pool, s = alpha / r is applied inside the kernel;
+ *   - the LoRA input X is either the bf16 activation from before quantization
+ *     (x_dtype MLORA_DTYPE_BF16; x_scale ignored) or the FP8 e4m3 codes the base GEMM
+ *     reads (MLORA_DTYPE_FP8_E4M3), whose value is code * x_scale (one per-tensor
+ *     scale); the codes are widened exactly, the shrink sums in fp32 and H is scaled by
+ *     x_scale before the expand;
+ *   - the two paths add once, on the base GEMM's output in its own dtype
+ *     (y_dtype MLORA_DTYPE_BF16, _FP16 or _FP32): Y[t, :] = round(Y0[t, :] + s H B^T)
+ *     with the sum in fp32 and one rounding to y_dtype (none for fp32).
+ * X: device [n_rows, d_in] of x_dtype, row stride ldx elements (a multiple of 16 for
+ * FP8 codes, of 8 for bf16; FP8 also needs d_in a multiple of 16); Y: device
+ * [n_rows, d_out] of y_dtype, row stride ldy (a multiple of 8, of 4 for fp32); both
+ * 16-byte aligned.  The all-bf16 pair is mlora_apply itself.  Other pairs run every
+ * segment on the decode-shaped kernel (the tensor-memory kernels for segments of 128+
+ * consecutive rows are bf16 only), so they allocate nothing.  Errors as mlora_apply,
+ * plus MLORA_ERR_INVALID_ARG for another dtype or a non-finite x_scale.
+ */
+mlora_status mlora_apply_ex(mlora_pool *pool, const mlora_segments *segs, const void *X, int32_t x_dtype,
+                            float x_scale, int64_t ldx, void *Y, int32_t y_dtype, int64_t ldy, void *stream);
+
 /* Projections one mlora_apply_multi call may cover. */
 #define MLORA_MAX_FUSED 4
 

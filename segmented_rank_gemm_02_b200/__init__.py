@@ -31,7 +31,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_OUT_OF_MEMORY, ERR_BAD_METADATA, ERR_C
 EXPORTS = ("mlora_pool_create", "mlora_pool_destroy", "mlora_pool_load_slot",
            "mlora_pool_clear_slot", "mlora_pool_slot_info", "mlora_pool_shape",
            "mlora_pool_check", "mlora_shrink", "mlora_expand", "mlora_apply",
-           "mlora_apply_noalloc", "mlora_apply_multi", "mlora_build_segments", "mlora_status_string",
+           "mlora_apply_noalloc", "mlora_apply_multi", "mlora_apply_ex", "mlora_build_segments", "mlora_status_string",
            "mlora_version", "mlora_pool_slot_generation", "mlora_slot_cache_create",
            "mlora_slot_cache_destroy", "mlora_slot_cache_acquire", "mlora_slot_cache_release",
            "mlora_slot_cache_invalidate", "mlora_slot_cache_lookup", "mlora_slot_cache_stats")
@@ -70,6 +70,7 @@ def _load():
         "mlora_expand": [vp, seg_p, vp, i64, vp, i64, vp],
         "mlora_apply": [vp, seg_p, vp, i64, vp, i64, vp],
         "mlora_apply_noalloc": [vp, seg_p, vp, i64, vp, i64, vp],
+        "mlora_apply_ex": [vp, seg_p, vp, i32, f32, i64, vp, i32, i64, vp],
         "mlora_apply_multi": [ctypes.POINTER(vp), i32, seg_p, vp, i64, ctypes.POINTER(vp),
                               ctypes.POINTER(i64), vp],
         "mlora_build_segments": [vp, i32, vp, vp, vp, i32p, i32p, vp, vp],
@@ -286,6 +287,25 @@ def apply_noalloc(pool: Pool, segs: DeviceSegments, X, Y, stream=None) -> None:
 
 
 MAX_FUSED = 4
+
+DTYPE_BF16, DTYPE_FP16, DTYPE_FP32, DTYPE_FP8_E4M3 = 0, 1, 2, 3
+
+
+def _dtype_code(t) -> int:
+    import torch
+    codes = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_FP16, torch.float32: DTYPE_FP32,
+             torch.float8_e4m3fn: DTYPE_FP8_E4M3}
+    if t.dtype not in codes:
+        raise ValueError(f"unsupported dtype {t.dtype}")
+    return codes[t.dtype]
+
+
+def apply_ex(pool: Pool, segs: DeviceSegments, X, Y, x_scale: float = 1.0, stream=None) -> None:
+    """mlora_apply at a quantized base model's dtype boundary (mlora_apply_ex): X bf16 or
+    FP8 e4m3 codes (value = code * x_scale), Y bf16, fp16 or fp32, updated in place."""
+    _check(lib().mlora_apply_ex(pool.handle, ctypes.byref(segs.struct), _ptr(X), _dtype_code(X), float(x_scale),
+                                _ld(X, "X"), _ptr(Y), _dtype_code(Y), _ld(Y, "Y"), _stream_ptr(stream)),
+           "mlora_apply_ex")
 
 
 def apply_multi(pools, segs: DeviceSegments, X, Ys, stream=None) -> None:

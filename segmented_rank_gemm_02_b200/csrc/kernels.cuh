@@ -105,6 +105,8 @@ struct TileParams {
     // d_in, the segment metadata and the slot numbering)
     int32_t n_proj;
     ProjView proj[kMaxFused];
+    // per-tensor scale of FP8 activation codes (dtype boundary variants only)
+    float x_scale;
 };
 
 // A segment [p0, p1) goes to the long-segment kernels when it holds at least
@@ -143,6 +145,12 @@ int long_shrink_split(int rmax_bucket, int d_in, int64_t tiles);
 // can be resident at once, but no more than `max_tiles` (each loops over tiles).
 cudaError_t launch_tile_kernel(int mode, int rmax_bucket, const TileParams &p, int cluster,
                                int64_t max_tiles, cudaStream_t stream);
+
+// The fused apply (MODE_APPLY, one projection) at another dtype boundary of a quantized
+// base model: dt = 3 * xt + yt, xt 0 = bf16 X, 1 = FP8 e4m3 codes (times p.x_scale);
+// yt 0 = bf16 Y, 1 = fp16, 2 = fp32 (1 <= dt <= 5; 0 is launch_tile_kernel's path).
+cudaError_t launch_tile_kernel_dt(int dt, int rmax_bucket, const TileParams &p, int cluster, int64_t max_tiles,
+                                  cudaStream_t stream);
 
 // Fused launch over p.n_proj projections (MODE_APPLY): a work item is one tile of one
 // projection, and the items of a tile are adjacent so its X rows come from HBM once.

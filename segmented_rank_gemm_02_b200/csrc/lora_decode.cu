@@ -57,6 +57,10 @@
 // bounded: on expiry it flags a timeout and leaves the tile's rows alone.
 #include <climits>
 #include <mutex>
+#include <type_traits>
+
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -99,10 +103,24 @@ struct ShrinkOps {
     uint4 a[RankCfg<R>::NT];    // adapter rows n*8+g, same columns
 };
 
-template <int R>
+// Element types of the activation X and of the base output Y (the dtype boundary of
+// a quantized base model): DT = 3 * XT + YT with XT 0 = bf16, 1 = FP8 e4m3 codes (times
+// a per-tensor scale); YT 0 = bf16, 1 = fp16, 2 = fp32.  DT 0 is the all-bf16 path.
+__host__ __device__ constexpr int dt_x(int dt) { return dt / 3; }
+__host__ __device__ constexpr int dt_y(int dt) { return dt % 3; }
+__host__ __device__ constexpr int x_bytes(int dt) { return dt_x(dt) == 1 ? 1 : 2; }
+__host__ __device__ constexpr int y_bytes(int dt) { return dt_y(dt) == 2 ? 4 : 2; }
+
+template <int R, int YT = 0>
 struct ExpandOps {
     uint2 b[4][RankCfg<R>::KS];  // B rows of the four n8 tiles, this lane's ranks
-    uint4 y;                     // Y0 row g, columns 8t..8t+7 of the group
+    uint4 y;                     // Y0 row g, columns 8t..8t+7 of the group (bf16 or fp16)
+};
+
+template <int R>
+struct ExpandOps<R, 2> {
+    uint2 b[4][RankCfg<R>::KS];
+    uint4 y, y2;                 // fp32 Y0: columns 8t..8t+3, 8t+4..8t+7
 };
 
 struct SharedCtl {
@@ -269,12 +287,37 @@ __device__ __forceinline__ void load_a(ShrinkOps<R> &o, const __nv_bfloat16 *slo
         o.a[n] = kin ? ldg_nc(slotA + ((int64_t)(k / 8) * R + n * 8 + g) * 8) : make_uint4(0, 0, 0, 0);
 }
 
-template <int R>
-__device__ __forceinline__ void load_x(ShrinkOps<R> &o, const __nv_bfloat16 *xrow, bool row_ok,
-                                       const Slices &sl, int blk, int t)
+// Two FP8 e4m3 codes (low byte first) as the bf16x2 of their values: exact, since every
+// e4m3 value is a bf16 value.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two)
+{
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h));
+    return pack_bf16x2(f.x, f.y);
+}
+
+// X's element type: bf16 values or FP8 e4m3 codes (bytes).
+template <int XT>
+using XElem = typename std::conditional<XT == 1, const uint8_t, const __nv_bfloat16>::type;
+// Y's element type: bf16, fp16 or fp32.
+template <int YT>
+using YElem =
+    typename std::conditional<YT == 2, float, typename std::conditional<YT == 1, __half, __nv_bfloat16>::type>::type;
+
+template <int R, int XT = 0>
+__device__ __forceinline__ void load_x(ShrinkOps<R> &o, XElem<XT> *xrow, bool row_ok, const Slices &sl, int blk,
+                                       int t)
 {
     const int k = sl.k_begin + blk * 32 + 8 * t;
-    o.x = (row_ok && blk < sl.nblk && k < sl.k_end) ? ldg_nc(xrow + k) : make_uint4(0, 0, 0, 0);
+    if constexpr (XT == 0) {
+        o.x = (row_ok && blk < sl.nblk && k < sl.k_end) ? ldg_nc(xrow + k) : make_uint4(0, 0, 0, 0);
+    } else {
+        // eight e4m3 codes, widened to bf16 (the per-tensor scale is applied to H)
+        const bool in = row_ok && blk < sl.nblk && k < sl.k_end;
+        const uint2 c = in ? __ldg(reinterpret_cast<const uint2 *>(xrow + k)) : make_uint2(0u, 0u);
+        o.x = make_uint4(e4m3x2_to_bf16x2(c.x), e4m3x2_to_bf16x2(c.x >> 16), e4m3x2_to_bf16x2(c.y),
+                         e4m3x2_to_bf16x2(c.y >> 16));
+    }
 }
 
 template <int R>
@@ -289,8 +332,8 @@ __device__ __forceinline__ void mma_shrink(float (&acc)[RankCfg<R>::NT][4], cons
 
 // B row fed by lane (g, t) in n8 tile i of a group: base + 8 (g / 2) + (g % 2) + 2 i, so
 // that thread (g, t) accumulates columns base + 8t .. base + 8t + 7 of row g.
-template <int R>
-__device__ __forceinline__ void load_b(ExpandOps<R> &o, const __nv_bfloat16 *slotB, int d_out,
+template <int R, int YT>
+__device__ __forceinline__ void load_b(ExpandOps<R, YT> &o, const __nv_bfloat16 *slotB, int d_out,
                                        const Slices &sl, int grp, int g, int t)
 {
     const int base = sl.n_begin + grp * 32;
@@ -313,21 +356,28 @@ __device__ __forceinline__ void load_b(ExpandOps<R> &o, const __nv_bfloat16 *slo
         }
 }
 
-template <int R>
-__device__ __forceinline__ void load_y(ExpandOps<R> &o, const __nv_bfloat16 *yrow, bool row_ok,
-                                       const Slices &sl, int grp, int t)
+template <int R, int YT>
+__device__ __forceinline__ void load_y(ExpandOps<R, YT> &o, const YElem<YT> *yrow, bool row_ok, const Slices &sl,
+                                       int grp, int t)
 {
     const int c = sl.n_begin + grp * 32 + 8 * t;
-    o.y = (row_ok && grp < sl.ngrp && c < sl.n_end) ? *reinterpret_cast<const uint4 *>(yrow + c)
-                                                     : make_uint4(0, 0, 0, 0);
+    if constexpr (YT == 2) {   // eight fp32
+        const bool in = row_ok && grp < sl.ngrp && c < sl.n_end;
+        const uint4 *src = reinterpret_cast<const uint4 *>(yrow + c);
+        o.y = in ? src[0] : make_uint4(0, 0, 0, 0);
+        o.y2 = in ? src[1] : make_uint4(0, 0, 0, 0);
+    } else {                   // eight bf16 or fp16
+        o.y = (row_ok && grp < sl.ngrp && c < sl.n_end) ? *reinterpret_cast<const uint4 *>(yrow + c)
+                                                         : make_uint4(0, 0, 0, 0);
+    }
 }
 
-// y = bf16(y0 + s (H B^T)) for one group; thread (g, t) stores row g, columns 8t..8t+7.
-template <int R>
-__device__ __forceinline__ void mma_expand_store(const ExpandOps<R> &o, const uint32_t (&ah)[RankCfg<R>::KS][2],
-                                                 const uint32_t (&al)[RankCfg<R>::KS][2], float scale,
-                                                 __nv_bfloat16 *yrow, bool store, const Slices &sl,
-                                                 int grp, int t)
+// y = y0 + s (H B^T), rounded once to Y's type, for one group; thread (g, t) stores row
+// g, columns 8t..8t+7.
+template <int R, int YT>
+__device__ __forceinline__ void mma_expand_store(const ExpandOps<R, YT> &o, const uint32_t (&ah)[RankCfg<R>::KS][2],
+                                                 const uint32_t (&al)[RankCfg<R>::KS][2], float scale, YElem<YT> *yrow,
+                                                 bool store, const Slices &sl, int grp, int t)
 {
     float d[4][4];
 #pragma unroll
@@ -346,15 +396,34 @@ __device__ __forceinline__ void mma_expand_store(const ExpandOps<R> &o, const ui
     }
     const int c = sl.n_begin + grp * 32 + 8 * t;
     if (!store || grp >= sl.ngrp || c >= sl.n_end) return;
-    const __nv_bfloat162 *y0 = reinterpret_cast<const __nv_bfloat162 *>(&o.y);
-    uint4 out;
-    uint32_t *w = reinterpret_cast<uint32_t *>(&out);
+    if constexpr (YT == 2) {
+        const float4 a = *reinterpret_cast<const float4 *>(&o.y), b = *reinterpret_cast<const float4 *>(&o.y2);
+        float4 *dst = reinterpret_cast<float4 *>(yrow + c);
+        dst[0] = make_float4(fmaf(scale, d[0][0], a.x), fmaf(scale, d[0][1], a.y), fmaf(scale, d[1][0], a.z),
+                             fmaf(scale, d[1][1], a.w));
+        dst[1] = make_float4(fmaf(scale, d[2][0], b.x), fmaf(scale, d[2][1], b.y), fmaf(scale, d[3][0], b.z),
+                             fmaf(scale, d[3][1], b.w));
+    } else {
+        uint4 out;
+        uint32_t *w = reinterpret_cast<uint32_t *>(&out);
+        if constexpr (YT == 0) {
+            const __nv_bfloat162 *y0 = reinterpret_cast<const __nv_bfloat162 *>(&o.y);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(y0[i]);
-        w[i] = pack_bf16x2(fmaf(scale, d[i][0], f.x), fmaf(scale, d[i][1], f.y));
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(y0[i]);
+                w[i] = pack_bf16x2(fmaf(scale, d[i][0], f.x), fmaf(scale, d[i][1], f.y));
+            }
+        } else {
+            const __half2 *y0 = reinterpret_cast<const __half2 *>(&o.y);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __half22float2(y0[i]);
+                const __half2 hv = __floats2half2_rn(fmaf(scale, d[i][0], f.x), fmaf(scale, d[i][1], f.y));
+                w[i] = *reinterpret_cast<const uint32_t *>(&hv);
+            }
+        }
+        *reinterpret_cast<uint4 *>(yrow + c) = out;
     }
-    *reinterpret_cast<uint4 *>(yrow + c) = out;
 }
 
 // One tile, specialised for rank bucket R.  Loads are issued as early as their
@@ -398,7 +467,7 @@ __device__ void prefetch_slices(const TileParams &p, const ProjView &v, int slot
     }
 }
 
-template <int RMAX, int MODE, int NT>
+template <int RMAX, int MODE, int NT, int DT>
 __device__ void prefetch_first_tile(const TileParams &p, const ProjView &v, int want, SharedCtl &ctl,
                                     uint32_t crank)
 {
@@ -423,19 +492,25 @@ __device__ void prefetch_first_tile(const TileParams &p, const ProjView &v, int 
                 if (MODE != MODE_EXPAND) {
                     const int k0 = min(p.d_in, (int)crank * p.k_slice);
                     const int k1 = min(p.d_in, k0 + p.k_slice);
-                    if (k1 > k0) prefetch_l2_bulk(p.X + (int64_t)row * p.ldx + k0, (uint32_t)(k1 - k0) * 2);
+                    using XE = typename std::conditional<dt_x(DT) == 1, const uint8_t, const __nv_bfloat16>::type;
+                    if (k1 > k0)
+                        prefetch_l2_bulk(reinterpret_cast<XE *>(p.X) + (int64_t)row * p.ldx + k0,
+                                         (uint32_t)(k1 - k0) * x_bytes(DT));
                 }
                 if (MODE != MODE_SHRINK) {
                     const int n0 = min(v.d_out, (int)crank * v.n_slice);
                     const int n1 = min(v.d_out, n0 + v.n_slice);
-                    if (n1 > n0) prefetch_l2_bulk(v.Y + (int64_t)row * v.ldy + n0, (uint32_t)(n1 - n0) * 2);
+                    using YE = typename std::conditional<dt_y(DT) == 2, const float, const __nv_bfloat16>::type;
+                    if (n1 > n0)
+                        prefetch_l2_bulk(reinterpret_cast<YE *>(v.Y) + (int64_t)row * v.ldy + n0,
+                                         (uint32_t)(n1 - n0) * y_bytes(DT));
                 }
             }
         }
     }
 }
 
-template <int RMAX, int MODE, int R, int NT>
+template <int RMAX, int MODE, int R, int NT, int DT>
 __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl, int r_meta,
                          float seg_scale, SharedCtl &ctl, float *smem_f, uint32_t crank,
                          uint32_t csize, uint32_t nt)
@@ -472,13 +547,14 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
         sscale = v.slot_scale[tl.slot];
         if (ctl.stale) srank = -1;   // rank -1 marks a stale generation
     }
+    constexpr int XT = dt_x(DT), YT = dt_y(DT);
     ShrinkOps<R> s0, s1;
-    ExpandOps<R> e0, e1;
+    ExpandOps<R, YT> e0, e1;
     if constexpr (MODE != MODE_EXPAND) {
         load_a<R>(s0, slotA, sl, warp, g, t);
         load_a<R>(s1, slotA, sl, warp + kWarps, g, t);
     }
-    if constexpr (MODE != MODE_SHRINK && RC::EARLY_EXPAND) load_b<R>(e0, slotB, v.d_out, sl, warp, g, t);
+    if constexpr (MODE != MODE_SHRINK && RC::EARLY_EXPAND) load_b<R, YT>(e0, slotB, v.d_out, sl, warp, g, t);
 
     // ---- requests that need the row
     if (g < tl.nvalid && (row_g < 0 || row_g >= p.n_rows)) {
@@ -486,13 +562,14 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
         row_g = -1;
     }
     const bool row_ok = row_g >= 0;
-    const __nv_bfloat16 *xrow = p.X + (int64_t)(row_ok ? row_g : 0) * p.ldx;
-    __nv_bfloat16 *yrow = v.Y + (int64_t)(row_ok ? row_g : 0) * v.ldy;
+    // row pointers in X's and Y's element types
+    XElem<XT> *xrow = reinterpret_cast<XElem<XT> *>(p.X) + (int64_t)(row_ok ? row_g : 0) * p.ldx;
+    YElem<YT> *yrow = reinterpret_cast<YElem<YT> *>(v.Y) + (int64_t)(row_ok ? row_g : 0) * v.ldy;
     if constexpr (MODE != MODE_EXPAND) {
-        load_x<R>(s0, xrow, row_ok, sl, warp, t);
-        load_x<R>(s1, xrow, row_ok, sl, warp + kWarps, t);
+        load_x<R, XT>(s0, xrow, row_ok, sl, warp, t);
+        load_x<R, XT>(s1, xrow, row_ok, sl, warp + kWarps, t);
     }
-    if constexpr (MODE != MODE_SHRINK && RC::EARLY_EXPAND) load_y<R>(e0, yrow, row_ok, sl, warp, t);
+    if constexpr (MODE != MODE_SHRINK && RC::EARLY_EXPAND) load_y<R, YT>(e0, yrow, row_ok, sl, warp, t);
 
     // ---- shrink: this CTA's d_in slice, two blocks in flight per warp
     if constexpr (MODE != MODE_EXPAND) {
@@ -504,25 +581,25 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
             if (i + 2 < nb) {
                 const int b = warp + (i + 2) * kWarps;
                 load_a<R>(s0, slotA, sl, b, g, t);
-                load_x<R>(s0, xrow, row_ok, sl, b, t);
+                load_x<R, XT>(s0, xrow, row_ok, sl, b, t);
             }
             if (i + 1 < nb) {
                 mma_shrink<R>(acc, s1);
                 if (i + 3 < nb) {
                     const int b = warp + (i + 3) * kWarps;
                     load_a<R>(s1, slotA, sl, b, g, t);
-                    load_x<R>(s1, xrow, row_ok, sl, b, t);
+                    load_x<R, XT>(s1, xrow, row_ok, sl, b, t);
                 }
             }
         }
         if constexpr (MODE != MODE_SHRINK) {
             // the expand's first groups travel while the cluster sums H
             if constexpr (!RC::EARLY_EXPAND) {
-                load_b<R>(e0, slotB, v.d_out, sl, warp, g, t);
-                load_y<R>(e0, yrow, row_ok, sl, warp, t);
+                load_b<R, YT>(e0, slotB, v.d_out, sl, warp, g, t);
+                load_y<R, YT>(e0, yrow, row_ok, sl, warp, t);
             }
-            load_b<R>(e1, slotB, v.d_out, sl, warp + kWarps, g, t);
-            load_y<R>(e1, yrow, row_ok, sl, warp + kWarps, t);
+            load_b<R, YT>(e1, slotB, v.d_out, sl, warp + kWarps, g, t);
+            load_y<R, YT>(e1, yrow, row_ok, sl, warp + kWarps, t);
         }
 #pragma unroll
         for (int n = 0; n < RC::NT; ++n) {
@@ -530,11 +607,11 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
             wpart[(warp * TM + g) * R + n * 8 + 2 * t + 1] = acc[n][1];
         }
     } else {
-        load_b<R>(e1, slotB, v.d_out, sl, warp + kWarps, g, t);
-        load_y<R>(e1, yrow, row_ok, sl, warp + kWarps, t);
+        load_b<R, YT>(e1, slotB, v.d_out, sl, warp + kWarps, g, t);
+        load_y<R, YT>(e1, yrow, row_ok, sl, warp + kWarps, t);
         if constexpr (!RC::EARLY_EXPAND) {
-            load_b<R>(e0, slotB, v.d_out, sl, warp, g, t);
-            load_y<R>(e0, yrow, row_ok, sl, warp, t);
+            load_b<R, YT>(e0, slotB, v.d_out, sl, warp, g, t);
+            load_y<R, YT>(e0, yrow, row_ok, sl, warp, t);
         }
     }
     if (tid == 0) {
@@ -588,6 +665,7 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
 #pragma unroll
             for (int c = 0; c < kMaxCluster; ++c) sum += v[c];
             if (!landed) sum = 0.f;   // (the tile's rows are then left alone)
+            if constexpr (XT == 1) sum *= p.x_scale;   // the FP8 codes' per-tensor scale
             if constexpr (MODE == MODE_APPLY) {
                 hfull[i * DC::HPITCH + j] = sum;
             } else {
@@ -625,18 +703,18 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
         }
         const bool store = ok && row_ok && h_ok;
         for (int i = 0; i < ng; i += 2) {
-            mma_expand_store<R>(e0, ah, al, scale, yrow, store, sl, warp + i * kWarps, t);
+            mma_expand_store<R, YT>(e0, ah, al, scale, yrow, store, sl, warp + i * kWarps, t);
             if (i + 2 < ng) {
                 const int q = warp + (i + 2) * kWarps;
-                load_b<R>(e0, slotB, v.d_out, sl, q, g, t);
-                load_y<R>(e0, yrow, row_ok, sl, q, t);
+                load_b<R, YT>(e0, slotB, v.d_out, sl, q, g, t);
+                load_y<R, YT>(e0, yrow, row_ok, sl, q, t);
             }
             if (i + 1 < ng) {
-                mma_expand_store<R>(e1, ah, al, scale, yrow, store, sl, warp + (i + 1) * kWarps, t);
+                mma_expand_store<R, YT>(e1, ah, al, scale, yrow, store, sl, warp + (i + 1) * kWarps, t);
                 if (i + 3 < ng) {
                     const int q = warp + (i + 3) * kWarps;
-                    load_b<R>(e1, slotB, v.d_out, sl, q, g, t);
-                    load_y<R>(e1, yrow, row_ok, sl, q, t);
+                    load_b<R, YT>(e1, slotB, v.d_out, sl, q, g, t);
+                    load_y<R, YT>(e1, yrow, row_ok, sl, q, t);
                 }
             }
         }
@@ -648,7 +726,7 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
 // work item is (tile, projection), projection fastest, so the clusters working on one
 // tile's projections run side by side and its X rows come from HBM once (the later
 // reads hit L2).  Otherwise the only projection is p.proj[0].
-template <int RMAX, int MODE, int NT, bool FUSED>
+template <int RMAX, int MODE, int NT, bool FUSED, int DT = 0>
 __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
     lora_decode_kernel(const __grid_constant__ TileParams p)
 {
@@ -676,7 +754,7 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
         cluster_arrive_release();
         cluster_wait_acquire();
     }
-    if (p.early) prefetch_first_tile<RMAX, MODE, NT>(p, p.proj[k], tile, ctl, crank);
+    if (p.early) prefetch_first_tile<RMAX, MODE, NT, DT>(p, p.proj[k], tile, ctl, crank);
     griddep_wait();
     const int item2 = item + n_clusters;   // this cluster's next work item
     const int total = scan_tiles<false, NT, MODE, RMAX>(p, p.proj[k].slot_gen, tile, item2 / np,
@@ -714,23 +792,23 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
             if (R == 0 || R > RMAX) R = 8;   // rejected inside; moves rank-8 bytes
         }
         if (R == 8) {
-            run_tile<RMAX, MODE, 8, NT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+            run_tile<RMAX, MODE, 8, NT, DT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else if (R == 16) {
             if constexpr (RMAX >= 16)
-                run_tile<RMAX, MODE, 16, NT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+                run_tile<RMAX, MODE, 16, NT, DT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else if (R == 32) {
             if constexpr (RMAX >= 32)
-                run_tile<RMAX, MODE, 32, NT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+                run_tile<RMAX, MODE, 32, NT, DT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else {
             if constexpr (RMAX >= 64)
-                run_tile<RMAX, MODE, 64, NT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+                run_tile<RMAX, MODE, 64, NT, DT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         }
         __syncthreads();   // ctl and the H buffers are rewritten by the next tile
     }
 }
 
 // Clusters of `cluster` CTAs of this kernel resident at once (cached per device).
-template <int RMAX, int MODE, int NT, bool FUSED>
+template <int RMAX, int MODE, int NT, bool FUSED, int DT = 0>
 cudaError_t active_clusters(int cluster, int &active)
 {
     static std::mutex mu;
@@ -751,14 +829,14 @@ cudaError_t active_clusters(int cluster, int &active)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaOccupancyMaxActiveClusters(&active, lora_decode_kernel<RMAX, MODE, NT, FUSED>, &cfg);
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&active, lora_decode_kernel<RMAX, MODE, NT, FUSED, DT>, &cfg);
     if (e != cudaSuccess) return e;
     if (active <= 0) return cudaErrorInvalidConfiguration;
     cached[dev][cluster] = active;
     return cudaSuccess;
 }
 
-template <int RMAX, int MODE, int NT, bool FUSED>
+template <int RMAX, int MODE, int NT, bool FUSED, int DT = 0>
 cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, int active,
                        cudaStream_t stream)
 {
@@ -779,7 +857,7 @@ cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, int 
     cfg.numAttrs = p.early ? 2 : 1;
     const int64_t n = max_tiles < active ? max_tiles : active;
     cfg.gridDim = dim3((unsigned)(n * cluster), 1, 1);
-    return cudaLaunchKernelEx(&cfg, lora_decode_kernel<RMAX, MODE, NT, FUSED>, p);
+    return cudaLaunchKernelEx(&cfg, lora_decode_kernel<RMAX, MODE, NT, FUSED, DT>, p);
 }
 
 // CTA width.  256 threads keep each warp's operands in one round of loads; when the
@@ -787,24 +865,39 @@ cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, int 
 // long decode segments), 128-thread CTAs let twice as many tiles be in flight, which
 // hides more latency than their second round of loads costs (measured: a 4096 x 4096
 // batch of 60 tiles is 36% slower with 128 threads, batches of 300+ tiles 3-6% faster).
-template <int RMAX, int MODE, bool FUSED = false>
+template <int RMAX, int MODE, bool FUSED = false, int DT = 0>
 cudaError_t launch_mode(const TileParams &p, int cluster, int64_t max_tiles, cudaStream_t stream)
 {
     int active = 0;
-    cudaError_t e = active_clusters<RMAX, MODE, 256, FUSED>(cluster, active);
+    cudaError_t e = active_clusters<RMAX, MODE, 256, FUSED, DT>(cluster, active);
     if (e != cudaSuccess) return e;
     if (2 * max_tiles > 3 * (int64_t)active) {
         int active128 = 0;
-        e = active_clusters<RMAX, MODE, 128, FUSED>(cluster, active128);
+        e = active_clusters<RMAX, MODE, 128, FUSED, DT>(cluster, active128);
         if (e != cudaSuccess) return e;
         // Early launch with adapter prefetch only pays for batches of about one wave of
         // tiles: with many more, the prefetched slices thrash L2 and the early CTAs
         // hold slots (measured 16% slower on 2048 decode rows over 128 adapters).
         TileParams q = p;
         q.early = 0;
-        return launch_one<RMAX, MODE, 128, FUSED>(q, cluster, max_tiles, active128, stream);
+        return launch_one<RMAX, MODE, 128, FUSED, DT>(q, cluster, max_tiles, active128, stream);
     }
-    return launch_one<RMAX, MODE, 256, FUSED>(p, cluster, max_tiles, active, stream);
+    return launch_one<RMAX, MODE, 256, FUSED, DT>(p, cluster, max_tiles, active, stream);
+}
+
+// The fused apply with another dtype boundary (DT != 0: FP8 X codes and / or an fp16 or
+// fp32 base output).
+template <int RMAX>
+cudaError_t launch_dt(int dt, const TileParams &p, int cluster, int64_t max_tiles, cudaStream_t stream)
+{
+    switch (dt) {
+    case 1: return launch_mode<RMAX, MODE_APPLY, false, 1>(p, cluster, max_tiles, stream);
+    case 2: return launch_mode<RMAX, MODE_APPLY, false, 2>(p, cluster, max_tiles, stream);
+    case 3: return launch_mode<RMAX, MODE_APPLY, false, 3>(p, cluster, max_tiles, stream);
+    case 4: return launch_mode<RMAX, MODE_APPLY, false, 4>(p, cluster, max_tiles, stream);
+    case 5: return launch_mode<RMAX, MODE_APPLY, false, 5>(p, cluster, max_tiles, stream);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 template <int RMAX>
@@ -839,12 +932,32 @@ cudaError_t set_attrs_nt()
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX, NT>::SMEM);
 }
 
+template <int RMAX, int NT, int DT>
+cudaError_t set_attrs_dt()
+{
+    return cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_APPLY, NT, false, DT>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX, NT>::SMEM);
+}
+
+template <int RMAX, int NT>
+cudaError_t set_attrs_dts()
+{
+    cudaError_t e;
+    if ((e = set_attrs_dt<RMAX, NT, 1>()) != cudaSuccess) return e;
+    if ((e = set_attrs_dt<RMAX, NT, 2>()) != cudaSuccess) return e;
+    if ((e = set_attrs_dt<RMAX, NT, 3>()) != cudaSuccess) return e;
+    if ((e = set_attrs_dt<RMAX, NT, 4>()) != cudaSuccess) return e;
+    return set_attrs_dt<RMAX, NT, 5>();
+}
+
 template <int RMAX>
 cudaError_t set_attrs()
 {
     cudaError_t e = set_attrs_nt<RMAX, 256>();
     if (e != cudaSuccess) return e;
-    return set_attrs_nt<RMAX, 128>();
+    if ((e = set_attrs_nt<RMAX, 128>()) != cudaSuccess) return e;
+    if ((e = set_attrs_dts<RMAX, 256>()) != cudaSuccess) return e;
+    return set_attrs_dts<RMAX, 128>();
 }
 
 // Repack: A [rank, d_in] -> [d_in/8][R][8]; B [d_out, rank] -> [R/8][d_out][8]; zero
@@ -895,6 +1008,19 @@ __global__ void publish_slot_kernel(int32_t *rank_entry, float *scale_entry, uin
 }
 
 }  // namespace
+
+cudaError_t launch_tile_kernel_dt(int dt, int rmax_bucket, const TileParams &p, int cluster, int64_t max_tiles,
+                                  cudaStream_t stream)
+{
+    if (cluster < 1 || cluster > kMaxCluster || max_tiles < 1) return cudaErrorInvalidValue;
+    switch (rmax_bucket) {
+    case 8: return launch_dt<8>(dt, p, cluster, max_tiles, stream);
+    case 16: return launch_dt<16>(dt, p, cluster, max_tiles, stream);
+    case 32: return launch_dt<32>(dt, p, cluster, max_tiles, stream);
+    case 64: return launch_dt<64>(dt, p, cluster, max_tiles, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
 
 cudaError_t launch_tile_kernel(int mode, int rmax_bucket, const TileParams &p, int cluster,
                                int64_t max_tiles, cudaStream_t stream)

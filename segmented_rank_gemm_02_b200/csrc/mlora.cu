@@ -572,6 +572,48 @@ mlora_status mlora_apply(mlora_pool *pool, const mlora_segments *segs, const voi
     return launch(pool, segs, mlora::MODE_APPLY, p, stream);
 }
 
+mlora_status mlora_apply_ex(mlora_pool *pool, const mlora_segments *segs, const void *X, int32_t x_dtype,
+                            float x_scale, int64_t ldx, void *Y, int32_t y_dtype, int64_t ldy, void *stream)
+{
+    if (x_dtype != MLORA_DTYPE_BF16 && x_dtype != MLORA_DTYPE_FP8_E4M3) return MLORA_ERR_INVALID_ARG;
+    if (y_dtype != MLORA_DTYPE_BF16 && y_dtype != MLORA_DTYPE_FP16 && y_dtype != MLORA_DTYPE_FP32)
+        return MLORA_ERR_INVALID_ARG;
+    if (x_dtype == MLORA_DTYPE_BF16 && y_dtype == MLORA_DTYPE_BF16)
+        return mlora_apply(pool, segs, X, ldx, Y, ldy, stream);
+    mlora_status st = check_segments(pool, segs);
+    if (st != MLORA_OK) return st;
+    const bool x8 = x_dtype == MLORA_DTYPE_FP8_E4M3;
+    if (x8 && (!std::isfinite(x_scale) || pool->d_in % 16 != 0)) return MLORA_ERR_INVALID_ARG;
+    if (segs->n_segments == 0 || segs->n_tokens == 0) return MLORA_OK;
+    if (X == nullptr || Y == nullptr || !aligned16(X) || !aligned16(Y)) return MLORA_ERR_INVALID_ARG;
+    // rows of whole 16-byte vectors
+    const int64_t x_vec = x8 ? 16 : 8, y_vec = y_dtype == MLORA_DTYPE_FP32 ? 4 : 8;
+    if (ldx < pool->d_in || ldx % x_vec != 0 || ldy < pool->d_out || ldy % y_vec != 0) return MLORA_ERR_INVALID_ARG;
+    DeviceGuard guard(pool->device);
+    if (!guard.ok) return MLORA_ERR_CUDA;
+    mlora::TileParams p = base_params(pool, segs);
+    p.X = static_cast<const __nv_bfloat16 *>(X);   // (element type per x_dtype)
+    p.ldx = ldx;
+    p.Y = static_cast<__nv_bfloat16 *>(Y);         // (element type per y_dtype)
+    p.ldy = ldy;
+    p.x_scale = x8 ? x_scale : 1.f;
+    const int c = choose_cluster(pool->d_in, pool->d_out);
+    p.k_slice = (int32_t)round_up((pool->d_in + c - 1) / c, 32);
+    p.n_slice = (int32_t)round_up((pool->d_out + c - 1) / c, 8);
+    set_single_projection(p);
+    // every segment takes the decode-shaped kernel (the tensor-memory kernels are bf16 only)
+    p.long_rows = 0x7fffffff;
+    p.early = 1;
+    st = prepare_device(pool->device);
+    if (st != MLORA_OK) return st;
+    const int dt = 3 * (x8 ? 1 : 0) + (y_dtype == MLORA_DTYPE_FP16 ? 1 : y_dtype == MLORA_DTYPE_FP32 ? 2 : 0);
+    const int64_t tiles = (int64_t)segs->n_segments + (int64_t)segs->n_tokens / mlora::kTileRows + 1;
+    if (mlora::launch_tile_kernel_dt(dt, pool->r_bucket_max, p, c, tiles, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+        return MLORA_ERR_CUDA;
+    return MLORA_OK;
+}
+
 mlora_status mlora_apply_multi(mlora_pool *const *pools, int32_t n_proj, const mlora_segments *segs,
                                const void *X, int64_t ldx, void *const *Y, const int64_t *ldy,
                                void *stream)
