@@ -244,6 +244,32 @@ mlora_status mlora_apply(mlora_pool *pool, const mlora_segments *segs, const voi
 mlora_status mlora_apply_ex(mlora_pool *pool, const mlora_segments *segs, const void *X, int32_t x_dtype,
                             float x_scale, int64_t ldx, void *Y, int32_t y_dtype, int64_t ldy, void *stream);
 
+/*
+ * The base projection and the LoRA delta in one pass (page "LoRA/QLoRA multi-tenant
+ * serving", section 3.3 on fusing W0 x + B(A x) into one kernel, and its paragraph on
+ * cuBLASLt epilogue fusion after section 5.3):
+ *
+ *   Y[t, :] = bf16(X[t, :] W^T + s_g (X[t, :] A_a^T) B_a^T)   rows t of adapter segments
+ *   Y[t, :] = bf16(X[t, :] W^T)                                every other row
+ *
+ * with the whole sum in fp32 and one rounding.  Unlike mlora_apply, Y is an output
+ * only: it is never read, and every row of it is written.  The shrink runs first (as
+ * in mlora_shrink, into the pool's workspace); then a tensor-core GEMM adds each
+ * 128-row tile's low-rank products (one per distinct adapter among its rows, on the
+ * same fp32 H as the other entry points) into the accumulator of X W^T before the
+ * single store.
+ * X: device bf16 [n_rows, d_in] (row stride ldx); W: the base weight, device bf16
+ * [d_out, d_in] (row stride ldw, the nn.Linear layout); Y: device bf16
+ * [n_rows, d_out] (row stride ldy).  Strides are multiples of 8 elements, pointers
+ * 16-byte aligned (else MLORA_ERR_INVALID_ARG).  The workspace (H, a 16-byte row map
+ * per row and per 128 rows a list of slots) is the pool's, grown as for mlora_apply
+ * (not during stream capture: MLORA_ERR_UNSUPPORTED) and shared with it.  Segments
+ * that mlora_apply rejects set the same status bits here and their rows get X W^T
+ * only; a row claimed by two segments keeps one claim and sets MLORA_FLAG_BAD_ROW.
+ */
+mlora_status mlora_base_gemm_apply(mlora_pool *pool, const mlora_segments *segs, const void *X, int64_t ldx,
+                                   const void *W, int64_t ldw, void *Y, int64_t ldy, void *stream);
+
 /* Projections one mlora_apply_multi call may cover. */
 #define MLORA_MAX_FUSED 4
 

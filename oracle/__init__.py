@@ -236,6 +236,20 @@ def apply_rows_xf64(X: np.ndarray, Y0: np.ndarray, row_slot, row_scale, slot_ran
     return Y, int(flags)
 
 
+def base_gemm_apply(X: np.ndarray, W: np.ndarray, row_slot, row_scale, slot_rank, slot_alpha,
+                    A: Dict[int, np.ndarray], B: Dict[int, np.ndarray],
+                    n_threads: int = 0) -> Tuple[np.ndarray, int]:
+    """The base projection and the LoRA branch together (page "LoRA/QLoRA multi-tenant
+    serving", section 3.3, W0 x + B(A x) in one kernel; page "Multi-LoRA Serving:
+    adapter batching", section "LoRA on one Linear layer", Y = X W^T + s (X A^T) B^T):
+    Y[t] = X[t] W^T + s_a (X[t] A_a^T) B_a^T for rows of adapter a, X[t] W^T for base
+    rows, in fp64.  ``X`` [n_rows, d_in] and ``W`` [d_out, d_in] (the nn.Linear
+    layout) are bf16 bits.  The base term is a library fp64 matmul of the exact bf16
+    values; it is then the Y0 of the per-row entry.  Returns ``(Y, flags)``."""
+    base = bf16_to_f64(X) @ bf16_to_f64(W).T
+    return apply_rows(X, base, row_slot, row_scale, slot_rank, slot_alpha, A, B, n_threads)
+
+
 def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
     """Exact values of FP8 e4m3 codes (1 sign bit, 4 exponent bits with bias 7, 3
     mantissa bits; exponent field 0 is subnormal, 2^-6 * m/8; S.1111.111 is NaN and

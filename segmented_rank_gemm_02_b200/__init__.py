@@ -31,7 +31,8 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_OUT_OF_MEMORY, ERR_BAD_METADATA, ERR_C
 EXPORTS = ("mlora_pool_create", "mlora_pool_destroy", "mlora_pool_load_slot",
            "mlora_pool_clear_slot", "mlora_pool_slot_info", "mlora_pool_shape",
            "mlora_pool_check", "mlora_shrink", "mlora_expand", "mlora_apply",
-           "mlora_apply_noalloc", "mlora_apply_multi", "mlora_apply_ex", "mlora_build_segments", "mlora_status_string",
+           "mlora_apply_noalloc", "mlora_apply_multi", "mlora_apply_ex", "mlora_base_gemm_apply",
+           "mlora_build_segments", "mlora_status_string",
            "mlora_version", "mlora_pool_slot_generation", "mlora_slot_cache_create",
            "mlora_slot_cache_destroy", "mlora_slot_cache_acquire", "mlora_slot_cache_release",
            "mlora_slot_cache_invalidate", "mlora_slot_cache_lookup", "mlora_slot_cache_stats")
@@ -71,6 +72,7 @@ def _load():
         "mlora_apply": [vp, seg_p, vp, i64, vp, i64, vp],
         "mlora_apply_noalloc": [vp, seg_p, vp, i64, vp, i64, vp],
         "mlora_apply_ex": [vp, seg_p, vp, i32, f32, i64, vp, i32, i64, vp],
+        "mlora_base_gemm_apply": [vp, seg_p, vp, i64, vp, i64, vp, i64, vp],
         "mlora_apply_multi": [ctypes.POINTER(vp), i32, seg_p, vp, i64, ctypes.POINTER(vp),
                               ctypes.POINTER(i64), vp],
         "mlora_build_segments": [vp, i32, vp, vp, vp, i32p, i32p, vp, vp],
@@ -306,6 +308,15 @@ def apply_ex(pool: Pool, segs: DeviceSegments, X, Y, x_scale: float = 1.0, strea
     _check(lib().mlora_apply_ex(pool.handle, ctypes.byref(segs.struct), _ptr(X), _dtype_code(X), float(x_scale),
                                 _ld(X, "X"), _ptr(Y), _dtype_code(Y), _ld(Y, "Y"), _stream_ptr(stream)),
            "mlora_apply_ex")
+
+
+def base_gemm_apply(pool: Pool, segs: DeviceSegments, X, W, Y, stream=None) -> None:
+    """Y = bf16(X W^T + s (X A^T) B^T) for adapter rows, bf16(X W^T) for the others, in
+    one pass (mlora_base_gemm_apply).  X [n_rows, d_in], W [d_out, d_in] (nn.Linear
+    layout) and Y [n_rows, d_out], all bf16 on the pool's device; Y is written, not read."""
+    _check(lib().mlora_base_gemm_apply(pool.handle, ctypes.byref(segs.struct), _ptr(X), _ld(X, "X"), _ptr(W),
+                                       _ld(W, "W"), _ptr(Y), _ld(Y, "Y"), _stream_ptr(stream)),
+           "mlora_base_gemm_apply")
 
 
 def apply_multi(pools, segs: DeviceSegments, X, Ys, stream=None) -> None:

@@ -23,7 +23,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmlora.so")
 
-SOURCES = ["mlora.cu", "lora_decode.cu", "lora_prefill.cu", "noalloc.cu", "slot_cache.cu"]
+SOURCES = ["mlora.cu", "lora_decode.cu", "lora_prefill.cu", "base_gemm.cu", "noalloc.cu", "slot_cache.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
          "-I", INCLUDE, "-I", CSRC]

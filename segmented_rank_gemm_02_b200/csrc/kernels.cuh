@@ -173,4 +173,35 @@ cudaError_t launch_publish_slot(int32_t *slot_rank_entry, float *slot_scale_entr
                                 uint32_t *slot_gen_entry, int rank, float scale,
                                 uint32_t generation, cudaStream_t stream);
 
+// ---- fused base GEMM + LoRA (base_gemm.cu)
+
+constexpr int kGemmRows = 128;   // rows of Y per GEMM tile
+constexpr int kGemmCols = 256;   // columns of Y per GEMM tile
+// Per 128-row block: the number of distinct slots, then (slot, rank bucket) pairs.
+constexpr int kBlockSlotsPitch = 1 + 2 * kGemmRows;
+
+// Everything one launch of the fused base GEMM needs.  Passed by value.
+struct GemmParams {
+    CUtensorMap x_map;          // X [n_rows][d_in] bf16, box 64 x 128, 128-byte swizzle
+    CUtensorMap w_map;          // W [d_out][d_in] bf16, box 64 x 256, 128-byte swizzle
+    CUtensorMap b_map[4];       // the pool's B blocks per rank bucket 8..64, box {8, 256, R/8, 1}
+    const int4 *row_info;       // [n_rows] {grouped position or -1, slot, scale bits, rank}
+    const int32_t *block_slots; // [n_mblk][kBlockSlotsPitch]
+    const float *H;             // [n_tokens][ldh] fp32, grouped order (the shrink's output)
+    int64_t ldh;
+    __nv_bfloat16 *Y;           // [n_rows][ldy] bf16, written for every row
+    int64_t ldy;
+    unsigned int *status;
+    int32_t n_rows, d_in, d_out, n_mblk, n_nblk;
+};
+
+// row_info for every row (memset to -1, then the valid segments' rows); reports the
+// segments' problems in p.status.
+cudaError_t launch_row_map(const TileParams &p, int4 *row_info, cudaStream_t stream);
+// The distinct slots of each 128-row block of rows.
+cudaError_t launch_block_slots(const int4 *row_info, int n_rows, int32_t *block_slots, cudaStream_t stream);
+// Persistent GEMM over all (128-row, 256-column) tiles, one CTA per SM.
+cudaError_t launch_base_gemm(const GemmParams &p, cudaStream_t stream);
+cudaError_t prepare_base_gemm();
+
 }  // namespace mlora

@@ -42,6 +42,8 @@ struct mlora_pool {
     // TMA views of the B blocks for rank buckets 8, 16, 32, 64 (those <= r_bucket_max):
     // one load brings one 128-column chunk of one slot's B, all its rank groups
     CUtensorMap b_maps[4];
+    // the same views with 256-column boxes (one B chunk per tile of the fused base GEMM)
+    CUtensorMap b_maps256[4];
     bool b_maps_ok;
 };
 
@@ -78,6 +80,7 @@ mlora_status prepare_device(int dev)
     if (g_prepared[dev]) return MLORA_OK;
     if (mlora::prepare_tile_kernels() != cudaSuccess) return MLORA_ERR_CUDA;
     if (mlora::prepare_long_kernels() != cudaSuccess) return MLORA_ERR_CUDA;
+    if (mlora::prepare_base_gemm() != cudaSuccess) return MLORA_ERR_CUDA;
     g_prepared[dev] = true;
     return MLORA_OK;
 }
@@ -167,15 +170,15 @@ bool encode_rows_map(CUtensorMap *map, const void *base, int64_t rows, int64_t c
 }
 
 // The pool's B blocks as a 4-D tensor [slot][rank group][d_out][8] (bf16), box
-// {8, 128, R/8, 1}: one 128-column chunk of one slot's B for rank bucket R.
-bool encode_b_map(CUtensorMap *map, const mlora_pool *pool, int R)
+// {8, cols, R/8, 1}: one chunk of `cols` columns of one slot's B for rank bucket R.
+bool encode_b_map(CUtensorMap *map, const mlora_pool *pool, int R, int cols)
 {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (enc == nullptr) return false;
     const int groups = pool->r_bucket_max / 8;
     cuuint64_t dims[4] = {8, (cuuint64_t)pool->d_out, (cuuint64_t)groups, (cuuint64_t)pool->n_slots};
     cuuint64_t strides[3] = {16, (cuuint64_t)pool->d_out * 16, (cuuint64_t)pool->slot_stride * 2};
-    cuuint32_t box[4] = {8, (cuuint32_t)mlora::kExpandChunk, (cuuint32_t)(R / 8), 1};
+    cuuint32_t box[4] = {8, (cuuint32_t)cols, (cuuint32_t)(R / 8), 1};
     cuuint32_t elem[4] = {1, 1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, pool->buf + pool->b_offset, dims, strides, box,
                elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -415,7 +418,9 @@ mlora_status mlora_pool_create(int32_t d_in, int32_t d_out, int32_t n_slots, int
     if (st == MLORA_OK) {
         pool->b_maps_ok = tensor_map_encoder() != nullptr;
         for (int i = 0; i < 4 && pool->b_maps_ok; ++i)
-            if ((8 << i) <= rb) pool->b_maps_ok = encode_b_map(&pool->b_maps[i], pool, 8 << i);
+            if ((8 << i) <= rb)
+                pool->b_maps_ok = encode_b_map(&pool->b_maps[i], pool, 8 << i, mlora::kExpandChunk) &&
+                                  encode_b_map(&pool->b_maps256[i], pool, 8 << i, mlora::kGemmCols);
     }
     if (st != MLORA_OK) {
         cudaGetLastError();   // clear a sticky allocation error
@@ -612,6 +617,73 @@ mlora_status mlora_apply_ex(mlora_pool *pool, const mlora_segments *segs, const 
         cudaSuccess)
         return MLORA_ERR_CUDA;
     return MLORA_OK;
+}
+
+mlora_status mlora_base_gemm_apply(mlora_pool *pool, const mlora_segments *segs, const void *X, int64_t ldx,
+                                   const void *W, int64_t ldw, void *Y, int64_t ldy, void *stream)
+{
+    mlora_status st = check_segments(pool, segs);
+    if (st != MLORA_OK) return st;
+    if (segs->n_rows == 0) return MLORA_OK;
+    if (X == nullptr || W == nullptr || Y == nullptr || !aligned16(X) || !aligned16(W) || !aligned16(Y))
+        return MLORA_ERR_INVALID_ARG;
+    if (ldx < pool->d_in || ldx % 8 != 0 || ldw < pool->d_in || ldw % 8 != 0 || ldy < pool->d_out ||
+        ldy % 8 != 0)
+        return MLORA_ERR_INVALID_ARG;
+    if (!pool->b_maps_ok) return MLORA_ERR_UNSUPPORTED;
+    DeviceGuard guard(pool->device);
+    if (!guard.ok) return MLORA_ERR_CUDA;
+    st = prepare_device(pool->device);
+    if (st != MLORA_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const int rk = std::max(16, pool->r_bucket_max);
+    const int64_t n_mblk = (segs->n_rows + mlora::kGemmRows - 1) / mlora::kGemmRows;
+    const int64_t n_nblk = (pool->d_out + mlora::kGemmCols - 1) / mlora::kGemmCols;
+    // workspace: H (grouped order), the row map, the slot lists of the row blocks
+    const size_t h_bytes = (size_t)round_up((int64_t)segs->n_tokens * rk * 4, 256);
+    const size_t map_bytes = (size_t)round_up((int64_t)segs->n_rows * 16, 256);
+    const size_t slot_bytes = (size_t)n_mblk * mlora::kBlockSlotsPitch * 4;
+    std::lock_guard<std::mutex> lock(pool->ws_mutex);   // held until the kernels are launched
+    st = ensure_workspace(pool, h_bytes + map_bytes + slot_bytes, cs);
+    if (st != MLORA_OK) return st;
+    uint8_t *ws = reinterpret_cast<uint8_t *>(pool->ws);
+    float *H = reinterpret_cast<float *>(ws);
+    int4 *row_info = reinterpret_cast<int4 *>(ws + h_bytes);
+    int32_t *block_slots = reinterpret_cast<int32_t *>(ws + h_bytes + map_bytes);
+
+    // 1. H = X A^T for every valid segment (decode-shaped and long-segment kernels)
+    mlora::TileParams p = base_params(pool, segs);
+    p.X = static_cast<const __nv_bfloat16 *>(X);
+    p.ldx = ldx;
+    p.H = H;
+    p.ldh = rk;
+    if (segs->n_segments > 0 && segs->n_tokens > 0) {
+        st = launch(pool, segs, mlora::MODE_SHRINK, p, stream);
+        if (st != MLORA_OK) return st;
+    }
+    // 2. each row's grouped position, slot, scale and rank; each row block's slots
+    if (mlora::launch_row_map(p, row_info, cs) != cudaSuccess ||
+        mlora::launch_block_slots(row_info, segs->n_rows, block_slots, cs) != cudaSuccess)
+        return MLORA_ERR_CUDA;
+    // 3. Y = X W^T + s (H B^T) per tile
+    mlora::GemmParams g{};
+    if (!encode_rows_map(&g.x_map, X, segs->n_rows, pool->d_in, ldx, mlora::kGemmRows) ||
+        !encode_rows_map(&g.w_map, W, pool->d_out, pool->d_in, ldw, mlora::kGemmCols))
+        return MLORA_ERR_CUDA;
+    for (int i = 0; i < 4; ++i) g.b_map[i] = pool->b_maps256[i];
+    g.row_info = row_info;
+    g.block_slots = block_slots;
+    g.H = H;
+    g.ldh = rk;
+    g.Y = static_cast<__nv_bfloat16 *>(Y);
+    g.ldy = ldy;
+    g.status = pool->d_status;
+    g.n_rows = segs->n_rows;
+    g.d_in = pool->d_in;
+    g.d_out = pool->d_out;
+    g.n_mblk = (int32_t)n_mblk;
+    g.n_nblk = (int32_t)n_nblk;
+    return mlora::launch_base_gemm(g, cs) == cudaSuccess ? MLORA_OK : MLORA_ERR_CUDA;
 }
 
 mlora_status mlora_apply_multi(mlora_pool *const *pools, int32_t n_proj, const mlora_segments *segs,

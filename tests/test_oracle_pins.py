@@ -464,3 +464,99 @@ def test_fp64_activation_is_linear_in_the_activation():
 MUTANT_CHECKS = PIN_CHECKS + [test_fp64_activation_entry_equals_bf16_entry,
                               test_fp64_activation_merged_weight_identity_with_fp8_codes,
                               test_fp64_activation_is_linear_in_the_activation]
+
+
+# ---------------------------------------------------------------------------
+# the base projection and the LoRA branch together (page "LoRA/QLoRA multi-tenant
+# serving", section 3.3: W0 x + B(A x) in one kernel)
+# ---------------------------------------------------------------------------
+
+def _base_problem(seed, n_rows, d_in, d_out, ranks, base_rows):
+    rng = np.random.default_rng(seed)
+    P = _small_problem(seed=seed, n_rows=n_rows, d_in=d_in, d_out=d_out, n_slots=len(ranks), ranks=ranks,
+                       base_rows=base_rows)
+    P["W"] = _bf16(rng.normal(0, 0.5, (d_out, d_in)))
+    return P
+
+
+def check_base_gemm_brute_force_tiny(fn=None):
+    # every output element as explicit sums over k and over the rank, in Python floats
+    fn = fn or oracle.base_gemm_apply
+    P = _base_problem(41, n_rows=5, d_in=6, d_out=4, ranks=(2, 1), base_rows=(3,))
+    Y, flags = fn(P["X"], P["W"], P["row_slot"], None, P["slot_rank"], P["slot_alpha"], P["A"], P["B"])
+    assert flags == 0
+    x, w = oracle.bf16_to_f64(P["X"]), oracle.bf16_to_f64(P["W"])
+    for t in range(5):
+        a = int(P["row_slot"][t])
+        for o in range(4):
+            want = sum(float(x[t, k]) * float(w[o, k]) for k in range(6))
+            if a >= 0:
+                r = int(P["slot_rank"][a])
+                s = float(P["slot_alpha"][a]) / r
+                av, bv = oracle.bf16_to_f64(P["A"][a]), oracle.bf16_to_f64(P["B"][a])
+                for q in range(r):
+                    h = sum(float(x[t, k]) * float(av[q, k]) for k in range(6))
+                    want += s * h * float(bv[o, q])
+            assert abs(Y[t, o] - want) <= 1e-12 * (1 + abs(want)), (t, o)
+
+
+def check_base_gemm_merged_weight(fn=None):
+    # adapter rows see the merged weight W + s B A, base rows W alone; square W, so a
+    # missing transpose shows too
+    fn = fn or oracle.base_gemm_apply
+    P = _base_problem(42, n_rows=20, d_in=32, d_out=32, ranks=(3, 5, 2), base_rows=(0, 9))
+    Y, flags = fn(P["X"], P["W"], P["row_slot"], None, P["slot_rank"], P["slot_alpha"], P["A"], P["B"])
+    assert flags == 0
+    x, w = oracle.bf16_to_f64(P["X"]), oracle.bf16_to_f64(P["W"])
+    for t in range(20):
+        a = int(P["row_slot"][t])
+        Wt = w
+        if a >= 0:
+            s = P["slot_alpha"][a] / P["slot_rank"][a]
+            Wt = w + s * oracle.bf16_to_f64(P["B"][a]) @ oracle.bf16_to_f64(P["A"][a])
+        want = np.einsum("k,ok->o", x[t], Wt)
+        assert np.allclose(Y[t], want, rtol=1e-12, atol=1e-12), t
+
+
+def check_base_gemm_zero_weight_is_the_lora_branch(fn=None):
+    # W = 0: exactly the LoRA branch onto a zero base output
+    fn = fn or oracle.base_gemm_apply
+    P = _base_problem(43, n_rows=16, d_in=24, d_out=20, ranks=(4, 2), base_rows=(2,))
+    Z = np.zeros_like(P["W"])
+    Y, _ = fn(P["X"], Z, P["row_slot"], None, P["slot_rank"], P["slot_alpha"], P["A"], P["B"])
+    Yl, _ = oracle.apply_rows(P["X"], np.zeros((16, 20)), P["row_slot"], None, P["slot_rank"], P["slot_alpha"],
+                              P["A"], P["B"])
+    assert np.array_equal(Y, Yl) and np.all(Y[2] == 0)
+
+
+BASE_GEMM_CHECKS = [check_base_gemm_brute_force_tiny, check_base_gemm_merged_weight,
+                    check_base_gemm_zero_weight_is_the_lora_branch]
+
+
+@pytest.mark.parametrize("check", BASE_GEMM_CHECKS, ids=[c.__name__ for c in BASE_GEMM_CHECKS])
+def test_base_gemm_pin(check):
+    check()
+
+
+BASE_GEMM_MUTANTS = {
+    "untransposed_W": ("bf16_to_f64(W).T", "bf16_to_f64(W)"),
+    "dropped_base_term": ("return apply_rows(X, base,", "return apply_rows(X, 0 * base,"),
+    "base_from_adapter_input": ("base = bf16_to_f64(X) @", "base = bf16_to_f64(X[::-1]) @"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(BASE_GEMM_MUTANTS))
+def test_base_gemm_planted_mistake_is_caught(name):
+    import inspect
+    find, repl = BASE_GEMM_MUTANTS[name]
+    src = inspect.getsource(oracle.base_gemm_apply)
+    assert src.count(find) == 1, name
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(find, repl), "<mutant>", "exec"), ns)
+    failed = []
+    for check in BASE_GEMM_CHECKS:
+        try:
+            check(ns["base_gemm_apply"])
+        except (AssertionError, ValueError):
+            failed.append(check.__name__)
+    assert failed, f"mutant {name} passed every pin"

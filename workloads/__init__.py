@@ -31,6 +31,8 @@ Recipe (per workload seed):
   * each projection ``j`` (0-based, in the listed order) draws from
     ``default_rng([seed, j + 1])``: A then B for every referenced slot in
     ascending slot order, then X, then Y0.
+  * the base weight W of projection ``j`` (used where the base GEMM itself is part
+    of the computation) comes from ``default_rng([seed, j + 1, 87])``.
 
 ``scale_rows`` shrinks the row counts (same structure, fewer rows) so the oracle
 finishes in seconds; full-size workloads are used for sampled parity checks and
@@ -131,6 +133,13 @@ class Workload:
         if cache:
             self._proj_cache[j] = p
         return p
+
+    def base_weight(self, j: int) -> np.ndarray:
+        """Base weight W [d_out, d_in] of projection ``j`` (nn.Linear layout), bf16 bits
+        drawn N(0, 0.02) from its own stream ``default_rng([seed, j + 1, 87])``, so that
+        the projection's other draws do not depend on whether it is made."""
+        _, d_in, d_out = self.proj_shapes[j]
+        return _normal_bf16(np.random.default_rng([self.seed, j + 1, 87]), (d_out, d_in), WEIGHT_STD)
 
     def projections(self):
         for j in range(len(self.proj_shapes)):
