@@ -99,8 +99,10 @@ struct TileParams {
     // 64 x 128 tiles for runs of consecutive rows, 64 x 1 rows for gathers
     CUtensorMap x_tile, x_rows, y_tile, y_rows;
     // TMA views of the pool's B blocks, one per rank bucket 8, 16, 32, 64: a box is
-    // one 128-column chunk of one slot's B (all its rank groups)
+    // one 128-column chunk of one slot's B (all its rank groups), [R/8][128][8] in
+    // shared memory; its second coordinate is (first column) / b_col_div
     CUtensorMap b_map[4];
+    int32_t b_col_div;
     // decode-shaped kernel: the projections it applies (1 unless fused; all share X,
     // d_in, the segment metadata and the slot numbering)
     int32_t n_proj;
@@ -175,16 +177,17 @@ cudaError_t launch_publish_slot(int32_t *slot_rank_entry, float *slot_scale_entr
 
 // ---- fused base GEMM + LoRA (base_gemm.cu)
 
-constexpr int kGemmRows = 128;   // rows of Y per GEMM tile
-constexpr int kGemmCols = 256;   // columns of Y per GEMM tile
-// Per 128-row block: the number of distinct slots, then (slot, rank bucket) pairs.
+constexpr int kGemmRows = 256;   // rows of Y per GEMM tile (a pair of CTAs, 128 each)
+// Per 256-row block: the number of distinct slots, then (slot, rank bucket) pairs.
 constexpr int kBlockSlotsPitch = 1 + 2 * kGemmRows;
 
 // Everything one launch of the fused base GEMM needs.  Passed by value.
 struct GemmParams {
     CUtensorMap x_map;          // X [n_rows][d_in] bf16, box 64 x 128, 128-byte swizzle
-    CUtensorMap w_map;          // W [d_out][d_in] bf16, box 64 x 256, 128-byte swizzle
-    CUtensorMap b_map[4];       // the pool's B blocks per rank bucket 8..64, box {8, 256, R/8, 1}
+    CUtensorMap w_map;          // W [d_out][d_in] bf16, box 64 x 128, 128-byte swizzle
+    CUtensorMap b_map[4];       // the pool's B blocks per rank bucket 8..64: one box is one slot's
+                                // 128-column chunk, [R/8][128][8] in shared memory
+    int32_t b_col_div;          // the box's second coordinate is (first column) / b_col_div
     const int4 *row_info;       // [n_rows] {grouped position or -1, slot, scale bits, rank}
     const int32_t *block_slots; // [n_mblk][kBlockSlotsPitch]
     const float *H;             // [n_tokens][ldh] fp32, grouped order (the shrink's output)
@@ -198,10 +201,13 @@ struct GemmParams {
 // row_info for every row (memset to -1, then the valid segments' rows); reports the
 // segments' problems in p.status.
 cudaError_t launch_row_map(const TileParams &p, int4 *row_info, cudaStream_t stream);
-// The distinct slots of each 128-row block of rows.
+// The distinct slots of each 256-row block of rows.
 cudaError_t launch_block_slots(const int4 *row_info, int n_rows, int32_t *block_slots, cudaStream_t stream);
-// Persistent GEMM over all (128-row, 256-column) tiles, one CTA per SM.
-cudaError_t launch_base_gemm(const GemmParams &p, cudaStream_t stream);
+// Tile width (256 or 512 columns of Y) for n_mblk 256-row blocks and d_out columns.
+int choose_gemm_cols(int n_mblk, int d_out);
+// Persistent GEMM over all (256-row, gn-column) tiles, one pair of CTAs per two SMs;
+// p.n_nblk = ceil(d_out / gn).
+cudaError_t launch_base_gemm(int gn, const GemmParams &p, cudaStream_t stream);
 cudaError_t prepare_base_gemm();
 
 }  // namespace mlora

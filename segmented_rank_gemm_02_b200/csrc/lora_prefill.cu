@@ -684,7 +684,7 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
                     if (ui.ok) bytes += (uint32_t)halves * PM * 64 * 2;
                     mbar_arrive_expect_tx(&ctl.full[s], bytes);
                     const int bi = ui.R == 8 ? 0 : ui.R == 16 ? 1 : ui.R == 32 ? 2 : 3;
-                    tma_load_4d(bs, &p.b_map[bi], 0, c0, 0, u.slot, &ctl.full[s]);
+                    tma_load_4d(bs, &p.b_map[bi], 0, c0 / p.b_col_div, 0, u.slot, &ctl.full[s]);
                     if (ui.ok && contiguous)
                         for (int h = 0; h < halves; ++h)
                             tma_load_2d(ys + h * PM * 128, &p.y_tile, c0 + 64 * h, row0, &ctl.full[s]);

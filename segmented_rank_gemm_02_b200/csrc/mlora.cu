@@ -42,8 +42,11 @@ struct mlora_pool {
     // TMA views of the B blocks for rank buckets 8, 16, 32, 64 (those <= r_bucket_max):
     // one load brings one 128-column chunk of one slot's B, all its rank groups
     CUtensorMap b_maps[4];
-    // the same views with 256-column boxes (one B chunk per tile of the fused base GEMM)
-    CUtensorMap b_maps256[4];
+    // the same blocks viewed as [slot][rank group][d_out / 32][32 columns x 8] (when
+    // d_out is a multiple of 32): one box {256, 4, R/8, 1} brings the same 128-column
+    // chunk in 512-byte rows instead of 16-byte ones
+    CUtensorMap b_maps_wide[4];
+    bool b_maps_wide_ok;
     bool b_maps_ok;
 };
 
@@ -132,7 +135,8 @@ mlora::TileParams base_params(const mlora_pool *pool, const mlora_segments *s)
     p.scales = s->scales;
     p.token_indices = s->token_indices;
     p.generations = s->generations;
-    for (int i = 0; i < 4; ++i) p.b_map[i] = pool->b_maps[i];
+    for (int i = 0; i < 4; ++i) p.b_map[i] = pool->b_maps_wide_ok ? pool->b_maps_wide[i] : pool->b_maps[i];
+    p.b_col_div = pool->b_maps_wide_ok ? 32 : 1;
     return p;
 }
 
@@ -179,6 +183,21 @@ bool encode_b_map(CUtensorMap *map, const mlora_pool *pool, int R, int cols)
     cuuint64_t dims[4] = {8, (cuuint64_t)pool->d_out, (cuuint64_t)groups, (cuuint64_t)pool->n_slots};
     cuuint64_t strides[3] = {16, (cuuint64_t)pool->d_out * 16, (cuuint64_t)pool->slot_stride * 2};
     cuuint32_t box[4] = {8, (cuuint32_t)cols, (cuuint32_t)(R / 8), 1};
+    cuuint32_t elem[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, pool->buf + pool->b_offset, dims, strides, box,
+               elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The wide view of the pool's B blocks (d_out a multiple of 32), box {256, 4, R/8, 1}.
+bool encode_b_map_wide(CUtensorMap *map, const mlora_pool *pool, int R)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (enc == nullptr || pool->d_out % 32 != 0) return false;
+    const int groups = pool->r_bucket_max / 8;
+    cuuint64_t dims[4] = {256, (cuuint64_t)pool->d_out / 32, (cuuint64_t)groups, (cuuint64_t)pool->n_slots};
+    cuuint64_t strides[3] = {512, (cuuint64_t)pool->d_out * 16, (cuuint64_t)pool->slot_stride * 2};
+    cuuint32_t box[4] = {256, (cuuint32_t)mlora::kExpandChunk / 32, (cuuint32_t)(R / 8), 1};
     cuuint32_t elem[4] = {1, 1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, pool->buf + pool->b_offset, dims, strides, box,
                elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -419,8 +438,10 @@ mlora_status mlora_pool_create(int32_t d_in, int32_t d_out, int32_t n_slots, int
         pool->b_maps_ok = tensor_map_encoder() != nullptr;
         for (int i = 0; i < 4 && pool->b_maps_ok; ++i)
             if ((8 << i) <= rb)
-                pool->b_maps_ok = encode_b_map(&pool->b_maps[i], pool, 8 << i, mlora::kExpandChunk) &&
-                                  encode_b_map(&pool->b_maps256[i], pool, 8 << i, mlora::kGemmCols);
+                pool->b_maps_ok = encode_b_map(&pool->b_maps[i], pool, 8 << i, mlora::kExpandChunk);
+        pool->b_maps_wide_ok = pool->b_maps_ok && pool->d_out % 32 == 0;
+        for (int i = 0; i < 4 && pool->b_maps_wide_ok; ++i)
+            if ((8 << i) <= rb) pool->b_maps_wide_ok = encode_b_map_wide(&pool->b_maps_wide[i], pool, 8 << i);
     }
     if (st != MLORA_OK) {
         cudaGetLastError();   // clear a sticky allocation error
@@ -638,7 +659,8 @@ mlora_status mlora_base_gemm_apply(mlora_pool *pool, const mlora_segments *segs,
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const int rk = std::max(16, pool->r_bucket_max);
     const int64_t n_mblk = (segs->n_rows + mlora::kGemmRows - 1) / mlora::kGemmRows;
-    const int64_t n_nblk = (pool->d_out + mlora::kGemmCols - 1) / mlora::kGemmCols;
+    const int gn = mlora::choose_gemm_cols((int)n_mblk, pool->d_out);
+    const int64_t n_nblk = (pool->d_out + gn - 1) / gn;
     // workspace: H (grouped order), the row map, the slot lists of the row blocks
     const size_t h_bytes = (size_t)round_up((int64_t)segs->n_tokens * rk * 4, 256);
     const size_t map_bytes = (size_t)round_up((int64_t)segs->n_rows * 16, 256);
@@ -667,10 +689,12 @@ mlora_status mlora_base_gemm_apply(mlora_pool *pool, const mlora_segments *segs,
         return MLORA_ERR_CUDA;
     // 3. Y = X W^T + s (H B^T) per tile
     mlora::GemmParams g{};
-    if (!encode_rows_map(&g.x_map, X, segs->n_rows, pool->d_in, ldx, mlora::kGemmRows) ||
-        !encode_rows_map(&g.w_map, W, pool->d_out, pool->d_in, ldw, mlora::kGemmCols))
+    // each CTA of a pair loads 128-row boxes of X and W
+    if (!encode_rows_map(&g.x_map, X, segs->n_rows, pool->d_in, ldx, mlora::kGemmRows / 2) ||
+        !encode_rows_map(&g.w_map, W, pool->d_out, pool->d_in, ldw, mlora::kGemmRows / 2))
         return MLORA_ERR_CUDA;
-    for (int i = 0; i < 4; ++i) g.b_map[i] = pool->b_maps256[i];
+    for (int i = 0; i < 4; ++i) g.b_map[i] = pool->b_maps_wide_ok ? pool->b_maps_wide[i] : pool->b_maps[i];
+    g.b_col_div = pool->b_maps_wide_ok ? 32 : 1;
     g.row_info = row_info;
     g.block_slots = block_slots;
     g.H = H;
@@ -683,7 +707,7 @@ mlora_status mlora_base_gemm_apply(mlora_pool *pool, const mlora_segments *segs,
     g.d_out = pool->d_out;
     g.n_mblk = (int32_t)n_mblk;
     g.n_nblk = (int32_t)n_nblk;
-    return mlora::launch_base_gemm(g, cs) == cudaSuccess ? MLORA_OK : MLORA_ERR_CUDA;
+    return mlora::launch_base_gemm(gn, g, cs) == cudaSuccess ? MLORA_OK : MLORA_ERR_CUDA;
 }
 
 mlora_status mlora_apply_multi(mlora_pool *const *pools, int32_t n_proj, const mlora_segments *segs,

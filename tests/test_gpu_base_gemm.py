@@ -71,6 +71,26 @@ def test_base_gemm_ragged_shapes_and_all_buckets(shuffle):
     free()
 
 
+@pytest.mark.parametrize("n_rows,d_out", [(9472, 512), (2048, 8448), (4096, 6000), (600, 4096)])
+def test_base_gemm_tile_widths(n_rows, d_out):
+    # shapes for which the host picks each tile width on a full B200 (256 columns for
+    # the first and last, 512 for the others: one with a last tile whose second half
+    # lies wholly past d_out, one with a ragged second half); rows sorted into runs,
+    # several slots per 256-row block
+    W = wl.random_case(26, n_rows, 256, d_out, 5, (16, 64), shuffle=False)
+    proj = W.projection(0)
+    Wb = W.base_weight(0)
+    st, Y = _run(W, proj, Wb)
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.concatenate([np.arange(0, n_rows, 97), rng.choice(n_rows, 64, replace=False),
+                                     [n_rows - 1]]))
+    ref, _ = oracle.base_gemm_apply(proj.X[rows], Wb, W.row_slot[rows], None, W.slot_rank, W.slot_alpha,
+                                    proj.A, proj.B)
+    _check(mlora.bf16_bits(Y)[rows], ref, f"{n_rows}x{d_out}")
+    del st
+    free()
+
+
 def test_base_gemm_without_segments_is_the_base_projection():
     W = wl.random_case(24, 130, 64, 264, 3, (16,))
     proj = W.projection(0)
