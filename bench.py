@@ -25,6 +25,10 @@ dependent launch lets the next step's kernels start early) the line reports the
 isolated step (one step after an L2 flush, nothing to overlap with) and the first
 step of the process.
 
+The default line also carries ``base_gemm``: the base projection fused with the LoRA
+branch (mlora_base_gemm_apply) against torch.matmul followed by mlora_apply, on the
+prefill workload (--base-gemm runs that leg alone).
+
 With --gpus N > 1 outside torchrun the script relaunches itself under
 torch.distributed.run with N ranks.  Each rank runs its own batch of the same shape
 (independent problems, no collective on the data path); value = all ranks' tokens /
@@ -177,9 +181,11 @@ def measured_peaks() -> dict:
         with open(path) as f:
             d = json.load(f)
         return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
                 "source": "measured"}
     except Exception:
-        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
 
 
 def kernel_source_hash() -> str:
@@ -577,6 +583,124 @@ def parity_only(cfg: int, device_index: int) -> dict:
     return {"workload": W.name, "parity": {"rows_checked": W.n_rows, "max_err_over_tolerance": worst}}
 
 
+def base_gemm_leg(args, device_index: int, cfg: int = 3) -> dict:
+    """The base projection fused with the LoRA branch (mlora_base_gemm_apply: one
+    shrink, then one tensor-core GEMM that adds s (X A^T) B^T into the accumulator of
+    X W^T) against the two-kernel path a caller would otherwise run (torch.matmul for
+    X W^T, then mlora_apply onto it), on the prefill workload.  Each arm is a CUDA
+    graph of K steps over rotating buffer sets larger than twice L2, timed R times."""
+    import torch
+    import segmented_rank_gemm_02_b200 as mlora
+    import workloads as wl
+
+    dev = torch.device("cuda", device_index)
+    W = wl.make(cfg)
+    proj = W.projection(0)
+    Wb = W.base_weight(0)
+    meta = mlora.build_segments(W.row_slot)
+    meta["ranks"] = np.array([0 if s < 0 else W.slot_rank[s] for s in meta["slots"]], np.int32)
+    X0 = mlora.as_bf16_tensor(proj.X, dev)
+    W0 = mlora.as_bf16_tensor(Wb, dev)
+    set_bytes = (W.n_rows * (proj.d_in + 2 * proj.d_out) + proj.d_out * proj.d_in) * 2
+    try:
+        l2 = int(torch.cuda.get_device_properties(dev).L2_cache_size)
+    except Exception:
+        l2 = L2_FALLBACK
+    n_sets = max(2, math.ceil(2 * l2 / set_bytes))
+    sets = []
+    for _ in range(n_sets):
+        pool = mlora.Pool(proj.d_in, proj.d_out, W.n_slots, W.r_max)
+        for s in sorted(proj.A):
+            pool.load_slot(s, int(W.slot_rank[s]), float(W.slot_alpha[s]), proj.A[s], proj.B[s])
+        sets.append({"pool": pool, "segs": mlora.DeviceSegments(meta, W.n_rows, dev), "X": X0.clone(),
+                     "W": W0.clone(), "Y": torch.empty((W.n_rows, proj.d_out), dtype=torch.bfloat16, device=dev)})
+    stream = torch.cuda.Stream(device=dev)
+
+    def fused(e):
+        mlora.base_gemm_apply(e["pool"], e["segs"], e["X"], e["W"], e["Y"], stream=stream)
+
+    def two_kernel(e):
+        torch.matmul(e["X"], e["W"].t(), out=e["Y"])
+        mlora.apply(e["pool"], e["segs"], e["X"], e["Y"], stream=stream)
+
+    def matmul(e):
+        torch.matmul(e["X"], e["W"].t(), out=e["Y"])
+
+    def time_arm(fn):
+        with torch.cuda.stream(stream):
+            for k in range(max(args.warmup, n_sets)):   # sizes every workspace before capture
+                fn(sets[k % n_sets])
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(graph, stream=stream):
+            for k in range(args.steps):
+                fn(sets[k % n_sets])
+        launches = graph_kernel_count(graph)
+        graph.instantiate()
+        with torch.cuda.stream(stream):
+            graph.replay()
+        stream.synchronize()
+        ms = []
+        for _ in range(args.repeats):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                a.record(stream)
+                graph.replay()
+                b.record(stream)
+            stream.synchronize()
+            ms.append(a.elapsed_time(b))
+        del graph
+        return Repeated(ms), launches
+
+    with ClockSampler(device_index) as clk:
+        t0 = time.perf_counter()
+        r_fused, n_fused = time_arm(fused)
+        r_two, n_two = time_arm(two_kernel)
+        r_mm, _ = time_arm(matmul)
+        t1 = time.perf_counter()
+    clocks = clk.summary(t0, t1)
+    # the two arms' outputs on the same inputs: both round once to bf16, the two-kernel
+    # arm twice (X W^T, then the sum), so they agree to about one bf16 step
+    e = sets[0]
+    fused(e)
+    Yf = e["Y"].float()
+    two_kernel(e)
+    Yt = e["Y"].float()
+    torch.cuda.synchronize()
+    agree = float(((Yf - Yt).abs() / (1e-2 * (1 + Yt.abs()))).max().item())
+    assert e["pool"].check() == 0
+    steps = args.steps
+    us = {name: r.median * 1e3 / steps for name, r in (("fused", r_fused), ("two_kernel", r_two),
+                                                          ("matmul", r_mm))}
+    adapter_rows = int((W.row_slot >= 0).sum())
+    base_flops = 2.0 * W.n_rows * proj.d_in * proj.d_out
+    lora_flops = 2.0 * adapter_rows * int(W.slot_rank.max()) * (proj.d_in + proj.d_out)
+    peaks = measured_peaks()
+    achieved = (base_flops + lora_flops) / (us["fused"] * 1e-6) / 1e12
+    for s in sets:
+        s["pool"].close()
+    del sets
+    torch.cuda.empty_cache()
+    return {
+        "workload": W.name, "call": "mlora_base_gemm_apply",
+        "shape": {"rows": W.n_rows, "d_in": proj.d_in, "d_out": proj.d_out, "adapter_rows": adapter_rows,
+                  "rank": int(W.slot_rank.max())},
+        "us_per_step": {"fused": us["fused"], "matmul_plus_apply": us["two_kernel"], "matmul_alone": us["matmul"]},
+        "spread_us": {"fused": r_fused.summary(steps / 1e3), "matmul_plus_apply": r_two.summary(steps / 1e3)},
+        "speedup_vs_matmul_plus_apply": us["two_kernel"] / us["fused"],
+        "delta_tokens_per_s": adapter_rows / (us["fused"] * 1e-6),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
+                     "peak_source": peaks["source"] + " (sustained bf16)",
+                     "flops_per_step": base_flops + lora_flops},
+        "gpu_launches_per_step": {"fused": n_fused / steps if n_fused else None,
+                                  "matmul_plus_apply": n_two / steps if n_two else None},
+        "agreement_with_two_kernel_over_tolerance": agree,
+        "l2": f"rotating {n_sets} buffer sets of {set_bytes / 2**20:.0f} MiB (> 2x L2)",
+        "clocks": clocks,
+    }
+
+
 def run_ours(args, rank: int, world: int, device_index: int):
     import torch
     torch.cuda.set_device(device_index)
@@ -615,6 +739,7 @@ def run_ours(args, rank: int, world: int, device_index: int):
                                        "kind": "oracle", "sample": sample, "seconds": el}
             per[str(cfg)] = e
         result["per_config"] = per
+        result["base_gemm"] = base_gemm_leg(args, device_index)
     return result
 
 
@@ -877,6 +1002,9 @@ def main(argv=None) -> int:
                          "(default); --no-fused: one mlora_apply per projection")
     ap.add_argument("--per-config", action=argparse.BooleanOptionalAction, default=None,
                     help="also measure the other workloads (default: with the default headline)")
+    ap.add_argument("--base-gemm", action="store_true",
+                    help="only the fused base GEMM + LoRA leg (mlora_base_gemm_apply against "
+                         "torch.matmul + mlora_apply) on the prefill workload (one GPU)")
     ap.add_argument("--slot-load", action="store_true",
                     help="measure adapter slot loads instead of the apply step (one GPU)")
     args = ap.parse_args(argv)
@@ -901,6 +1029,14 @@ def main(argv=None) -> int:
 
     if args.slot_load:
         print(json.dumps(run_slot_load(args)), flush=True)
+        return 0
+    if args.base_gemm:
+        import torch
+        torch.cuda.set_device(0)
+        leg = base_gemm_leg(args, 0)
+        print(json.dumps(dict({"metric": "fused base GEMM + LoRA delta vs torch.matmul + mlora_apply",
+                               "value": leg["us_per_step"]["fused"], "unit": "us per step",
+                               "higher_is_better": False}, **leg)), flush=True)
         return 0
 
     if args.impl == "reference":

@@ -530,6 +530,10 @@ __global__ void __launch_bounds__(GT, 1) base_gemm_kernel(const __grid_constant_
         // ---------------------------------------------------------------- LoRA operand
         const int r = tid - 6 * 32;               // row 0..127 of this CTA's half
         const uint32_t full_bar0 = leader_bar(&ctl.hop_full[0]), full_bar1 = leader_bar(&ctl.hop_full[1]);
+        // H comes from the shrink launched just before this kernel (which may still be
+        // running when launched with programmatic dependent launch); nothing else here
+        // reads what it writes
+        griddep_wait();
         uint32_t hc = 0;
         bool alive = true;
         for (int t = first; t < n_tiles && alive; t += n_clusters) {
@@ -606,7 +610,7 @@ cudaError_t launch_block_slots(const int4 *row_info, int n_rows, int32_t *block_
 namespace {
 
 template <int NSUB>
-cudaLaunchConfig_t gemm_config(unsigned pairs, cudaStream_t stream, cudaLaunchAttribute *attr)
+cudaLaunchConfig_t gemm_config(unsigned pairs, cudaStream_t stream, cudaLaunchAttribute *attr, bool pdl = false)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs, 1, 1);
@@ -617,8 +621,10 @@ cudaLaunchConfig_t gemm_config(unsigned pairs, cudaStream_t stream, cudaLaunchAt
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 2 : 1;
     return cfg;
 }
 
@@ -635,7 +641,7 @@ cudaError_t gemm_active_pairs(int &active)
         active = cached[dev];
         return cudaSuccess;
     }
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = gemm_config<NSUB>(1, nullptr, attr);
     cudaError_t e = cudaOccupancyMaxActiveClusters(&active, base_gemm_kernel<NSUB>, &cfg);
     if (e != cudaSuccess) return e;
@@ -645,7 +651,7 @@ cudaError_t gemm_active_pairs(int &active)
 }
 
 template <int NSUB>
-cudaError_t launch_units(const GemmParams &p, cudaStream_t stream)
+cudaError_t launch_units(const GemmParams &p, cudaStream_t stream, bool pdl)
 {
     const int64_t tiles = (int64_t)p.n_mblk * p.n_nblk;
     if (tiles <= 0) return cudaSuccess;
@@ -653,8 +659,8 @@ cudaError_t launch_units(const GemmParams &p, cudaStream_t stream)
     cudaError_t e = gemm_active_pairs<NSUB>(active);
     if (e != cudaSuccess) return e;
     const unsigned pairs = (unsigned)std::min<int64_t>(tiles, active);   // persistent
-    cudaLaunchAttribute attr[1];
-    cudaLaunchConfig_t cfg = gemm_config<NSUB>(pairs, stream, attr);
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = gemm_config<NSUB>(pairs, stream, attr, pdl);
     return cudaLaunchKernelEx(&cfg, base_gemm_kernel<NSUB>, p);
 }
 
@@ -683,11 +689,11 @@ int choose_gemm_cols(int n_mblk, int d_out)
     return c2 < c1 ? 2 * UN : UN;
 }
 
-cudaError_t launch_base_gemm(int gn, const GemmParams &p, cudaStream_t stream)
+cudaError_t launch_base_gemm(int gn, const GemmParams &p, cudaStream_t stream, bool pdl)
 {
     switch (gn) {
-    case UN: return launch_units<1>(p, stream);
-    case 2 * UN: return launch_units<2>(p, stream);
+    case UN: return launch_units<1>(p, stream, pdl);
+    case 2 * UN: return launch_units<2>(p, stream, pdl);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -206,8 +206,9 @@ cudaError_t launch_block_slots(const int4 *row_info, int n_rows, int32_t *block_
 // Tile width (256 or 512 columns of Y) for n_mblk 256-row blocks and d_out columns.
 int choose_gemm_cols(int n_mblk, int d_out);
 // Persistent GEMM over all (256-row, gn-column) tiles, one pair of CTAs per two SMs;
-// p.n_nblk = ceil(d_out / gn).
-cudaError_t launch_base_gemm(int gn, const GemmParams &p, cudaStream_t stream);
+// p.n_nblk = ceil(d_out / gn).  With `pdl` it is launched with programmatic dependent
+// launch after the kernel before it, whose results (H) it reads only after waiting.
+cudaError_t launch_base_gemm(int gn, const GemmParams &p, cudaStream_t stream, bool pdl);
 cudaError_t prepare_base_gemm();
 
 }  // namespace mlora

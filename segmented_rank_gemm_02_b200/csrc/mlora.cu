@@ -673,20 +673,26 @@ mlora_status mlora_base_gemm_apply(mlora_pool *pool, const mlora_segments *segs,
     int4 *row_info = reinterpret_cast<int4 *>(ws + h_bytes);
     int32_t *block_slots = reinterpret_cast<int32_t *>(ws + h_bytes + map_bytes);
 
-    // 1. H = X A^T for every valid segment (decode-shaped and long-segment kernels)
+    // 1. each row's grouped position, slot, scale and rank; each row block's slots
     mlora::TileParams p = base_params(pool, segs);
     p.X = static_cast<const __nv_bfloat16 *>(X);
     p.ldx = ldx;
     p.H = H;
     p.ldh = rk;
-    if (segs->n_segments > 0 && segs->n_tokens > 0) {
-        st = launch(pool, segs, mlora::MODE_SHRINK, p, stream);
-        if (st != MLORA_OK) return st;
-    }
-    // 2. each row's grouped position, slot, scale and rank; each row block's slots
     if (mlora::launch_row_map(p, row_info, cs) != cudaSuccess ||
         mlora::launch_block_slots(row_info, segs->n_rows, block_slots, cs) != cudaSuccess)
         return MLORA_ERR_CUDA;
+    // 2. H = X A^T for every valid segment (decode-shaped and long-segment kernels)
+    const bool shrink = segs->n_segments > 0 && segs->n_tokens > 0;
+    if (shrink) {
+        st = launch(pool, segs, mlora::MODE_SHRINK, p, stream);
+        if (st != MLORA_OK) return st;
+    }
+    // The GEMM reads H only in its LoRA steps, after griddepcontrol.wait, so it may
+    // start while the long-segment shrink finishes (programmatic dependent launch).
+    // Only then: that shrink follows a plainly launched kernel, so everything before it
+    // (the row map, X) is complete when the GEMM starts.
+    const bool pdl = shrink && long_path(pool, segs);
     // 3. Y = X W^T + s (H B^T) per tile
     mlora::GemmParams g{};
     // each CTA of a pair loads 128-row boxes of X and W
@@ -707,7 +713,7 @@ mlora_status mlora_base_gemm_apply(mlora_pool *pool, const mlora_segments *segs,
     g.d_out = pool->d_out;
     g.n_mblk = (int32_t)n_mblk;
     g.n_nblk = (int32_t)n_nblk;
-    return mlora::launch_base_gemm(gn, g, cs) == cudaSuccess ? MLORA_OK : MLORA_ERR_CUDA;
+    return mlora::launch_base_gemm(gn, g, cs, pdl) == cudaSuccess ? MLORA_OK : MLORA_ERR_CUDA;
 }
 
 mlora_status mlora_apply_multi(mlora_pool *const *pools, int32_t n_proj, const mlora_segments *segs,
