@@ -125,6 +125,7 @@ struct ExpandOps<R, 2> {
 
 struct SharedCtl {
     uint64_t hbar[2];   // partial H tiles of the cluster landed (one per tile parity)
+    int fail;           // a partial-H wait ran out: no later tile of this launch is trusted
     int scan[kMaxWarps];
     int rows[TM];       // original row of each tile position, -1 = absent or invalid
     int tile[5];        // segment, first position, end position, slot, rank from metadata
@@ -650,13 +651,19 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
             for (uint32_t c = 0; c < csize; ++c)
                 st_async_f32x4(map_to_rank(slot_s + 16u * e4, c), sum, map_to_rank(bar_s, c));
         }
-        // the cluster's partials, summed in CTA order
+        // the cluster's partials, summed in CTA order.  After a wait has run out, the
+        // barriers' phases no longer match the tiles (late bytes may complete a later
+        // phase), so no later tile of this launch writes anything either (ctl.fail).
         const bool landed = mbar_wait_bounded(bar, (nt >> 1) & 1u, 1000000000ull);
-        if (!landed && tid == 0) report(v, kFlagTimeout);
+        if (!landed) {
+            ctl.fail = 1;
+            report(v, kFlagTimeout);
+        }
         for (int e = tid; e < TM * R; e += kThreads) {
             const int i = e / R, j = e % R;
             if (MODE == MODE_SHRINK &&
-                ((uint32_t)i % csize != crank || i >= tl.nvalid || j >= rank || ctl.rows[i] < 0 || !landed))
+                ((uint32_t)i % csize != crank || i >= tl.nvalid || j >= rank || ctl.rows[i] < 0 || !landed ||
+                 ctl.fail))
                 continue;
             float v[kMaxCluster];
 #pragma unroll
@@ -701,7 +708,7 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
                 al[s][q] = pack_bf16x2(l0, l1);
             }
         }
-        const bool store = ok && row_ok && h_ok;
+        const bool store = ok && row_ok && h_ok && (MODE == MODE_EXPAND || ctl.fail == 0);
         for (int i = 0; i < ng; i += 2) {
             mma_expand_store<R, YT>(e0, ah, al, scale, yrow, store, sl, warp + i * kWarps, t);
             if (i + 2 < ng) {
@@ -750,6 +757,7 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
             mbar_init(&ctl.hbar[0], 1);
             mbar_init(&ctl.hbar[1], 1);
             fence_mbar_init();
+            ctl.fail = 0;
         }
         cluster_arrive_release();
         cluster_wait_acquire();
