@@ -245,9 +245,9 @@ mlora_status mlora_apply_ex(mlora_pool *pool, const mlora_segments *segs, const 
                             float x_scale, int64_t ldx, void *Y, int32_t y_dtype, int64_t ldy, void *stream);
 
 /*
- * The base projection and the LoRA delta in one pass (page "LoRA/QLoRA multi-tenant
- * serving", section 3.3 on fusing W0 x + B(A x) into one kernel, and its paragraph on
- * cuBLASLt epilogue fusion after section 5.3):
+ * The base projection and the LoRA delta in one pass (page "Multi-LoRA serving",
+ * ybb.press ai-applications, section 3.3 on fusing W0 x + B(A x) into one kernel, and
+ * its paragraph on cuBLASLt epilogue fusion after section 5.3):
  *
  *   Y[t, :] = bf16(X[t, :] W^T + s_g (X[t, :] A_a^T) B_a^T)   rows t of adapter segments
  *   Y[t, :] = bf16(X[t, :] W^T)                                every other row

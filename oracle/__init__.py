@@ -239,8 +239,8 @@ def apply_rows_xf64(X: np.ndarray, Y0: np.ndarray, row_slot, row_scale, slot_ran
 def base_gemm_apply(X: np.ndarray, W: np.ndarray, row_slot, row_scale, slot_rank, slot_alpha,
                     A: Dict[int, np.ndarray], B: Dict[int, np.ndarray],
                     n_threads: int = 0) -> Tuple[np.ndarray, int]:
-    """The base projection and the LoRA branch together (page "LoRA/QLoRA multi-tenant
-    serving", section 3.3, W0 x + B(A x) in one kernel; page "Multi-LoRA Serving:
+    """The base projection and the LoRA branch together (page "Multi-LoRA serving",
+    ybb.press ai-applications, section 3.3, W0 x + B(A x) in one kernel; page "Multi-LoRA Serving:
     adapter batching", section "LoRA on one Linear layer", Y = X W^T + s (X A^T) B^T):
     Y[t] = X[t] W^T + s_a (X[t] A_a^T) B_a^T for rows of adapter a, X[t] W^T for base
     rows, in fp64.  ``X`` [n_rows, d_in] and ``W`` [d_out, d_in] (the nn.Linear

@@ -1,9 +1,9 @@
 // base_gemm.cu -- the base projection and the LoRA delta in one tensor-core pass.
 //
 // Y = X W^T + s_a (X A_a^T) B_a^T for the rows of adapter segments and Y = X W^T for
-// every other row (page "LoRA/QLoRA multi-tenant serving", section 3.3 on fusing
-// W0 x + B(A x) into one kernel, and the paragraph on cuBLASLt epilogue fusion after
-// section 5.3: the low-rank product goes into the base GEMM's accumulator, so Y is
+// every other row (page "Multi-LoRA serving", ybb.press ai-applications, section 3.3
+// on fusing W0 x + B(A x) into one kernel, and its paragraph on cuBLASLt epilogue
+// fusion after section 5.3: the low-rank product goes into the base GEMM's accumulator, so Y is
 // written once, in bf16, and never read).
 //
 // Order of work.  The shrink H = X A_a^T is the library's segmented shrink (the

@@ -1,8 +1,8 @@
 """The base projection and the LoRA delta in one pass (mlora_base_gemm_apply), against
 the oracle.
 
-Page "LoRA/QLoRA multi-tenant serving", section 3.3 (W0 x + B(A x) fused into one
-kernel): Y = X W^T + s (X A^T) B^T for adapter rows and X W^T for every other row,
+Page "Multi-LoRA serving" (ybb.press ai-applications), section 3.3 (W0 x + B(A x)
+fused into one kernel): Y = X W^T + s (X A^T) B^T for adapter rows and X W^T for every other row,
 accumulated in fp32 and rounded to bf16 once.  The oracle is the fp64 per-row entry
 with Y0 = X W^T computed in fp64 from the exact bf16 values (oracle.base_gemm_apply).
 Every element must satisfy |gpu - oracle| <= 1e-2 (1 + |oracle|), base rows included;

@@ -467,8 +467,8 @@ MUTANT_CHECKS = PIN_CHECKS + [test_fp64_activation_entry_equals_bf16_entry,
 
 
 # ---------------------------------------------------------------------------
-# the base projection and the LoRA branch together (page "LoRA/QLoRA multi-tenant
-# serving", section 3.3: W0 x + B(A x) in one kernel)
+# the base projection and the LoRA branch together (page "Multi-LoRA serving",
+# ybb.press ai-applications, section 3.3: W0 x + B(A x) in one kernel)
 # ---------------------------------------------------------------------------
 
 def _base_problem(seed, n_rows, d_in, d_out, ranks, base_rows):
