@@ -11,7 +11,8 @@ namespace mlora {
 enum TileMode : int { MODE_APPLY = 0, MODE_SHRINK = 1, MODE_EXPAND = 2 };
 
 // Grouped positions in one work tile of the segmented (decode-family) kernel: the
-// top half of one m16 MMA tile.
+// top half of one m16 MMA tile (batches of long decode segments at rank <= 16 use
+// 16-row tiles, the whole m16 tile; see lora_decode.cu).
 constexpr int kTileRows = 8;
 
 // Device status bits (same values as the MLORA_FLAG_* macros of the public header).

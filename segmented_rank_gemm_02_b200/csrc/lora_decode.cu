@@ -7,10 +7,11 @@
 //     H[p, :] = X[t, :] A_a^T                       (shrink, rank r)
 //     Y[t, :] = bf16(Y[t, :] + s_g H[p, :] B_a^T)   (expand + scatter)
 //
-// Work decomposition.  A work tile is (segment, up to 8 consecutive grouped
-// positions).  A thread-block cluster of C CTAs owns a tile: CTA c covers its
+// Work decomposition.  A work tile is (segment, up to 16 consecutive grouped
+// positions: the rows of one m16 MMA tile, so an adapter's slices are read once per 16
+// rows of its segment).  A thread-block cluster of C CTAs owns a tile: CTA c covers its
 // slice of d_in in the shrink (split-K) and its slice of d_out in the expand.
-// Each CTA pushes its partial H tile (8 x R fp32) into every CTA of the cluster
+// Each CTA pushes its partial H tile (16 x R fp32) into every CTA of the cluster
 // with st.async (distributed shared memory, completion counted on the receiver's
 // mbarrier), and each sums the C partials in CTA order, so in the fused mode H
 // never leaves the chip.  The grid holds as many
@@ -20,14 +21,14 @@
 // copies to pay off, so every thread loads its mma.sync operands straight from
 // global memory with 128-bit loads:
 //   * shrink: per 32-column block of d_in, thread (g, t) of a warp loads 8
-//     consecutive bf16 of X row g and of adapter row n at columns 8t..8t+7; the
-//     two k16 mma steps of the block consume them in that order.  The sum over k
+//     consecutive bf16 of X rows g and g + 8 and of adapter row n at columns
+//     8t..8t+7; the two k16 mma steps of the block consume them in that order.  The sum over k
 //     does not care which columns share a step, as long as X and A agree.
 //   * expand: four n8 mma tiles cover 32 output columns; the B row a lane feeds
 //     is chosen so that thread (g, t) ends up owning columns 8t..8t+7 of row g,
-//     so Y0 is read and Y written as one 16-byte vector per thread and row.  The
-//     rank index inside each k16 step is permuted the same way for H and B.
-// The rows 8..15 of every m16 tile are zero (a tile has 8 rows).
+//     (and row g + 8), so Y0 is read and Y written as one 16-byte vector per thread
+//     and row.  The rank index inside each k16 step is permuted the same way for H
+//     and B.
 //
 // Rank buckets.  A kernel is compiled for the pool's largest bucket RMAX and runs
 // every tile with code specialised for its own slot's bucket R <= RMAX, so a
@@ -70,10 +71,16 @@ namespace mlora {
 namespace {
 
 constexpr int kMaxWarps = 8;     // CTAs of 256 threads, or 128 (see launch_rmax)
-constexpr int TM = kTileRows;   // 8
+// Grouped positions per work tile: 8 (rows g of the m16 MMA tile; rows 8..15 zero) or
+// 16 (rows g and g + 8).  16-row tiles read each adapter slice once per 16 rows of a
+// segment instead of 8 but need more registers and shared memory per CTA, so they are
+// used only where segments are long and the rank small (block70b, 2048 rows over 128
+// rank-16 adapters: 391.7 -> 361.9 us per step; with 8 or fewer rows per segment, or
+// rank 64, they measured much slower).
+constexpr int kMaxTM = 16;
 constexpr int kMaxCluster = 8;
 
-template <int RMAX, int NT>
+template <int RMAX, int NT, int TM = kTileRows>
 struct DecodeCfg {
     static constexpr int kWarps = NT / 32;
     static constexpr int WPART_FLOATS = kWarps * TM * RMAX;   // per-warp partial H
@@ -82,7 +89,7 @@ struct DecodeCfg {
     static constexpr int HPITCH = RMAX + 4;
     static constexpr int HFULL_FLOATS = TM * HPITCH;          // full H (after the cluster sum)
     static constexpr int SMEM = 4 * (WPART_FLOATS + RECV_FLOATS + HFULL_FLOATS);
-    static constexpr int MIN_BLOCKS = (RMAX <= 16 ? 4 : 2) * (256 / NT);
+    static constexpr int MIN_BLOCKS = (RMAX <= 16 ? (TM == 16 ? 3 : 4) : 2) * (256 / NT);
 };
 
 // Per-R register operands: one k32 block of the shrink, one 32-column group of the
@@ -99,7 +106,7 @@ struct RankCfg {
 
 template <int R>
 struct ShrinkOps {
-    uint4 x;                    // X row g, columns 8t..8t+7 of the block
+    uint4 x, x8;                // X rows g and g + 8, columns 8t..8t+7 of the block
     uint4 a[RankCfg<R>::NT];    // adapter rows n*8+g, same columns
 };
 
@@ -114,20 +121,20 @@ __host__ __device__ constexpr int y_bytes(int dt) { return dt_y(dt) == 2 ? 4 : 2
 template <int R, int YT = 0>
 struct ExpandOps {
     uint2 b[4][RankCfg<R>::KS];  // B rows of the four n8 tiles, this lane's ranks
-    uint4 y;                     // Y0 row g, columns 8t..8t+7 of the group (bf16 or fp16)
+    uint4 y[2];                  // Y0 rows g, g + 8, columns 8t..8t+7 of the group (bf16 or fp16)
 };
 
 template <int R>
 struct ExpandOps<R, 2> {
     uint2 b[4][RankCfg<R>::KS];
-    uint4 y, y2;                 // fp32 Y0: columns 8t..8t+3, 8t+4..8t+7
+    uint4 y[2], y2[2];           // fp32 Y0 rows g, g + 8: columns 8t..8t+3, 8t+4..8t+7
 };
 
 struct SharedCtl {
     uint64_t hbar[2];   // partial H tiles of the cluster landed (one per tile parity)
     int fail;           // a partial-H wait ran out: no later tile of this launch is trusted
     int scan[kMaxWarps];
-    int rows[TM];       // original row of each tile position, -1 = absent or invalid
+    int rows[kMaxTM];   // original row of each tile position, -1 = absent or invalid
     int tile[5];        // segment, first position, end position, slot, rank from metadata
     int stale;          // the batch was built for an earlier generation of the slot
     float seg_scale;
@@ -196,7 +203,7 @@ __device__ __forceinline__ void prefetch_slices_one(const TileParams &p, const P
 // slices of that tile's adapter into L2, so that they travel while the current tile
 // runs.  Batches of several waves skip it: there the prefetches thrashed L2
 // (measured 11% slower on 2048 decode rows of 8192-wide projections).
-template <bool SPEC, int NT, int MODE, int RMAX>
+template <bool SPEC, int NT, int MODE, int RMAX, int TM>
 __device__ int scan_tiles(const TileParams &p, const uint32_t *slot_gen, int want, int want2,
                           const ProjView &v2, SharedCtl &ctl, bool reporter)
 {
@@ -305,29 +312,42 @@ template <int YT>
 using YElem =
     typename std::conditional<YT == 2, float, typename std::conditional<YT == 1, __half, __nv_bfloat16>::type>::type;
 
-template <int R, int XT = 0>
-__device__ __forceinline__ void load_x(ShrinkOps<R> &o, XElem<XT> *xrow, bool row_ok, const Slices &sl, int blk,
-                                       int t)
+template <int XT>
+__device__ __forceinline__ uint4 load_x_row(XElem<XT> *xrow, bool in, int k)
 {
-    const int k = sl.k_begin + blk * 32 + 8 * t;
     if constexpr (XT == 0) {
-        o.x = (row_ok && blk < sl.nblk && k < sl.k_end) ? ldg_nc(xrow + k) : make_uint4(0, 0, 0, 0);
+        return in ? ldg_nc(xrow + k) : make_uint4(0, 0, 0, 0);
     } else {
         // eight e4m3 codes, widened to bf16 (the per-tensor scale is applied to H)
-        const bool in = row_ok && blk < sl.nblk && k < sl.k_end;
         const uint2 c = in ? __ldg(reinterpret_cast<const uint2 *>(xrow + k)) : make_uint2(0u, 0u);
-        o.x = make_uint4(e4m3x2_to_bf16x2(c.x), e4m3x2_to_bf16x2(c.x >> 16), e4m3x2_to_bf16x2(c.y),
-                         e4m3x2_to_bf16x2(c.y >> 16));
+        return make_uint4(e4m3x2_to_bf16x2(c.x), e4m3x2_to_bf16x2(c.x >> 16), e4m3x2_to_bf16x2(c.y),
+                          e4m3x2_to_bf16x2(c.y >> 16));
     }
 }
 
-template <int R>
+// X rows g (xrow) and g + 8 (xrow8) of the tile, this thread's 8 columns of the block.
+template <int R, int XT, int TM>
+__device__ __forceinline__ void load_x(ShrinkOps<R> &o, XElem<XT> *xrow, bool row_ok, XElem<XT> *xrow8,
+                                       bool row_ok8, const Slices &sl, int blk, int t)
+{
+    const int k = sl.k_begin + blk * 32 + 8 * t;
+    const bool kin = blk < sl.nblk && k < sl.k_end;
+    o.x = load_x_row<XT>(xrow, row_ok && kin, k);
+    if constexpr (TM == 16) o.x8 = load_x_row<XT>(xrow8, row_ok8 && kin, k);
+}
+
+template <int R, int TM>
 __device__ __forceinline__ void mma_shrink(float (&acc)[RankCfg<R>::NT][4], const ShrinkOps<R> &o)
 {
 #pragma unroll
     for (int n = 0; n < RankCfg<R>::NT; ++n) {
-        mma_16816(acc[n], o.x.x, 0u, o.x.y, 0u, o.a[n].x, o.a[n].y);
-        mma_16816(acc[n], o.x.z, 0u, o.x.w, 0u, o.a[n].z, o.a[n].w);
+        if constexpr (TM == 16) {
+            mma_16816(acc[n], o.x.x, o.x8.x, o.x.y, o.x8.y, o.a[n].x, o.a[n].y);
+            mma_16816(acc[n], o.x.z, o.x8.z, o.x.w, o.x8.w, o.a[n].z, o.a[n].w);
+        } else {   // rows g + 8 of an 8-row tile are zero
+            mma_16816(acc[n], o.x.x, 0u, o.x.y, 0u, o.a[n].x, o.a[n].y);
+            mma_16816(acc[n], o.x.z, 0u, o.x.w, 0u, o.a[n].z, o.a[n].w);
+        }
     }
 }
 
@@ -357,28 +377,36 @@ __device__ __forceinline__ void load_b(ExpandOps<R, YT> &o, const __nv_bfloat16 
         }
 }
 
-template <int R, int YT>
-__device__ __forceinline__ void load_y(ExpandOps<R, YT> &o, const YElem<YT> *yrow, bool row_ok, const Slices &sl,
-                                       int grp, int t)
+// Y0 rows g (yrow) and g + 8 (yrow8, 16-row tiles), this thread's 8 columns of the group.
+template <int R, int YT, int TM>
+__device__ __forceinline__ void load_y(ExpandOps<R, YT> &o, const YElem<YT> *yrow, bool row_ok,
+                                       const YElem<YT> *yrow8, bool row_ok8, const Slices &sl, int grp, int t)
 {
     const int c = sl.n_begin + grp * 32 + 8 * t;
-    if constexpr (YT == 2) {   // eight fp32
-        const bool in = row_ok && grp < sl.ngrp && c < sl.n_end;
-        const uint4 *src = reinterpret_cast<const uint4 *>(yrow + c);
-        o.y = in ? src[0] : make_uint4(0, 0, 0, 0);
-        o.y2 = in ? src[1] : make_uint4(0, 0, 0, 0);
-    } else {                   // eight bf16 or fp16
-        o.y = (row_ok && grp < sl.ngrp && c < sl.n_end) ? *reinterpret_cast<const uint4 *>(yrow + c)
-                                                         : make_uint4(0, 0, 0, 0);
+    const bool cin = grp < sl.ngrp && c < sl.n_end;
+#pragma unroll
+    for (int h = 0; h < TM / 8; ++h) {
+        const YElem<YT> *row = h ? yrow8 : yrow;
+        const bool in = cin && (h ? row_ok8 : row_ok);
+        if constexpr (YT == 2) {   // eight fp32
+            const uint4 *src = reinterpret_cast<const uint4 *>(row + c);
+            o.y[h] = in ? src[0] : make_uint4(0, 0, 0, 0);
+            o.y2[h] = in ? src[1] : make_uint4(0, 0, 0, 0);
+        } else {                   // eight bf16 or fp16
+            o.y[h] = in ? *reinterpret_cast<const uint4 *>(row + c) : make_uint4(0, 0, 0, 0);
+        }
     }
 }
 
-// y = y0 + s (H B^T), rounded once to Y's type, for one group; thread (g, t) stores row
-// g, columns 8t..8t+7.
-template <int R, int YT>
-__device__ __forceinline__ void mma_expand_store(const ExpandOps<R, YT> &o, const uint32_t (&ah)[RankCfg<R>::KS][2],
-                                                 const uint32_t (&al)[RankCfg<R>::KS][2], float scale, YElem<YT> *yrow,
-                                                 bool store, const Slices &sl, int grp, int t)
+// y = y0 + s (H B^T), rounded once to Y's type, for one group; thread (g, t) stores rows
+// g and g + 8, columns 8t..8t+7.  ah / al: H rows g and g + 8 ([.][0..1] row g, [.][2..3]
+// row g + 8, as the m16 A fragment wants them).
+template <int R, int YT, int TM>
+__device__ __forceinline__ void mma_expand_store(const ExpandOps<R, YT> &o,
+                                                 const uint32_t (&ah)[RankCfg<R>::KS][TM / 4],
+                                                 const uint32_t (&al)[RankCfg<R>::KS][TM / 4], float scale, YElem<YT> *yrow,
+                                                 bool store, YElem<YT> *yrow8, bool store8, const Slices &sl, int grp,
+                                                 int t)
 {
     float d[4][4];
 #pragma unroll
@@ -386,44 +414,60 @@ __device__ __forceinline__ void mma_expand_store(const ExpandOps<R, YT> &o, cons
         d[i][0] = d[i][1] = d[i][2] = d[i][3] = 0.f;
 #pragma unroll
         for (int s = 0; s < RankCfg<R>::KS; ++s) {
-            if constexpr (R == 8) {
-                mma_1688(d[i], ah[0][0], 0u, o.b[i][0].x);
-                mma_1688(d[i], al[0][0], 0u, o.b[i][0].x);
-            } else {
-                mma_16816(d[i], ah[s][0], 0u, ah[s][1], 0u, o.b[i][s].x, o.b[i][s].y);
-                mma_16816(d[i], al[s][0], 0u, al[s][1], 0u, o.b[i][s].x, o.b[i][s].y);
+            if constexpr (TM == 16) {
+                if constexpr (R == 8) {
+                    mma_1688(d[i], ah[0][0], ah[0][2], o.b[i][0].x);
+                    mma_1688(d[i], al[0][0], al[0][2], o.b[i][0].x);
+                } else {
+                    mma_16816(d[i], ah[s][0], ah[s][2], ah[s][1], ah[s][3], o.b[i][s].x, o.b[i][s].y);
+                    mma_16816(d[i], al[s][0], al[s][2], al[s][1], al[s][3], o.b[i][s].x, o.b[i][s].y);
+                }
+            } else {   // rows g + 8 of an 8-row tile are zero
+                if constexpr (R == 8) {
+                    mma_1688(d[i], ah[0][0], 0u, o.b[i][0].x);
+                    mma_1688(d[i], al[0][0], 0u, o.b[i][0].x);
+                } else {
+                    mma_16816(d[i], ah[s][0], 0u, ah[s][1], 0u, o.b[i][s].x, o.b[i][s].y);
+                    mma_16816(d[i], al[s][0], 0u, al[s][1], 0u, o.b[i][s].x, o.b[i][s].y);
+                }
             }
         }
     }
     const int c = sl.n_begin + grp * 32 + 8 * t;
-    if (!store || grp >= sl.ngrp || c >= sl.n_end) return;
-    if constexpr (YT == 2) {
-        const float4 a = *reinterpret_cast<const float4 *>(&o.y), b = *reinterpret_cast<const float4 *>(&o.y2);
-        float4 *dst = reinterpret_cast<float4 *>(yrow + c);
-        dst[0] = make_float4(fmaf(scale, d[0][0], a.x), fmaf(scale, d[0][1], a.y), fmaf(scale, d[1][0], a.z),
-                             fmaf(scale, d[1][1], a.w));
-        dst[1] = make_float4(fmaf(scale, d[2][0], b.x), fmaf(scale, d[2][1], b.y), fmaf(scale, d[3][0], b.z),
-                             fmaf(scale, d[3][1], b.w));
-    } else {
-        uint4 out;
-        uint32_t *w = reinterpret_cast<uint32_t *>(&out);
-        if constexpr (YT == 0) {
-            const __nv_bfloat162 *y0 = reinterpret_cast<const __nv_bfloat162 *>(&o.y);
+    if (grp >= sl.ngrp || c >= sl.n_end) return;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 f = __bfloat1622float2(y0[i]);
-                w[i] = pack_bf16x2(fmaf(scale, d[i][0], f.x), fmaf(scale, d[i][1], f.y));
-            }
+    for (int h = 0; h < TM / 8; ++h) {
+        if (!(h ? store8 : store)) continue;
+        YElem<YT> *row = h ? yrow8 : yrow;
+        if constexpr (YT == 2) {
+            const float4 a = *reinterpret_cast<const float4 *>(&o.y[h]);
+            const float4 b = *reinterpret_cast<const float4 *>(&o.y2[h]);
+            float4 *dst = reinterpret_cast<float4 *>(row + c);
+            dst[0] = make_float4(fmaf(scale, d[0][2 * h], a.x), fmaf(scale, d[0][2 * h + 1], a.y),
+                                 fmaf(scale, d[1][2 * h], a.z), fmaf(scale, d[1][2 * h + 1], a.w));
+            dst[1] = make_float4(fmaf(scale, d[2][2 * h], b.x), fmaf(scale, d[2][2 * h + 1], b.y),
+                                 fmaf(scale, d[3][2 * h], b.z), fmaf(scale, d[3][2 * h + 1], b.w));
         } else {
-            const __half2 *y0 = reinterpret_cast<const __half2 *>(&o.y);
+            uint4 out;
+            uint32_t *w = reinterpret_cast<uint32_t *>(&out);
+            if constexpr (YT == 0) {
+                const __nv_bfloat162 *y0 = reinterpret_cast<const __nv_bfloat162 *>(&o.y[h]);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 f = __half22float2(y0[i]);
-                const __half2 hv = __floats2half2_rn(fmaf(scale, d[i][0], f.x), fmaf(scale, d[i][1], f.y));
-                w[i] = *reinterpret_cast<const uint32_t *>(&hv);
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __bfloat1622float2(y0[i]);
+                    w[i] = pack_bf16x2(fmaf(scale, d[i][2 * h], f.x), fmaf(scale, d[i][2 * h + 1], f.y));
+                }
+            } else {
+                const __half2 *y0 = reinterpret_cast<const __half2 *>(&o.y[h]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __half22float2(y0[i]);
+                    const __half2 hv = __floats2half2_rn(fmaf(scale, d[i][2 * h], f.x), fmaf(scale, d[i][2 * h + 1], f.y));
+                    w[i] = *reinterpret_cast<const uint32_t *>(&hv);
+                }
             }
+            *reinterpret_cast<uint4 *>(row + c) = out;
         }
-        *reinterpret_cast<uint4 *>(yrow + c) = out;
     }
 }
 
@@ -468,11 +512,11 @@ __device__ void prefetch_slices(const TileParams &p, const ProjView &v, int slot
     }
 }
 
-template <int RMAX, int MODE, int NT, int DT>
+template <int RMAX, int MODE, int NT, int DT, int TM>
 __device__ void prefetch_first_tile(const TileParams &p, const ProjView &v, int want, SharedCtl &ctl,
                                     uint32_t crank)
 {
-    if (want >= scan_tiles<true, NT, MODE, RMAX>(p, v.slot_gen, want, -1, v, ctl, false)) return;
+    if (want >= scan_tiles<true, NT, MODE, RMAX, TM>(p, v.slot_gen, want, -1, v, ctl, false)) return;
     const int tid = threadIdx.x;
     const int slot = ctl.tile[3];
     if (slot < 0 || slot >= p.n_slots) return;
@@ -511,14 +555,14 @@ __device__ void prefetch_first_tile(const TileParams &p, const ProjView &v, int 
     }
 }
 
-template <int RMAX, int MODE, int R, int NT, int DT>
+template <int RMAX, int MODE, int R, int NT, int DT, int TM>
 __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl, int r_meta,
                          float seg_scale, SharedCtl &ctl, float *smem_f, uint32_t crank,
                          uint32_t csize, uint32_t nt)
 {
     constexpr int kThreads = NT, kWarps = NT / 32;
     using RC = RankCfg<R>;
-    using DC = DecodeCfg<RMAX, NT>;
+    using DC = DecodeCfg<RMAX, NT, TM>;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
     float *wpart = smem_f;
@@ -539,8 +583,10 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
     const int ng = sl.ngrp > warp ? (sl.ngrp - warp + kWarps - 1) / kWarps : 0;
 
     // ---- requests that need only the segment's slot
-    int row_g = -1;
+    int row_g = -1, row_g8 = -1;   // original rows of tile positions g and g + 8
     if (g < tl.nvalid) row_g = p.token_indices ? __ldg(p.token_indices + tl.p0 + g) : tl.p0 + g;
+    if (TM == 16 && g + 8 < tl.nvalid)
+        row_g8 = p.token_indices ? __ldg(p.token_indices + tl.p0 + g + 8) : tl.p0 + g + 8;
     int srank = 0;
     float sscale = 0.f;
     if (tid == 0) {
@@ -562,15 +608,22 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
         if (crank == 0 && warp == 0 && t == 0) report(v, kFlagBadRow);
         row_g = -1;
     }
-    const bool row_ok = row_g >= 0;
+    if (TM == 16 && g + 8 < tl.nvalid && (row_g8 < 0 || row_g8 >= p.n_rows)) {
+        if (crank == 0 && warp == 0 && t == 0) report(v, kFlagBadRow);
+        row_g8 = -1;
+    }
+    const bool row_ok = row_g >= 0, row_ok8 = row_g8 >= 0;
     // row pointers in X's and Y's element types
     XElem<XT> *xrow = reinterpret_cast<XElem<XT> *>(p.X) + (int64_t)(row_ok ? row_g : 0) * p.ldx;
     YElem<YT> *yrow = reinterpret_cast<YElem<YT> *>(v.Y) + (int64_t)(row_ok ? row_g : 0) * v.ldy;
+    XElem<XT> *xrow8 = reinterpret_cast<XElem<XT> *>(p.X) + (int64_t)(row_ok8 ? row_g8 : 0) * p.ldx;
+    YElem<YT> *yrow8 = reinterpret_cast<YElem<YT> *>(v.Y) + (int64_t)(row_ok8 ? row_g8 : 0) * v.ldy;
     if constexpr (MODE != MODE_EXPAND) {
-        load_x<R, XT>(s0, xrow, row_ok, sl, warp, t);
-        load_x<R, XT>(s1, xrow, row_ok, sl, warp + kWarps, t);
+        load_x<R, XT, TM>(s0, xrow, row_ok, xrow8, row_ok8, sl, warp, t);
+        load_x<R, XT, TM>(s1, xrow, row_ok, xrow8, row_ok8, sl, warp + kWarps, t);
     }
-    if constexpr (MODE != MODE_SHRINK && RC::EARLY_EXPAND) load_y<R, YT>(e0, yrow, row_ok, sl, warp, t);
+    if constexpr (MODE != MODE_SHRINK && RC::EARLY_EXPAND)
+        load_y<R, YT, TM>(e0, yrow, row_ok, yrow8, row_ok8, sl, warp, t);
 
     // ---- shrink: this CTA's d_in slice, two blocks in flight per warp
     if constexpr (MODE != MODE_EXPAND) {
@@ -578,18 +631,18 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
 #pragma unroll
         for (int n = 0; n < RC::NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
         for (int i = 0; i < nb; i += 2) {
-            mma_shrink<R>(acc, s0);
+            mma_shrink<R, TM>(acc, s0);
             if (i + 2 < nb) {
                 const int b = warp + (i + 2) * kWarps;
                 load_a<R>(s0, slotA, sl, b, g, t);
-                load_x<R, XT>(s0, xrow, row_ok, sl, b, t);
+                load_x<R, XT, TM>(s0, xrow, row_ok, xrow8, row_ok8, sl, b, t);
             }
             if (i + 1 < nb) {
-                mma_shrink<R>(acc, s1);
+                mma_shrink<R, TM>(acc, s1);
                 if (i + 3 < nb) {
                     const int b = warp + (i + 3) * kWarps;
                     load_a<R>(s1, slotA, sl, b, g, t);
-                    load_x<R, XT>(s1, xrow, row_ok, sl, b, t);
+                    load_x<R, XT, TM>(s1, xrow, row_ok, xrow8, row_ok8, sl, b, t);
                 }
             }
         }
@@ -597,29 +650,36 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
             // the expand's first groups travel while the cluster sums H
             if constexpr (!RC::EARLY_EXPAND) {
                 load_b<R, YT>(e0, slotB, v.d_out, sl, warp, g, t);
-                load_y<R, YT>(e0, yrow, row_ok, sl, warp, t);
+                load_y<R, YT, TM>(e0, yrow, row_ok, yrow8, row_ok8, sl, warp, t);
             }
             load_b<R, YT>(e1, slotB, v.d_out, sl, warp + kWarps, g, t);
-            load_y<R, YT>(e1, yrow, row_ok, sl, warp + kWarps, t);
+            load_y<R, YT, TM>(e1, yrow, row_ok, yrow8, row_ok8, sl, warp + kWarps, t);
         }
 #pragma unroll
         for (int n = 0; n < RC::NT; ++n) {
             wpart[(warp * TM + g) * R + n * 8 + 2 * t] = acc[n][0];
             wpart[(warp * TM + g) * R + n * 8 + 2 * t + 1] = acc[n][1];
+            if constexpr (TM == 16) {
+                wpart[(warp * TM + g + 8) * R + n * 8 + 2 * t] = acc[n][2];
+                wpart[(warp * TM + g + 8) * R + n * 8 + 2 * t + 1] = acc[n][3];
+            }
         }
     } else {
         load_b<R, YT>(e1, slotB, v.d_out, sl, warp + kWarps, g, t);
-        load_y<R, YT>(e1, yrow, row_ok, sl, warp + kWarps, t);
+        load_y<R, YT, TM>(e1, yrow, row_ok, yrow8, row_ok8, sl, warp + kWarps, t);
         if constexpr (!RC::EARLY_EXPAND) {
             load_b<R, YT>(e0, slotB, v.d_out, sl, warp, g, t);
-            load_y<R, YT>(e0, yrow, row_ok, sl, warp, t);
+            load_y<R, YT, TM>(e0, yrow, row_ok, yrow8, row_ok8, sl, warp, t);
         }
     }
     if (tid == 0) {
         ctl.slot_rank = srank;
         ctl.slot_scale = sscale;
     }
-    if (warp == 0 && t == 0) ctl.rows[g] = row_g;
+    if (warp == 0 && t == 0) {
+        ctl.rows[g] = row_g;
+        if constexpr (TM == 16) ctl.rows[g + 8] = row_g8;
+    }
     __syncthreads();
     const int r = ctl.slot_rank;
     const bool ok = r > 0 && (p.ranks == nullptr || r_meta == r) && rank_bucket(r) == R;
@@ -693,35 +753,38 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
     // ---- expand: this CTA's d_out slice, two groups in flight per warp
     if constexpr (MODE != MODE_SHRINK) {
         __syncthreads();
-        // H row g as bf16 hi + lo fragments; step s covers rank 16s + 4t .. 16s + 4t + 3
-        // (rank bucket 8: 2t, 2t + 1)
-        uint32_t ah[RC::KS][2], al[RC::KS][2];
+        // H rows g ([.][0..1]) and g + 8 ([.][2..3]) as bf16 hi + lo fragments; step s
+        // covers rank 16s + 4t .. 16s + 4t + 3 (rank bucket 8: 2t, 2t + 1)
+        uint32_t ah[RC::KS][TM / 4], al[RC::KS][TM / 4];
 #pragma unroll
         for (int s = 0; s < RC::KS; ++s) {
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int col = (R == 8) ? 2 * t : 16 * s + 4 * t + 2 * q;
+            for (int q = 0; q < TM / 4; ++q) {
+                const int col = (R == 8) ? 2 * t : 16 * s + 4 * t + 2 * (q & 1);
+                const int hr = g + 8 * (q >> 1);
                 float h0, l0, h1, l1;
-                split_bf16(hfull[g * DC::HPITCH + col], h0, l0);
-                split_bf16(hfull[g * DC::HPITCH + col + 1], h1, l1);
+                split_bf16(hfull[hr * DC::HPITCH + col], h0, l0);
+                split_bf16(hfull[hr * DC::HPITCH + col + 1], h1, l1);
                 ah[s][q] = pack_bf16x2(h0, h1);
                 al[s][q] = pack_bf16x2(l0, l1);
             }
         }
-        const bool store = ok && row_ok && h_ok && (MODE == MODE_EXPAND || ctl.fail == 0);
+        const bool live = ok && h_ok && (MODE == MODE_EXPAND || ctl.fail == 0);
+        const bool store = live && row_ok, store8 = live && row_ok8;
         for (int i = 0; i < ng; i += 2) {
-            mma_expand_store<R, YT>(e0, ah, al, scale, yrow, store, sl, warp + i * kWarps, t);
+            mma_expand_store<R, YT, TM>(e0, ah, al, scale, yrow, store, yrow8, store8, sl, warp + i * kWarps, t);
             if (i + 2 < ng) {
                 const int q = warp + (i + 2) * kWarps;
                 load_b<R, YT>(e0, slotB, v.d_out, sl, q, g, t);
-                load_y<R, YT>(e0, yrow, row_ok, sl, q, t);
+                load_y<R, YT, TM>(e0, yrow, row_ok, yrow8, row_ok8, sl, q, t);
             }
             if (i + 1 < ng) {
-                mma_expand_store<R, YT>(e1, ah, al, scale, yrow, store, sl, warp + (i + 1) * kWarps, t);
+                mma_expand_store<R, YT, TM>(e1, ah, al, scale, yrow, store, yrow8, store8, sl, warp + (i + 1) * kWarps,
+                                        t);
                 if (i + 3 < ng) {
                     const int q = warp + (i + 3) * kWarps;
                     load_b<R, YT>(e1, slotB, v.d_out, sl, q, g, t);
-                    load_y<R, YT>(e1, yrow, row_ok, sl, q, t);
+                    load_y<R, YT, TM>(e1, yrow, row_ok, yrow8, row_ok8, sl, q, t);
                 }
             }
         }
@@ -733,8 +796,8 @@ __device__ void run_tile(const TileParams &p, const ProjView &v, const Tile &tl,
 // work item is (tile, projection), projection fastest, so the clusters working on one
 // tile's projections run side by side and its X rows come from HBM once (the later
 // reads hit L2).  Otherwise the only projection is p.proj[0].
-template <int RMAX, int MODE, int NT, bool FUSED, int DT = 0>
-__global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
+template <int RMAX, int MODE, int NT, bool FUSED, int DT = 0, int TM = kTileRows>
+__global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT, TM>::MIN_BLOCKS))
     lora_decode_kernel(const __grid_constant__ TileParams p)
 {
     extern __shared__ __align__(16) float smem_f[];
@@ -762,10 +825,10 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
         cluster_arrive_release();
         cluster_wait_acquire();
     }
-    if (p.early) prefetch_first_tile<RMAX, MODE, NT, DT>(p, p.proj[k], tile, ctl, crank);
+    if (p.early) prefetch_first_tile<RMAX, MODE, NT, DT, TM>(p, p.proj[k], tile, ctl, crank);
     griddep_wait();
     const int item2 = item + n_clusters;   // this cluster's next work item
-    const int total = scan_tiles<false, NT, MODE, RMAX>(p, p.proj[k].slot_gen, tile, item2 / np,
+    const int total = scan_tiles<false, NT, MODE, RMAX, TM>(p, p.proj[k].slot_gen, tile, item2 / np,
                                                         p.proj[FUSED ? item2 % np : 0], ctl, reporter) *
                       np;
     uint32_t nt = 0;   // tiles done by this CTA (parity of the exchange buffers and barriers)
@@ -779,7 +842,7 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
         const ProjView &v = p.proj[k];
         if (item != (int)cluster_index()) {
             const int next = item + n_clusters;
-            scan_tiles<false, NT, MODE, RMAX>(p, v.slot_gen, tile, next / np, p.proj[FUSED ? next % np : 0],
+            scan_tiles<false, NT, MODE, RMAX, TM>(p, v.slot_gen, tile, next / np, p.proj[FUSED ? next % np : 0],
                                               ctl, false);
         }
         // every CTA of the cluster reads the same metadata and reaches the same tile
@@ -800,23 +863,23 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT>::MIN_BLOCKS))
             if (R == 0 || R > RMAX) R = 8;   // rejected inside; moves rank-8 bytes
         }
         if (R == 8) {
-            run_tile<RMAX, MODE, 8, NT, DT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+            run_tile<RMAX, MODE, 8, NT, DT, TM>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else if (R == 16) {
             if constexpr (RMAX >= 16)
-                run_tile<RMAX, MODE, 16, NT, DT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+                run_tile<RMAX, MODE, 16, NT, DT, TM>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else if (R == 32) {
             if constexpr (RMAX >= 32)
-                run_tile<RMAX, MODE, 32, NT, DT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+                run_tile<RMAX, MODE, 32, NT, DT, TM>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         } else {
             if constexpr (RMAX >= 64)
-                run_tile<RMAX, MODE, 64, NT, DT>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
+                run_tile<RMAX, MODE, 64, NT, DT, TM>(p, v, tl, r_meta, seg_scale, ctl, smem_f, crank, csize, nt);
         }
         __syncthreads();   // ctl and the H buffers are rewritten by the next tile
     }
 }
 
 // Clusters of `cluster` CTAs of this kernel resident at once (cached per device).
-template <int RMAX, int MODE, int NT, bool FUSED, int DT = 0>
+template <int RMAX, int MODE, int NT, bool FUSED, int DT = 0, int TM = kTileRows>
 cudaError_t active_clusters(int cluster, int &active)
 {
     static std::mutex mu;
@@ -829,7 +892,7 @@ cudaError_t active_clusters(int cluster, int &active)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)cluster, 1, 1);
     cfg.blockDim = dim3(NT, 1, 1);
-    cfg.dynamicSmemBytes = DecodeCfg<RMAX, NT>::SMEM;
+    cfg.dynamicSmemBytes = DecodeCfg<RMAX, NT, TM>::SMEM;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)cluster;
@@ -837,20 +900,21 @@ cudaError_t active_clusters(int cluster, int &active)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaOccupancyMaxActiveClusters(&active, lora_decode_kernel<RMAX, MODE, NT, FUSED, DT>, &cfg);
+    cudaError_t e =
+        cudaOccupancyMaxActiveClusters(&active, lora_decode_kernel<RMAX, MODE, NT, FUSED, DT, TM>, &cfg);
     if (e != cudaSuccess) return e;
     if (active <= 0) return cudaErrorInvalidConfiguration;
     cached[dev][cluster] = active;
     return cudaSuccess;
 }
 
-template <int RMAX, int MODE, int NT, bool FUSED, int DT = 0>
+template <int RMAX, int MODE, int NT, bool FUSED, int DT = 0, int TM = kTileRows>
 cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, int active,
                        cudaStream_t stream)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(NT, 1, 1);
-    cfg.dynamicSmemBytes = DecodeCfg<RMAX, NT>::SMEM;
+    cfg.dynamicSmemBytes = DecodeCfg<RMAX, NT, TM>::SMEM;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -865,7 +929,7 @@ cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, int 
     cfg.numAttrs = p.early ? 2 : 1;
     const int64_t n = max_tiles < active ? max_tiles : active;
     cfg.gridDim = dim3((unsigned)(n * cluster), 1, 1);
-    return cudaLaunchKernelEx(&cfg, lora_decode_kernel<RMAX, MODE, NT, FUSED, DT>, p);
+    return cudaLaunchKernelEx(&cfg, lora_decode_kernel<RMAX, MODE, NT, FUSED, DT, TM>, p);
 }
 
 // CTA width.  256 threads keep each warp's operands in one round of loads; when the
@@ -873,24 +937,36 @@ cudaError_t launch_one(const TileParams &p, int cluster, int64_t max_tiles, int 
 // long decode segments), 128-thread CTAs let twice as many tiles be in flight, which
 // hides more latency than their second round of loads costs (measured: a 4096 x 4096
 // batch of 60 tiles is 36% slower with 128 threads, batches of 300+ tiles 3-6% faster).
-template <int RMAX, int MODE, bool FUSED = false, int DT = 0>
+template <int RMAX, int MODE, bool FUSED = false, int DT = 0, int TM = kTileRows>
 cudaError_t launch_mode(const TileParams &p, int cluster, int64_t max_tiles, cudaStream_t stream)
 {
     int active = 0;
-    cudaError_t e = active_clusters<RMAX, MODE, 256, FUSED, DT>(cluster, active);
+    cudaError_t e = active_clusters<RMAX, MODE, 256, FUSED, DT, TM>(cluster, active);
     if (e != cudaSuccess) return e;
     if (2 * max_tiles > 3 * (int64_t)active) {
         int active128 = 0;
-        e = active_clusters<RMAX, MODE, 128, FUSED, DT>(cluster, active128);
+        e = active_clusters<RMAX, MODE, 128, FUSED, DT, TM>(cluster, active128);
         if (e != cudaSuccess) return e;
         // Early launch with adapter prefetch only pays for batches of about one wave of
         // tiles: with many more, the prefetched slices thrash L2 and the early CTAs
         // hold slots (measured 16% slower on 2048 decode rows over 128 adapters).
         TileParams q = p;
         q.early = 0;
-        return launch_one<RMAX, MODE, 128, FUSED, DT>(q, cluster, max_tiles, active128, stream);
+        return launch_one<RMAX, MODE, 128, FUSED, DT, TM>(q, cluster, max_tiles, active128, stream);
     }
-    return launch_one<RMAX, MODE, 256, FUSED, DT>(p, cluster, max_tiles, active, stream);
+    return launch_one<RMAX, MODE, 256, FUSED, DT, TM>(p, cluster, max_tiles, active, stream);
+}
+
+// 16-row tiles for batches of long decode segments at small rank (see kMaxTM).
+// max_tiles counts 8-row tiles; a 16-row tile takes about two of them.
+template <int RMAX, bool FUSED>
+cudaError_t launch_apply(const TileParams &p, int cluster, int64_t max_tiles, cudaStream_t stream)
+{
+    if constexpr (RMAX <= 16) {
+        if ((int64_t)p.n_tokens >= 8 * (int64_t)p.n_segments)
+            return launch_mode<RMAX, MODE_APPLY, FUSED, 0, 16>(p, cluster, (max_tiles + 1) / 2 + 1, stream);
+    }
+    return launch_mode<RMAX, MODE_APPLY, FUSED>(p, cluster, max_tiles, stream);
 }
 
 // The fused apply with another dtype boundary (DT != 0: FP8 X codes and / or an fp16 or
@@ -913,7 +989,7 @@ cudaError_t launch_rmax(int mode, const TileParams &p, int cluster, int64_t max_
                         cudaStream_t stream)
 {
     switch (mode) {
-    case MODE_APPLY: return launch_mode<RMAX, MODE_APPLY>(p, cluster, max_tiles, stream);
+    case MODE_APPLY: return launch_apply<RMAX, false>(p, cluster, max_tiles, stream);
     case MODE_SHRINK: return launch_mode<RMAX, MODE_SHRINK>(p, cluster, max_tiles, stream);
     case MODE_EXPAND: return launch_mode<RMAX, MODE_EXPAND>(p, cluster, max_tiles, stream);
     default: return cudaErrorInvalidValue;
@@ -927,6 +1003,14 @@ template <int RMAX, int NT>
 cudaError_t set_attrs_nt()
 {
     cudaError_t e;
+    if constexpr (RMAX <= 16) {
+        e = cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_APPLY, NT, false, 0, 16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX, NT, 16>::SMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_APPLY, NT, true, 0, 16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX, NT, 16>::SMEM);
+        if (e != cudaSuccess) return e;
+    }
     e = cudaFuncSetAttribute(lora_decode_kernel<RMAX, MODE_APPLY, NT, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeCfg<RMAX, NT>::SMEM);
     if (e != cudaSuccess) return e;
@@ -1049,8 +1133,8 @@ cudaError_t launch_tile_kernel_fused(int rmax_bucket, const TileParams &p, int c
     if (cluster < 1 || cluster > kMaxCluster || max_items < 1) return cudaErrorInvalidValue;
     if (p.n_proj < 1 || p.n_proj > kMaxFused) return cudaErrorInvalidValue;
     switch (rmax_bucket) {
-    case 8: return launch_mode<8, MODE_APPLY, true>(p, cluster, max_items, stream);
-    case 16: return launch_mode<16, MODE_APPLY, true>(p, cluster, max_items, stream);
+    case 8: return launch_apply<8, true>(p, cluster, max_items, stream);
+    case 16: return launch_apply<16, true>(p, cluster, max_items, stream);
     case 32: return launch_mode<32, MODE_APPLY, true>(p, cluster, max_items, stream);
     case 64: return launch_mode<64, MODE_APPLY, true>(p, cluster, max_items, stream);
     default: return cudaErrorInvalidValue;
