@@ -47,6 +47,8 @@ struct ProjView {
     int32_t d_out, n_slice;
     __nv_bfloat16 *Y;
     int64_t ldy;
+    float *ws;                  // fused long-segment shrink: this projection's H workspace
+    int64_t ws_ld;
 };
 
 // Everything one launch of the segmented tile kernel needs.  Passed by value.
@@ -133,8 +135,10 @@ constexpr int kExpandChunk = 128;
 
 // Long-segment shrink (H of the long tiles into p.ws) and expand (reads p.ws; in
 // MODE_EXPAND it also reports the tiles' metadata problems); persistent grids.
+// np >= 2: one launch for projections 0 .. np-1 of a fused call (projection 0 from
+// p's own fields, the others from p.proj[j], each H into its own workspace).
 cudaError_t launch_long_shrink(int rmax_bucket, const TileParams &p, int64_t max_tiles,
-                               cudaStream_t stream);
+                               cudaStream_t stream, int np = 1);
 cudaError_t launch_long_expand(int rmax_bucket, int mode, const TileParams &p, int64_t max_tiles,
                                cudaStream_t stream);
 cudaError_t prepare_long_kernels();

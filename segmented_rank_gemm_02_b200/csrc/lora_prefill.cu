@@ -31,6 +31,11 @@
 // coalesced 16-byte stores) and releases the stages.  The roles meet only at
 // mbarriers, so copies, tensor-core work, epilogue and stores overlap.
 //
+// Fused projections (mlora_apply_multi): one shrink launch serves up to four
+// projections that share X, with one A block per projection in each stage and one
+// accumulator per projection in tensor memory, so the prefill rows of X are read
+// once; each projection's H goes to its own workspace and its own expand follows.
+//
 // Which segments come here: those of at least 128 grouped positions whose rows are
 // consecutive in X and Y (prefill requests); see long_segment().  The shrink is
 // launched after the decode-shaped kernel and the expand after the shrink with
@@ -67,16 +72,26 @@ constexpr uint64_t kWaitNs = 1000000000ull;
 
 __host__ __device__ constexpr int padded_rank(int r) { return r < 16 ? 16 : r; }
 
-template <int RMAX>
-struct LongCfg {
+// Shrink of NP projections that share X (one A block per projection per stage, one
+// accumulator of RK columns per projection in tensor memory).
+template <int RMAX, int NP = 1>
+struct ShrinkCfg {
     static constexpr int RK = padded_rank(RMAX);
     static constexpr int X_STAGE = PM * KB * 2;          // 16 KB, 128-byte swizzle
     static constexpr int A_STAGE = (8 * RK * 16 + 1023) / 1024 * 1024;   // [8][RK][8]
-    static constexpr int S_STAGE = X_STAGE + A_STAGE;    // multiple of 1024
+    static constexpr int S_STAGE = X_STAGE + NP * A_STAGE;   // multiple of 1024
+    static constexpr int NSTAGE_FIT = (200 * 1024) / S_STAGE;
+    static constexpr int NSTAGE = NSTAGE_FIT < NS ? NSTAGE_FIT : NS;
     static constexpr int RED_PITCH = RK + 4;             // floats per row of a partial tile
-    static constexpr int S_SMEM = 1024 + NS * S_STAGE + kZeroBytes;   // + alignment slack
-    static_assert(PM * RED_PITCH * 4 <= NS * S_STAGE, "partial tile must fit in the ring");
-    static constexpr int S_TMEM = RK < 32 ? 32 : RK;
+    static constexpr int S_SMEM = 1024 + NSTAGE * S_STAGE + kZeroBytes;   // + alignment slack
+    static_assert(NSTAGE >= 3, "shrink ring");
+    static_assert(PM * RED_PITCH * 4 <= NSTAGE * S_STAGE, "partial tile must fit in the ring");
+    static constexpr int S_TMEM = NP * RK <= 32 ? 32 : NP * RK <= 64 ? 64 : NP * RK <= 128 ? 128 : 256;
+};
+
+template <int RMAX>
+struct LongCfg {
+    static constexpr int RK = padded_rank(RMAX);
     static constexpr int H_BYTES = PM * RK * 2;          // one of hi / lo: [RK/8][16][8][8]
     static constexpr int B_BYTES = (NCH * RK * 2 + 1023) / 1024 * 1024;  // [RK/8][128][8]
     static constexpr int Y_BYTES = PM * NCH * 2;         // two 64-column halves, swizzled
@@ -222,23 +237,30 @@ __device__ __forceinline__ bool wait_or_fail(const TileParams &p, LongCtl &ctl, 
 // the CTA's partial tile goes from tensor memory to shared memory, and the cluster
 // sums its partials through distributed shared memory, each CTA one contiguous
 // share of the tile, written to H with coalesced 16-byte stores.
-template <int RMAX, int R>
+// Projection j of a shrink launch: j = 0 is the launch's own pool and H workspace,
+// j >= 1 the further projections of a fused launch (same X, same slot numbering).
+__device__ __forceinline__ const __nv_bfloat16 *proj_slot_a(const TileParams &p, int j, int slot)
+{
+    return j == 0 ? p.pool + (int64_t)slot * p.slot_stride : p.proj[j].pool + (int64_t)slot * p.proj[j].slot_stride;
+}
+
+template <int RMAX, int R, int NP>
 __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, uint8_t *zero,
                             uint32_t tmem, uint32_t &gb, uint32_t &tc, uint32_t crank, uint32_t csize,
                             int nvalid, int rank, bool ok)
 {
-    using C = LongCfg<RMAX>;
+    using C = ShrinkCfg<RMAX, NP>;
+    constexpr int NSTAGE = C::NSTAGE;
     constexpr int RK = padded_rank(R);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int p0 = ctl.tile[1], slot = ctl.tile[3];
-    const __nv_bfloat16 *slotA = p.pool + (int64_t)slot * p.slot_stride;
     const int k0 = min(p.d_in, (int)crank * p.k_part);
     const int k1 = min(p.d_in, k0 + p.k_part);
     const int nkb = (k1 - k0 + KB - 1) / KB;
     constexpr uint32_t A_BYTES = 8 * R * 16;
 
     if (warp == 0) {
-        // ---- copies: X block (tile or gathers) + A block per stage
+        // ---- copies: X block (tile or gathers) + one A block per projection per stage
         const bool contiguous = ctl.contiguous != 0;
         int r[4];
 #pragma unroll
@@ -248,146 +270,162 @@ __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, ui
         }
         for (int b = 0; b < nkb; ++b) {
             const uint32_t G = gb + b;
-            const int s = (int)(G % NS);
+            const int s = (int)(G % NSTAGE);
             bool go = true;
-            if (lane == 0 && G >= (uint32_t)NS) go = wait_or_fail(p, ctl, &ctl.bar[s], ((G / NS) - 1) & 1u);
+            if (lane == 0 && G >= (uint32_t)NSTAGE)
+                go = wait_or_fail(p, ctl, &ctl.bar[s], ((G / NSTAGE) - 1) & 1u);
             if (__shfl_sync(0xffffffffu, go ? 1 : 0, 0) == 0) break;
             uint8_t *xs = ring + s * C::S_STAGE;
             uint8_t *as = xs + C::X_STAGE;
             const int kb0 = k0 + b * KB;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&ctl.full[s], (uint32_t)C::X_STAGE + A_BYTES);
+                mbar_arrive_expect_tx(&ctl.full[s], (uint32_t)C::X_STAGE + NP * A_BYTES);
                 if (contiguous) tma_load_2d(xs, &p.x_tile, kb0, ctl.rows[0], &ctl.full[s]);
-                bulk_load(as, slotA + (int64_t)(kb0 / 8) * R * 8, A_BYTES, &ctl.full[s]);
+#pragma unroll
+                for (int j = 0; j < NP; ++j)
+                    bulk_load(as + j * C::A_STAGE, proj_slot_a(p, j, slot) + (int64_t)(kb0 / 8) * R * 8, A_BYTES,
+                              &ctl.full[s]);
             }
             __syncwarp();
             if (!contiguous)
                 tma_gather4(xs + lane * 4 * 128, &p.x_rows, kb0, r[0], r[1], r[2], r[3], &ctl.full[s]);
         }
     } else if (warp == 1 && lane == 0) {
-        // ---- tensor core: 4 K=16 steps per block into one fp32 accumulator
+        // ---- tensor core: 4 K=16 steps per block into one fp32 accumulator per projection
         const uint32_t idesc = umma_idesc_bf16(PM, RK);
         for (int b = 0; b < nkb; ++b) {
             const uint32_t G = gb + b;
-            const int s = (int)(G % NS);
-            if (!wait_or_fail(p, ctl, &ctl.full[s], (G / NS) & 1u)) break;
+            const int s = (int)(G % NSTAGE);
+            if (!wait_or_fail(p, ctl, &ctl.full[s], (G / NSTAGE) & 1u)) break;
             tc_fence_after();
             const uint32_t xs = smem_addr(ring + s * C::S_STAGE);
             const uint32_t as = xs + C::X_STAGE;
 #pragma unroll
             for (int st = 0; st < KB / 16; ++st) {
-                const uint32_t a0 = as + st * 2 * R * 16;
-                // adapter rows 8 .. 15 of bucket 8 come from the zero block
-                const uint32_t sbo = (R == 8) ? smem_addr(zero) - a0 : 128;
                 const uint64_t ad = umma_desc_sw128(xs + st * 32);
-                const uint64_t bd = umma_desc_kmajor(a0, R * 16, sbo);
-                umma_bf16(tmem, ad, bd, idesc, (b > 0 || st > 0) ? 1u : 0u);
+#pragma unroll
+                for (int j = 0; j < NP; ++j) {
+                    const uint32_t a0 = as + j * C::A_STAGE + st * 2 * R * 16;
+                    // adapter rows 8 .. 15 of bucket 8 come from the zero block
+                    const uint32_t sbo = (R == 8) ? smem_addr(zero) - a0 : 128;
+                    const uint64_t bd = umma_desc_kmajor(a0, R * 16, sbo);
+                    umma_bf16(tmem + (uint32_t)(j * RK), ad, bd, idesc, (b > 0 || st > 0) ? 1u : 0u);
+                }
             }
             umma_commit(&ctl.bar[s]);   // stage s is free once these MMAs end
         }
-        umma_commit(&ctl.done);         // the partial tile is complete
+        umma_commit(&ctl.done);         // the partial tiles are complete
     }
     gb += nkb;
     // the other threads (and lanes 1..31 of warp 1) wait here, at a hardware barrier,
     // instead of spinning beside the copy and MMA loops
     __syncthreads();
-    // everyone: the accumulator is final (bounded wait; a timeout leaves zeros)
+    // everyone: the accumulators are final (bounded wait; a timeout leaves zeros)
     // (warp-uniform: tcgen05.ld below is a warp-wide instruction)
     const bool acc_ok = __all_sync(0xffffffffu, wait_or_fail(p, ctl, &ctl.done, tc & 1u));
     ++tc;
     tc_fence_after();
 
-    // this CTA's partial tile from tensor memory: warp w holds rows 32 (w % 4) .. +31
-    // and columns [(w / 4) * RK/2, +RK/2)
-    constexpr int HC = RK / 2;
-    float h[HC];
-    const int col0 = (warp / 4) * HC;
-    if (nkb > 0 && acc_ok) {
-        const uint32_t taddr = tmem + ((uint32_t)(32 * (warp % 4)) << 16) + col0;
-        if constexpr (HC == 8) {
-            uint32_t v0[8];
-            tmem_ld8(taddr, v0);
-            tmem_wait_ld();
+    for (int j = 0; j < NP; ++j) {
+        // projection j: its pool must hold the slot at the same rank (a pool that does
+        // not is rejected by that projection's expand, which reads its own slot table)
+        bool ok_j = ok;
+        if (j > 0 && ok_j) ok_j = p.proj[j].slot_rank[slot] == rank;
+        float *ws = j == 0 ? p.ws : p.proj[j].ws;
+        const int64_t ws_ld = j == 0 ? p.ws_ld : p.proj[j].ws_ld;
+        // this CTA's partial tile from tensor memory: warp w holds rows 32 (w % 4) .. +31
+        // and columns [(w / 4) * RK/2, +RK/2) of projection j's accumulator
+        constexpr int HC = RK / 2;
+        float h[HC];
+        const int col0 = (warp / 4) * HC;
+        if (nkb > 0 && acc_ok) {
+            const uint32_t taddr = tmem + ((uint32_t)(32 * (warp % 4)) << 16) + (uint32_t)(j * RK) + col0;
+            if constexpr (HC == 8) {
+                uint32_t v0[8];
+                tmem_ld8(taddr, v0);
+                tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 8; ++j) h[j] = __uint_as_float(v0[j]);
-        } else if constexpr (HC == 16) {
-            uint32_t v0[8], v1[8];
-            tmem_ld8(taddr, v0);
-            tmem_ld8(taddr + 8, v1);
-            tmem_wait_ld();
+                for (int c = 0; c < 8; ++c) h[c] = __uint_as_float(v0[c]);
+            } else if constexpr (HC == 16) {
+                uint32_t v0[8], v1[8];
+                tmem_ld8(taddr, v0);
+                tmem_ld8(taddr + 8, v1);
+                tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                h[j] = __uint_as_float(v0[j]);
-                h[8 + j] = __uint_as_float(v1[j]);
+                for (int c = 0; c < 8; ++c) {
+                    h[c] = __uint_as_float(v0[c]);
+                    h[8 + c] = __uint_as_float(v1[c]);
+                }
+            } else {
+                uint32_t v[32];
+                tmem_ld32(taddr, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) h[c] = __uint_as_float(v[c]);
             }
         } else {
-            uint32_t v[32];
-            tmem_ld32(taddr, v);
-            tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) h[j] = __uint_as_float(v[j]);
+            for (int c = 0; c < HC; ++c) h[c] = 0.f;
         }
-    } else {
+        // every block of this tile has been consumed, so the ring holds the partial tile
+        float *red = reinterpret_cast<float *>(ring);
+        const int trow = 32 * (warp % 4) + (tid & 31);
 #pragma unroll
-        for (int j = 0; j < HC; ++j) h[j] = 0.f;
-    }
-    // every block of this tile has been consumed, so the ring holds the partial tile
-    float *red = reinterpret_cast<float *>(ring);
-    const int trow = 32 * (warp % 4) + (tid & 31);
-#pragma unroll
-    for (int j = 0; j < HC; j += 4)
-        *reinterpret_cast<float4 *>(red + trow * C::RED_PITCH + col0 + j) =
-            make_float4(h[j], h[j + 1], h[j + 2], h[j + 3]);
-    tc_fence_before();
-    cluster_arrive_release();
-    cluster_wait_acquire();
-    // CTA crank sums the cluster's partials (in CTA order) for its share of the tile's
-    // float4 slots, row-major, and writes them to H: consecutive threads write
-    // consecutive columns of a row
-    if (ok && !ctl.fail) {
-        constexpr int F4 = RK / 4;                       // float4 slots per row
-        const int total = PM * F4;
-        const int per = (total + (int)csize - 1) / (int)csize;
-        const int f_lo = (int)crank * per, f_hi = min(total, f_lo + per);
-        for (int f = f_lo + tid; f < f_hi; f += PT) {
-            const int row = f / F4, c4 = f % F4;
-            if (row >= nvalid || ctl.rows[row] < 0 || 4 * c4 >= rank) continue;
-            const uint32_t addr = smem_addr(red + row * C::RED_PITCH + 4 * c4);
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (uint32_t c = 0; c < csize; ++c) {
-                const float4 v = ld_dsmem_f32x4(map_to_rank(addr, c));
-                acc.x += v.x;
-                acc.y += v.y;
-                acc.z += v.z;
-                acc.w += v.w;
-            }
-            float *dst = p.ws + (int64_t)(p0 + row) * p.ws_ld + 4 * c4;
-            if (4 * c4 + 4 <= rank) {
-                *reinterpret_cast<float4 *>(dst) = acc;
-            } else {   // columns >= rank are left alone
-                const int n = rank - 4 * c4;
-                dst[0] = acc.x;
-                if (n > 1) dst[1] = acc.y;
-                if (n > 2) dst[2] = acc.z;
+        for (int c = 0; c < HC; c += 4)
+            *reinterpret_cast<float4 *>(red + trow * C::RED_PITCH + col0 + c) =
+                make_float4(h[c], h[c + 1], h[c + 2], h[c + 3]);
+        tc_fence_before();
+        cluster_arrive_release();
+        cluster_wait_acquire();
+        // CTA crank sums the cluster's partials (in CTA order) for its share of the tile's
+        // float4 slots, row-major, and writes them to H: consecutive threads write
+        // consecutive columns of a row
+        if (ok_j && !ctl.fail) {
+            constexpr int F4 = RK / 4;                       // float4 slots per row
+            const int total = PM * F4;
+            const int per = (total + (int)csize - 1) / (int)csize;
+            const int f_lo = (int)crank * per, f_hi = min(total, f_lo + per);
+            for (int f = f_lo + tid; f < f_hi; f += PT) {
+                const int row = f / F4, c4 = f % F4;
+                if (row >= nvalid || ctl.rows[row] < 0 || 4 * c4 >= rank) continue;
+                const uint32_t addr = smem_addr(red + row * C::RED_PITCH + 4 * c4);
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (uint32_t c = 0; c < csize; ++c) {
+                    const float4 v = ld_dsmem_f32x4(map_to_rank(addr, c));
+                    acc.x += v.x;
+                    acc.y += v.y;
+                    acc.z += v.z;
+                    acc.w += v.w;
+                }
+                float *dst = ws + (int64_t)(p0 + row) * ws_ld + 4 * c4;
+                if (4 * c4 + 4 <= rank) {
+                    *reinterpret_cast<float4 *>(dst) = acc;
+                } else {   // columns >= rank are left alone
+                    const int n = rank - 4 * c4;
+                    dst[0] = acc.x;
+                    if (n > 1) dst[1] = acc.y;
+                    if (n > 2) dst[2] = acc.z;
+                }
             }
         }
+        // peers are done reading this CTA's partial tile before it is overwritten (next
+        // projection) or the ring is refilled
+        cluster_arrive_release();
+        cluster_wait_acquire();
     }
-    // peers are done reading this CTA's partial tile before the ring is refilled
-    cluster_arrive_release();
-    cluster_wait_acquire();
     fence_proxy_async_smem();   // the ring is next written by TMA
     __syncthreads();
     tc_fence_after();
 }
 
-template <int RMAX>
+template <int RMAX, int NP>
 __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__ TileParams p)
 {
-    using C = LongCfg<RMAX>;
+    using C = ShrinkCfg<RMAX, NP>;
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ LongCtl ctl;
     uint8_t *ring = align1024(smem_raw);
-    uint8_t *zero = ring + NS * C::S_STAGE;
+    uint8_t *zero = ring + C::NSTAGE * C::S_STAGE;
     const int tid = threadIdx.x, warp = tid >> 5;
     const uint32_t crank = cluster_rank(), csize = cluster_size();
     const int n_clusters = (int)(gridDim.x / csize);
@@ -400,7 +438,7 @@ __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__
     for (int i = tid; i < kZeroBytes / 16; i += PT) reinterpret_cast<uint4 *>(zero)[i] = make_uint4(0, 0, 0, 0);
     if (tid == 0) {
 #pragma unroll
-        for (int s = 0; s < NS; ++s) {
+        for (int s = 0; s < C::NSTAGE; ++s) {
             mbar_init(&ctl.bar[s], 1);
             mbar_init(&ctl.full[s], 1);
         }
@@ -423,15 +461,15 @@ __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__
         int rank;
         const int R = tile_setup(p, ctl, nvalid, crank == 0, ok, rank);
         if (R == 8) {
-            shrink_tile<RMAX, 8>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
+            shrink_tile<RMAX, 8, NP>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
         } else if (R == 16) {
-            shrink_tile<RMAX, 16>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
+            shrink_tile<RMAX, 16, NP>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
         } else if (R == 32) {
             if constexpr (RMAX >= 32)
-                shrink_tile<RMAX, 32>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
+                shrink_tile<RMAX, 32, NP>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
         } else if (R == 64) {
             if constexpr (RMAX >= 64)
-                shrink_tile<RMAX, 64>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
+                shrink_tile<RMAX, 64, NP>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
         }
         __syncthreads();
     }
@@ -953,10 +991,10 @@ int resident_per_sm(K kernel, int threads, int smem, int tmem_cols)
 }
 
 // Clusters of `cluster` shrink CTAs resident at once on the current device (cached).
-template <int RMAX>
+template <int RMAX, int NP = 1>
 cudaError_t shrink_active(int cluster, int &active)
 {
-    using C = LongCfg<RMAX>;
+    using C = ShrinkCfg<RMAX, NP>;
     static std::mutex mu;
     static int cached[64][kMaxSplit + 1] = {};
     int dev = 0;
@@ -975,7 +1013,7 @@ cudaError_t shrink_active(int cluster, int &active)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaOccupancyMaxActiveClusters(&active, long_shrink_kernel<RMAX>, &cfg);
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&active, long_shrink_kernel<RMAX, NP>, &cfg);
     if (e != cudaSuccess) return e;
     if (active <= 0) return cudaErrorInvalidConfiguration;
     int sms = 0;
@@ -987,13 +1025,13 @@ cudaError_t shrink_active(int cluster, int &active)
     return cudaSuccess;
 }
 
-template <int RMAX>
+template <int RMAX, int NP = 1>
 cudaError_t shrink_rmax(const TileParams &p, int64_t max_tiles, cudaStream_t stream)
 {
-    using C = LongCfg<RMAX>;
+    using C = ShrinkCfg<RMAX, NP>;
     const int cluster = p.ksplit;
     int active = 0;
-    cudaError_t e = shrink_active<RMAX>(cluster, active);
+    cudaError_t e = shrink_active<RMAX, NP>(cluster, active);
     if (e != cudaSuccess) return e;
     const int64_t n = max_tiles < active ? max_tiles : active;
     if (n <= 0) return cudaSuccess;
@@ -1012,7 +1050,7 @@ cudaError_t shrink_rmax(const TileParams &p, int64_t max_tiles, cudaStream_t str
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, long_shrink_kernel<RMAX>, p);
+    return cudaLaunchKernelEx(&cfg, long_shrink_kernel<RMAX, NP>, p);
 }
 
 template <int RMAX, int MODE>
@@ -1053,14 +1091,23 @@ cudaError_t set_smem(K kernel, int bytes)
     return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
 }
 
+template <int RMAX, int NP>
+cudaError_t set_shrink_attrs()
+{
+    cudaError_t e;
+    if ((e = set_smem(long_shrink_kernel<RMAX, NP>, ShrinkCfg<RMAX, NP>::S_SMEM)) != cudaSuccess) return e;
+    return cudaFuncSetAttribute(long_shrink_kernel<RMAX, NP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+}
+
 template <int RMAX>
 cudaError_t set_long_attrs()
 {
     using C = LongCfg<RMAX>;
     cudaError_t e;
-    if ((e = set_smem(long_shrink_kernel<RMAX>, C::S_SMEM)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(long_shrink_kernel<RMAX>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess)
-        return e;
+    if ((e = set_shrink_attrs<RMAX, 1>()) != cudaSuccess) return e;
+    if ((e = set_shrink_attrs<RMAX, 2>()) != cudaSuccess) return e;
+    if ((e = set_shrink_attrs<RMAX, 3>()) != cudaSuccess) return e;
+    if ((e = set_shrink_attrs<RMAX, 4>()) != cudaSuccess) return e;
     if ((e = set_smem(long_expand_kernel<RMAX, MODE_APPLY>, C::E_SMEM)) != cudaSuccess) return e;
     return set_smem(long_expand_kernel<RMAX, MODE_EXPAND>, C::E_SMEM);
 }
@@ -1090,15 +1137,31 @@ int long_shrink_split(int rmax_bucket, int d_in, int64_t tiles)
     return best;
 }
 
-cudaError_t launch_long_shrink(int rmax_bucket, const TileParams &p, int64_t max_tiles,
-                               cudaStream_t stream)
+namespace {
+
+template <int NP>
+cudaError_t launch_shrink_np(int rmax_bucket, const TileParams &p, int64_t max_tiles, cudaStream_t stream)
 {
-    if (p.ksplit < 1 || p.ksplit > kMaxSplit) return cudaErrorInvalidValue;
     switch (rmax_bucket) {
     case 8:
-    case 16: return shrink_rmax<16>(p, max_tiles, stream);
-    case 32: return shrink_rmax<32>(p, max_tiles, stream);
-    case 64: return shrink_rmax<64>(p, max_tiles, stream);
+    case 16: return shrink_rmax<16, NP>(p, max_tiles, stream);
+    case 32: return shrink_rmax<32, NP>(p, max_tiles, stream);
+    case 64: return shrink_rmax<64, NP>(p, max_tiles, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_long_shrink(int rmax_bucket, const TileParams &p, int64_t max_tiles,
+                               cudaStream_t stream, int np)
+{
+    if (p.ksplit < 1 || p.ksplit > kMaxSplit) return cudaErrorInvalidValue;
+    switch (np) {
+    case 1: return launch_shrink_np<1>(rmax_bucket, p, max_tiles, stream);
+    case 2: return launch_shrink_np<2>(rmax_bucket, p, max_tiles, stream);
+    case 3: return launch_shrink_np<3>(rmax_bucket, p, max_tiles, stream);
+    case 4: return launch_shrink_np<4>(rmax_bucket, p, max_tiles, stream);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -248,7 +248,7 @@ void set_single_projection(mlora::TileParams &p)
 }
 
 mlora_status launch_long(mlora_pool *pool, const mlora_segments *s, int mode, mlora::TileParams &p,
-                         cudaStream_t stream, float *ext_ws, size_t ext_ws_bytes);
+                         cudaStream_t stream, float *ext_ws, size_t ext_ws_bytes, bool run_shrink = true);
 
 // `ext_ws` (optional): caller-provided memory of `ext_ws_bytes` for the long-segment H
 // workspace, used instead of the pool's own (which is then never grown).
@@ -274,28 +274,45 @@ mlora_status launch(mlora_pool *pool, const mlora_segments *s, int mode, mlora::
     return launch_long(pool, s, mode, p, stream, ext_ws, ext_ws_bytes);
 }
 
-// The long-segment kernels (shrink, then expand) of one projection.
+// Upper bound on the long tiles of a batch (grid sizing of the long kernels).
+int64_t long_tile_bound(const mlora_segments *s)
+{
+    return (int64_t)s->n_tokens / mlora::kLongTileRows + s->n_tokens / kLongRows + 1;
+}
+
+// Shrink geometry of the long-segment kernels (d_in split over a cluster of ksplit
+// CTAs per tile) and the TMA views of X (tiles of consecutive rows, single rows for
+// gathers).
+mlora_status setup_long_shrink(const mlora_pool *pool, const mlora_segments *s, mlora::TileParams &p)
+{
+    p.long_rows = kLongRows;
+    p.early = 0;
+    const int64_t est_tiles = std::max<int64_t>(1, (s->n_tokens + mlora::kLongTileRows - 1) / mlora::kLongTileRows);
+    int ksplit = mlora::long_shrink_split(pool->r_bucket_max, pool->d_in, est_tiles);
+    p.k_part = (int32_t)round_up((pool->d_in + ksplit - 1) / ksplit, 64);
+    ksplit = (pool->d_in + p.k_part - 1) / p.k_part;
+    p.ksplit = ksplit;
+    if (!encode_rows_map(&p.x_tile, p.X, s->n_rows, pool->d_in, p.ldx, mlora::kLongTileRows) ||
+        !encode_rows_map(&p.x_rows, p.X, s->n_rows, pool->d_in, p.ldx, 1))
+        return MLORA_ERR_CUDA;
+    return MLORA_OK;
+}
+
+// The long-segment kernels (shrink, then expand) of one projection; without
+// run_shrink only the expand, on the H a fused shrink already left in the workspace.
 mlora_status launch_long(mlora_pool *pool, const mlora_segments *s, int mode, mlora::TileParams &p,
-                         cudaStream_t stream, float *ext_ws, size_t ext_ws_bytes)
+                         cudaStream_t stream, float *ext_ws, size_t ext_ws_bytes, bool run_shrink)
 {
     mlora_status st = MLORA_OK;
     cudaError_t e = cudaSuccess;
     p.long_rows = kLongRows;
     p.early = 0;
-    const int64_t long_tiles = (int64_t)s->n_tokens / mlora::kLongTileRows + s->n_tokens / kLongRows + 1;
-    const int64_t est_tiles = std::max<int64_t>(1, (s->n_tokens + mlora::kLongTileRows - 1) / mlora::kLongTileRows);
+    const int64_t long_tiles = long_tile_bound(s);
     const int rk = std::max(16, pool->r_bucket_max);
-    // shrink: a cluster of ksplit CTAs per tile, each a part of d_in
-    int ksplit = mlora::long_shrink_split(pool->r_bucket_max, pool->d_in, est_tiles);
-    p.k_part = (int32_t)round_up((pool->d_in + ksplit - 1) / ksplit, 64);
-    ksplit = (pool->d_in + p.k_part - 1) / p.k_part;
-    p.ksplit = ksplit;
-
-    // TMA views of the activations (tiles of consecutive rows, and single rows for gathers)
-    if (mode != mlora::MODE_EXPAND &&
-        (!encode_rows_map(&p.x_tile, p.X, s->n_rows, pool->d_in, p.ldx, mlora::kLongTileRows) ||
-         !encode_rows_map(&p.x_rows, p.X, s->n_rows, pool->d_in, p.ldx, 1)))
-        return MLORA_ERR_CUDA;
+    if (mode != mlora::MODE_EXPAND && run_shrink) {
+        st = setup_long_shrink(pool, s, p);
+        if (st != MLORA_OK) return st;
+    }
     if (mode != mlora::MODE_SHRINK &&
         (!encode_rows_map(&p.y_tile, p.Y, s->n_rows, pool->d_out, p.ldy, mlora::kLongTileRows) ||
          !encode_rows_map(&p.y_rows, p.Y, s->n_rows, pool->d_out, p.ldy, 1)))
@@ -317,7 +334,7 @@ mlora_status launch_long(mlora_pool *pool, const mlora_segments *s, int mode, ml
         p.ws = p.H;
         p.ws_ld = p.ldh;
     }
-    if (mode != mlora::MODE_EXPAND) {
+    if (mode != mlora::MODE_EXPAND && run_shrink) {
         e = mlora::launch_long_shrink(pool->r_bucket_max, p, long_tiles, stream);
         if (e != cudaSuccess) return MLORA_ERR_CUDA;
     }
@@ -782,13 +799,31 @@ mlora_status mlora_apply_multi(mlora_pool *const *pools, int32_t n_proj, const m
     if (mlora::launch_tile_kernel_fused(rmax, p, c, tiles * n_proj, cs) != cudaSuccess)
         return MLORA_ERR_CUDA;
     if (!use_long) return MLORA_OK;
+    // Pools of one rank bucket share one shrink launch: X's prefill rows are read once
+    // for all projections, and each projection's H lands in its own workspace.
+    bool one_shrink = n_proj > 1;
+    for (int k = 1; k < n_proj; ++k) one_shrink = one_shrink && pools[k]->r_bucket_max == p0->r_bucket_max;
+    if (one_shrink) {
+        const int rk = std::max(16, p0->r_bucket_max);
+        mlora::TileParams q = p;
+        st = setup_long_shrink(p0, segs, q);
+        if (st != MLORA_OK) return st;
+        q.ws = p0->ws;
+        q.ws_ld = rk;
+        for (int k = 0; k < n_proj; ++k) {
+            q.proj[k].ws = pools[k]->ws;
+            q.proj[k].ws_ld = rk;
+        }
+        if (mlora::launch_long_shrink(p0->r_bucket_max, q, long_tile_bound(segs), cs, n_proj) != cudaSuccess)
+            return MLORA_ERR_CUDA;
+    }
     for (int k = 0; k < n_proj; ++k) {
         mlora::TileParams q = base_params(pools[k], segs);
         q.X = p.X;
         q.ldx = ldx;
         q.Y = static_cast<__nv_bfloat16 *>(Y[k]);
         q.ldy = ldy[k];
-        st = launch_long(pools[k], segs, mlora::MODE_APPLY, q, cs, nullptr, 0);
+        st = launch_long(pools[k], segs, mlora::MODE_APPLY, q, cs, nullptr, 0, !one_shrink);
         if (st != MLORA_OK) return st;
     }
     return MLORA_OK;

@@ -84,6 +84,31 @@ def test_fused_with_long_segments():
     free()
 
 
+@pytest.mark.parametrize("d_outs,ranks", [
+    ((512, 384, 256), (8, 16, 32)),            # three projections in one long shrink
+    ((256, 512, 128, 384), (16, 64)),          # four: the largest fused shrink
+])
+def test_fused_long_shrink_several_projections(d_outs, ranks):
+    # segments of >= 128 consecutive rows: one shrink launch computes H for every
+    # projection (X's rows read once), then each projection's expand
+    W, projs = fused_case(46, 900, 512, d_outs, 4, ranks, base_frac=0.0, shuffle=False)
+    assert mlora.build_segments(W.row_slot)["max_segment_rows"] >= 128
+    Ys, flags, _ = run_fused(W, projs)
+    assert flags == [0] * len(projs)
+    check_all(W, projs, Ys, f"long, {len(d_outs)} projections")
+    free()
+
+
+def test_fused_long_segments_pools_with_different_rmax():
+    # rank buckets differ between the pools: each projection takes its own shrink
+    W, projs = fused_case(47, 700, 512, (512, 384), 4, (8, 16), base_frac=0.0, shuffle=False)
+    pools = [make_pools(W, projs[:1], r_max=16)[0], make_pools(W, projs[1:], r_max=64)[0]]
+    Ys, flags, _ = run_fused(W, projs, pools=pools)
+    assert flags == [0, 0]
+    check_all(W, projs, Ys, "long, r_max 16 / 64")
+    free()
+
+
 def test_fused_pools_with_different_rmax():
     # projection 1's pool is built for rank 64, projection 0's for rank 16
     W, projs = fused_case(43, 150, 512, (512, 384), 4, (8, 16))
