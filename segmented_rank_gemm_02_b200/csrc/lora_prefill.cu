@@ -9,9 +9,9 @@
 //
 // Shrink (long_shrink_kernel).  A thread-block cluster of `ksplit` CTAs owns a tile;
 // CTA c covers one part of d_in.  Warp 0 streams the part through an 8-stage ring:
-// per 64-column block one TMA tile load of X (128 rows
+// per 64-column block (two per stage) one TMA tile load of X (128 rows
 // x 64 columns, 128-byte swizzle) when the tile's rows are consecutive in X, else
-// one four-row TMA gather per lane, plus one bulk copy of the adapter's A block
+// one four-row TMA gather per lane, plus the adapter's A blocks (one bulk copy)
 // (pool layout [8 groups][R][8] is already the tensor core's no-swizzle K-major
 // layout).  One thread of warp 1 issues tcgen05.mma (M=128, N=rank bucket, K=16
 // each) into an fp32 accumulator in tensor memory as stages land.  The epilogue
@@ -32,9 +32,10 @@
 // mbarriers, so copies, tensor-core work, epilogue and stores overlap.
 //
 // Fused projections (mlora_apply_multi): one shrink launch serves up to four
-// projections that share X, with one A block per projection in each stage and one
-// accumulator per projection in tensor memory, so the prefill rows of X are read
-// once; each projection's H goes to its own workspace and its own expand follows.
+// projections that share X and whose pools hold every slot at the same rank, with
+// one A block per projection in each stage and one accumulator per projection in
+// tensor memory, so the prefill rows of X are read once; each projection's H goes to
+// its own workspace and its own expand follows.
 //
 // Which segments come here: those of at least 128 grouped positions whose rows are
 // consecutive in X and Y (prefill requests); see long_segment().  The shrink is
@@ -64,6 +65,9 @@ constexpr int NCH = kExpandChunk;     // d_out columns per expand chunk
 // occupancy calculation grants it), so it keeps as many blocks in flight as fit
 // (qkv_prefill step 70.8 -> 66.8 us with 8 stages instead of 4)
 constexpr int NS = 8;
+// 64-column blocks per shrink stage where four stages of two still fit (qkv_prefill
+// step 68.3-69.0 -> 67.1-67.6 us): each X row is then read in runs of 256 bytes
+constexpr int kShrinkBoxes = 2;
 constexpr int kMaxExpandStages = 6;  // expand chunk ring, as deep as shared memory allows
 constexpr int kExpandSmemCap = 224 * 1024;   // dynamic shared memory of one expand CTA
 constexpr int kMaxSplit = 8;          // CTAs per shrink cluster
@@ -77,8 +81,11 @@ __host__ __device__ constexpr int padded_rank(int r) { return r < 16 ? 16 : r; }
 template <int RMAX, int NP = 1>
 struct ShrinkCfg {
     static constexpr int RK = padded_rank(RMAX);
-    static constexpr int X_STAGE = PM * KB * 2;          // 16 KB, 128-byte swizzle
-    static constexpr int A_STAGE = (8 * RK * 16 + 1023) / 1024 * 1024;   // [8][RK][8]
+    static constexpr int X_BOX = PM * KB * 2;            // 16 KB, 128-byte swizzle
+    static constexpr int A_BOX = 8 * RK * 16;            // [8][RK][8]
+    static constexpr int NBOX = 4 * (2 * X_BOX + NP * 2 * A_BOX) <= 200 * 1024 ? kShrinkBoxes : 1;
+    static constexpr int X_STAGE = NBOX * X_BOX;
+    static constexpr int A_STAGE = (NBOX * A_BOX + 1023) / 1024 * 1024;
     static constexpr int S_STAGE = X_STAGE + NP * A_STAGE;   // multiple of 1024
     static constexpr int NSTAGE_FIT = (200 * 1024) / S_STAGE;
     static constexpr int NSTAGE = NSTAGE_FIT < NS ? NSTAGE_FIT : NS;
@@ -256,8 +263,10 @@ __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, ui
     const int p0 = ctl.tile[1], slot = ctl.tile[3];
     const int k0 = min(p.d_in, (int)crank * p.k_part);
     const int k1 = min(p.d_in, k0 + p.k_part);
-    const int nkb = (k1 - k0 + KB - 1) / KB;
-    constexpr uint32_t A_BYTES = 8 * R * 16;
+    const int nkb = (k1 - k0 + KB - 1) / KB;            // 64-column blocks
+    constexpr int NBOX = C::NBOX;
+    const int nst = (nkb + NBOX - 1) / NBOX;             // stages
+    constexpr uint32_t A_BYTES = 8 * R * 16;             // one block of A
 
     if (warp == 0) {
         // ---- copies: X block (tile or gathers) + one A block per projection per stage
@@ -268,7 +277,7 @@ __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, ui
             const int t = ctl.rows[4 * lane + q];
             r[q] = t >= 0 ? t : p.n_rows;   // absent rows read as zeros
         }
-        for (int b = 0; b < nkb; ++b) {
+        for (int b = 0; b < nst; ++b) {
             const uint32_t G = gb + b;
             const int s = (int)(G % NSTAGE);
             bool go = true;
@@ -277,46 +286,55 @@ __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, ui
             if (__shfl_sync(0xffffffffu, go ? 1 : 0, 0) == 0) break;
             uint8_t *xs = ring + s * C::S_STAGE;
             uint8_t *as = xs + C::X_STAGE;
-            const int kb0 = k0 + b * KB;
+            const int kb0 = k0 + b * NBOX * KB;
+            const int nb = min(NBOX, nkb - b * NBOX);   // blocks in this stage
             if (lane == 0) {
-                mbar_arrive_expect_tx(&ctl.full[s], (uint32_t)C::X_STAGE + NP * A_BYTES);
-                if (contiguous) tma_load_2d(xs, &p.x_tile, kb0, ctl.rows[0], &ctl.full[s]);
+                mbar_arrive_expect_tx(&ctl.full[s], (uint32_t)nb * (C::X_BOX + NP * A_BYTES));
+                // the blocks of a stage go out back to back
+                if (contiguous)
+                    for (int i = 0; i < nb; ++i)
+                        tma_load_2d(xs + i * C::X_BOX, &p.x_tile, kb0 + i * KB, ctl.rows[0], &ctl.full[s]);
 #pragma unroll
                 for (int j = 0; j < NP; ++j)
-                    bulk_load(as + j * C::A_STAGE, proj_slot_a(p, j, slot) + (int64_t)(kb0 / 8) * R * 8, A_BYTES,
-                              &ctl.full[s]);
+                    bulk_load(as + j * C::A_STAGE, proj_slot_a(p, j, slot) + (int64_t)(kb0 / 8) * R * 8,
+                              (uint32_t)nb * A_BYTES, &ctl.full[s]);
             }
             __syncwarp();
             if (!contiguous)
-                tma_gather4(xs + lane * 4 * 128, &p.x_rows, kb0, r[0], r[1], r[2], r[3], &ctl.full[s]);
+                for (int i = 0; i < nb; ++i)
+                    tma_gather4(xs + i * C::X_BOX + lane * 4 * 128, &p.x_rows, kb0 + i * KB, r[0], r[1], r[2], r[3],
+                                &ctl.full[s]);
         }
     } else if (warp == 1 && lane == 0) {
         // ---- tensor core: 4 K=16 steps per block into one fp32 accumulator per projection
         const uint32_t idesc = umma_idesc_bf16(PM, RK);
-        for (int b = 0; b < nkb; ++b) {
+        for (int b = 0; b < nst; ++b) {
             const uint32_t G = gb + b;
             const int s = (int)(G % NSTAGE);
             if (!wait_or_fail(p, ctl, &ctl.full[s], (G / NSTAGE) & 1u)) break;
             tc_fence_after();
             const uint32_t xs = smem_addr(ring + s * C::S_STAGE);
             const uint32_t as = xs + C::X_STAGE;
+            const int nb = min(NBOX, nkb - b * NBOX);
+            for (int i = 0; i < nb; ++i) {
 #pragma unroll
-            for (int st = 0; st < KB / 16; ++st) {
-                const uint64_t ad = umma_desc_sw128(xs + st * 32);
+                for (int st = 0; st < KB / 16; ++st) {
+                    const uint64_t ad = umma_desc_sw128(xs + i * C::X_BOX + st * 32);
 #pragma unroll
-                for (int j = 0; j < NP; ++j) {
-                    const uint32_t a0 = as + j * C::A_STAGE + st * 2 * R * 16;
-                    // adapter rows 8 .. 15 of bucket 8 come from the zero block
-                    const uint32_t sbo = (R == 8) ? smem_addr(zero) - a0 : 128;
-                    const uint64_t bd = umma_desc_kmajor(a0, R * 16, sbo);
-                    umma_bf16(tmem + (uint32_t)(j * RK), ad, bd, idesc, (b > 0 || st > 0) ? 1u : 0u);
+                    for (int j = 0; j < NP; ++j) {
+                        const uint32_t a0 = as + j * C::A_STAGE + (i * (KB / 16) + st) * 2 * R * 16;
+                        // adapter rows 8 .. 15 of bucket 8 come from the zero block
+                        const uint32_t sbo = (R == 8) ? smem_addr(zero) - a0 : 128;
+                        const uint64_t bd = umma_desc_kmajor(a0, R * 16, sbo);
+                        umma_bf16(tmem + (uint32_t)(j * RK), ad, bd, idesc, (b > 0 || i > 0 || st > 0) ? 1u : 0u);
+                    }
                 }
             }
             umma_commit(&ctl.bar[s]);   // stage s is free once these MMAs end
         }
         umma_commit(&ctl.done);         // the partial tiles are complete
     }
-    gb += nkb;
+    gb += nst;
     // the other threads (and lanes 1..31 of warp 1) wait here, at a hardware barrier,
     // instead of spinning beside the copy and MMA loops
     __syncthreads();

@@ -801,8 +801,12 @@ mlora_status mlora_apply_multi(mlora_pool *const *pools, int32_t n_proj, const m
     if (!use_long) return MLORA_OK;
     // Pools of one rank bucket share one shrink launch: X's prefill rows are read once
     // for all projections, and each projection's H lands in its own workspace.
+    // (The launch takes each slot's rank from pool 0 and computes projection k only where
+    // pool k holds the slot at that rank, so the pools' ranks must agree slot by slot; an
+    // adapter with another rank per target module takes one shrink per projection.)
     bool one_shrink = n_proj > 1;
-    for (int k = 1; k < n_proj; ++k) one_shrink = one_shrink && pools[k]->r_bucket_max == p0->r_bucket_max;
+    for (int k = 1; k < n_proj; ++k)
+        one_shrink = one_shrink && pools[k]->r_bucket_max == p0->r_bucket_max && pools[k]->h_rank == p0->h_rank;
     if (one_shrink) {
         const int rk = std::max(16, p0->r_bucket_max);
         mlora::TileParams q = p;

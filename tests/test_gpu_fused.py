@@ -109,6 +109,27 @@ def test_fused_long_segments_pools_with_different_rmax():
     free()
 
 
+def test_fused_long_segments_slot_ranks_differ_between_pools():
+    # an adapter may use another rank in each target module; with equal pool buckets one
+    # shrink launch serves both projections, and each H must come from its own rank
+    W, projs = fused_case(48, 900, 512, (512, 384), 4, (16, 32, 64), base_frac=0.0, shuffle=False)
+    ranks1 = np.array([r // 2 + 3 if r > 0 else r for r in W.slot_rank], dtype=W.slot_rank.dtype)
+    A1 = {s: np.ascontiguousarray(a[:ranks1[s]]) for s, a in projs[1].A.items()}
+    B1 = {s: np.ascontiguousarray(b[:, :ranks1[s]]) for s, b in projs[1].B.items()}
+    W1 = dataclasses.replace(W, slot_rank=ranks1, _proj_cache={})
+    p1 = dataclasses.replace(projs[1], A=A1, B=B1)
+    pools = [staging.make_pool(512, 512, W.n_slots, 64, W.slot_rank, W.slot_alpha, projs[0].A, projs[0].B),
+             staging.make_pool(512, 384, W.n_slots, 64, ranks1, W.slot_alpha, A1, B1)]
+    meta = mlora.build_segments(W.row_slot)
+    meta.pop("ranks", None)   # the metadata cannot carry two ranks per segment
+    assert meta["max_segment_rows"] >= 128
+    Ys, flags, _ = run_fused(W, [projs[0], p1], pools=pools, meta=meta)
+    assert flags == [0, 0]
+    assert_close(Ys[0], oracle.reference(W, projs[0]), "projection 0, its own ranks")
+    assert_close(Ys[1], oracle.reference(W1, p1), "projection 1, other ranks")
+    free()
+
+
 def test_fused_pools_with_different_rmax():
     # projection 1's pool is built for rank 64, projection 0's for rank 16
     W, projs = fused_case(43, 150, 512, (512, 384), 4, (8, 16))
