@@ -23,10 +23,12 @@
 // 128-column chunk) pairs of all long tiles are cut into one contiguous range per
 // CTA.  A producer warp streams each chunk's B rows (one 4-D TMA load: 128 columns
 // x all rank groups of the slot) and Y0 rows (TMA tile, or four-row gathers) into a
-// ring of stages; an MMA warp multiplies H_hi B^T + H_lo B^T (M=128, N=128) into
-// one of two fp32 accumulators in tensor memory; eight epilogue warps (two threads
-// per row) add s * acc to Y0 in shared memory and stage the next unit's H as bf16
-// hi + lo parts (two buffers) ahead of its chunks; a store warp writes full tiles
+// ring of stages; an MMA warp multiplies H_hi B^T + H_lo B^T (M=128, N=128, H read
+// from tensor memory) into one of two fp32 accumulators in tensor memory; eight
+// epilogue warps (two threads per row) add s * acc to Y0 in shared memory and stage
+// the next unit's H as bf16 hi + lo parts in tensor memory (two buffers, written
+// with tcgen05.st) ahead of its chunks, which leaves shared memory to the ring (four
+// stages at rank 64 instead of three: qkv_prefill 67.7 -> 65.7-66.1 us); a store warp writes full tiles
 // of consecutive rows back with TMA stores (the epilogue writes other tiles with
 // coalesced 16-byte stores) and releases the stages.  The roles meet only at
 // mbarriers, so copies, tensor-core work, epilogue and stores overlap.
@@ -99,16 +101,18 @@ struct ShrinkCfg {
 template <int RMAX>
 struct LongCfg {
     static constexpr int RK = padded_rank(RMAX);
-    static constexpr int H_BYTES = PM * RK * 2;          // one of hi / lo: [RK/8][16][8][8]
     static constexpr int B_BYTES = (NCH * RK * 2 + 1023) / 1024 * 1024;  // [RK/8][128][8]
     static constexpr int Y_BYTES = PM * NCH * 2;         // two 64-column halves, swizzled
     static constexpr int E_STAGE = B_BYTES + Y_BYTES;    // one 128-column chunk
-    static constexpr int E_FIXED = 1024 + 2 * 2 * H_BYTES + kZeroBytes;   // + H hi/lo x 2
+    static constexpr int E_FIXED = 1024 + kZeroBytes;    // alignment slack + zero block
     static constexpr int E_NB_FIT = (kExpandSmemCap - E_FIXED) / E_STAGE;
     static constexpr int E_NB = E_NB_FIT < kMaxExpandStages ? E_NB_FIT : kMaxExpandStages;
     static_assert(E_NB >= 2, "expand stage ring");
     static constexpr int E_SMEM = E_FIXED + E_NB * E_STAGE;
-    static constexpr int E_TMEM = 2 * NCH;               // two accumulators
+    // tensor memory: two fp32 accumulators of NCH columns, then two H buffers of RK
+    // columns (bf16 hi in the first RK / 2, lo in the next, two values per column)
+    static constexpr int H_TCOL = 2 * NCH;
+    static constexpr int E_TMEM = H_TCOL + 2 * RK <= 256 ? 256 : 512;
 };
 
 struct LongCtl {
@@ -517,7 +521,7 @@ __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__
 //   full[s] / empty[s]      stage ring (B rows + Y0 rows of one 128-column chunk)
 //   res[s]                  the epilogue is done with stage s (results in place)
 //   acc_full[a] / acc_empty[a]  two fp32 accumulators of 128 columns in tensor memory
-//   h_full[b] / h_empty[b]  two H buffers (hi + lo), one per work unit in flight
+//   h_full[b] / h_empty[b]  two H buffers (hi + lo, tensor memory), one per work unit in flight
 constexpr int E_WARPS = 11;
 constexpr int ET = E_WARPS * 32;     // threads per expand CTA
 constexpr int E_EPI = 256;           // epilogue threads (warps 2..9)
@@ -578,6 +582,43 @@ __device__ __forceinline__ bool exp_wait(const TileParams &p, ExpCtl &ctl, uint6
         return false;
     }
     return true;
+}
+
+// One thread's part of a tile row of H for the expand: HC columns of H (the first
+// ncols read from src, the rest zero) as bf16 hi + lo parts, two per 32-bit column, to
+// tensor memory at columns hi_col .. and lo_col .. of the thread's lane.  The row's
+// loads all go out before any is used.
+template <int HC>
+__device__ __forceinline__ void stage_h_tmem(const float *src, int ncols, uint32_t hi_col, uint32_t lo_col)
+{
+    float h[HC];
+#pragma unroll
+    for (int c = 0; c < HC; c += 4) {
+        if (c + 4 <= ncols) {
+            const float4 v = *reinterpret_cast<const float4 *>(src + c);
+            h[c] = v.x;
+            h[c + 1] = v.y;
+            h[c + 2] = v.z;
+            h[c + 3] = v.w;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) h[c + e] = c + e < ncols ? src[c + e] : 0.f;
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < HC; c += 8) {
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float h0, l0, h1, l1;
+            split_bf16(h[c + 2 * e], h0, l0);
+            split_bf16(h[c + 2 * e + 1], h1, l1);
+            hw[e] = pack_bf16x2(h0, h1);
+            lw[e] = pack_bf16x2(l0, l1);
+        }
+        tmem_st4(hi_col + c / 2, hw);
+        tmem_st4(lo_col + c / 2, lw);
+    }
 }
 
 // Work split.  The (tile, 128-column chunk) pairs of all long tiles, tile-major, are
@@ -647,8 +688,7 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ ExpCtl ctl;
     uint8_t *stages = align1024(smem_raw);
-    uint8_t *hbufs = stages + C::E_NB * C::E_STAGE;   // [2][hi, lo]
-    uint8_t *zero = hbufs + 2 * 2 * C::H_BYTES;
+    uint8_t *zero = stages + C::E_NB * C::E_STAGE;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (warp == 1) {
@@ -768,8 +808,8 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
                 const UnitInfo ui = unit_info(p, ctl.unit[k]);
                 const int hb = k & 1;
                 if (!exp_wait(p, ctl, &ctl.h_full[hb], (uint32_t)(k >> 1) & 1u)) break;
-                const uint32_t a_hi = smem_addr(hbufs + hb * 2 * C::H_BYTES);
-                const uint32_t a_lo = a_hi + C::H_BYTES;
+                const uint32_t a_hi = tmem + (uint32_t)(C::H_TCOL + hb * C::RK);
+                const uint32_t a_lo = a_hi + C::RK / 2;
                 const int RK = padded_rank(ui.R);
                 for (int ci = 0; ci < ui.nch; ++ci, ++g, ++a) {
                     const int s = (int)(g % C::E_NB);
@@ -780,14 +820,13 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
                     const uint32_t b_s = smem_addr(stages + s * C::E_STAGE);
                     const uint32_t d = tmem + ab * NCH;
                     for (int st = 0; st < RK / 16; ++st) {
-                        const uint32_t koff = st * 2 * (PM / 8) * 128;
                         const uint32_t b0 = b_s + st * 2 * NCH * 16;
                         // bucket 8: the second rank group of B is the zero block
                         const uint32_t lbo = (ui.R == 8) ? smem_addr(zero) - b0 : NCH * 16;
                         const uint64_t bd = umma_desc_kmajor(b0, lbo, 128);
-                        umma_bf16(d, umma_desc_kmajor(a_hi + koff, (PM / 8) * 128, 128), bd, idesc,
-                                  st > 0 ? 1u : 0u);
-                        umma_bf16(d, umma_desc_kmajor(a_lo + koff, (PM / 8) * 128, 128), bd, idesc, 1u);
+                        // H from tensor memory: 16 ranks = 8 columns per step
+                        umma_bf16_tmem_a(d, a_hi + st * 8, bd, idesc, st > 0 ? 1u : 0u);
+                        umma_bf16_tmem_a(d, a_lo + st * 8, bd, idesc, 1u);
                     }
                     umma_commit(&ctl.acc_full[ab]);
                 }
@@ -821,44 +860,23 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
             if (MODE == MODE_EXPAND && u.c_begin == 0 && et == 0 && !ui.ok)
                 report(p, ui.slot_rank < 0 ? kFlagStaleSlot : ui.slot_rank == 0 ? kFlagSlotEmpty : kFlagBadRank);
             if (k >= 2 && !wait_all(&ctl.h_empty[hb], (uint32_t)((k >> 1) - 1) & 1u)) return false;
+            tc_fence_after();   // the tensor core's reads of buffer hb came before these writes
             if (half == 0) ctl.rows[hb][row] = t;
             const int RK = padded_rank(ui.R);
             const int HC = RK / 2;                            // H columns of this thread
             const bool hrow = ui.ok && row < ui.nvalid;
             const float *hsrc = p.ws + (int64_t)(u.p0 + (hrow ? row : 0)) * p.ws_ld + half * HC;
-            uint8_t *ahi = hbufs + hb * 2 * C::H_BYTES;
-            uint8_t *alo = ahi + C::H_BYTES;
-            for (int jg = 0; jg < HC / 8; ++jg) {
-                float h[8];
-                if (hrow && half * HC + 8 * jg + 8 <= ui.rank) {
-                    const float4 v0 = *reinterpret_cast<const float4 *>(hsrc + 8 * jg);
-                    const float4 v1 = *reinterpret_cast<const float4 *>(hsrc + 8 * jg + 4);
-                    h[0] = v0.x; h[1] = v0.y; h[2] = v0.z; h[3] = v0.w;
-                    h[4] = v1.x; h[5] = v1.y; h[6] = v1.z; h[7] = v1.w;
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const int col = half * HC + 8 * jg + c;
-                        h[c] = (hrow && col < ui.rank) ? hsrc[8 * jg + c] : 0.f;
-                    }
-                }
-                uint4 hi, lo;
-                uint32_t *ph = reinterpret_cast<uint32_t *>(&hi);
-                uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    float h0, l0, h1, l1;
-                    split_bf16(h[2 * c], h0, l0);
-                    split_bf16(h[2 * c + 1], h1, l1);
-                    ph[c] = pack_bf16x2(h0, h1);
-                    pl[c] = pack_bf16x2(l0, l1);
-                }
-                const int j = half * (HC / 8) + jg;
-                const int off = (j * (PM / 8) + row / 8) * 128 + (row % 8) * 16;
-                *reinterpret_cast<uint4 *>(ahi + off) = hi;
-                *reinterpret_cast<uint4 *>(alo + off) = lo;
-            }
-            fence_proxy_async_smem();   // the H tile is read by the tensor core
+            const int ncols = hrow ? min(HC, max(0, ui.rank - half * HC)) : 0;
+            // this thread's row of buffer hb: hi at column half * HC / 2, lo RK_max / 2 on
+            const uint32_t tcol = tmem + ((uint32_t)(32 * quarter) << 16) +
+                                  (uint32_t)(C::H_TCOL + hb * C::RK + half * HC / 2);
+            if (HC == 8) stage_h_tmem<8>(hsrc, ncols, tcol, tcol + C::RK / 2);
+            if constexpr (RMAX >= 32)
+                if (HC == 16) stage_h_tmem<16>(hsrc, ncols, tcol, tcol + C::RK / 2);
+            if constexpr (RMAX >= 64)
+                if (HC == 32) stage_h_tmem<32>(hsrc, ncols, tcol, tcol + C::RK / 2);
+            tmem_wait_st();
+            tc_fence_before();   // the H tile is read by the tensor core
             named_sync(kEpiBar, E_EPI);
             const bool run = named_sync_and(kEpiBar, E_EPI, ui.nvalid == PM && ctl.rows[hb][row] >= 0 &&
                                                                 ctl.rows[hb][row] == ctl.rows[hb][0] + row);
