@@ -885,6 +885,8 @@ __global__ void __launch_bounds__(ET, 1) long_expand_kernel(const __grid_constan
                 ctl.unit[k].row0 = ctl.rows[hb][0];
                 mbar_arrive(&ctl.h_full[hb]);
             }
+            // every epilogue thread reads the run flag (right away when the CTA has one unit)
+            named_sync(kEpiBar, E_EPI);
             return true;
         };
 
