@@ -130,6 +130,20 @@ struct ExpandOps<R, 2> {
     uint4 y[2], y2[2];           // fp32 Y0 rows g, g + 8: columns 8t..8t+3, 8t+4..8t+7
 };
 
+// Segments whose first-tile indices a CTA keeps after its first metadata scan, so that
+// its later tiles are found by a binary search instead of another scan.  Only the
+// 128-thread kernels keep the table: they run the batches of several waves of tiles;
+// the 256-thread ones run about one wave, where a cluster rarely has a second tile.
+constexpr int kSegTable = 256;
+template <bool KEEP>
+struct SegTable {
+    int first[kSegTable];   // first tile of each segment (the next segment's, if it has none)
+};
+template <>
+struct SegTable<false> {
+    int first[1];
+};
+
 struct SharedCtl {
     uint64_t hbar[2];   // partial H tiles of the cluster landed (one per tile parity)
     int fail;           // a partial-H wait ran out: no later tile of this launch is trusted
@@ -203,9 +217,10 @@ __device__ __forceinline__ void prefetch_slices_one(const TileParams &p, const P
 // slices of that tile's adapter into L2, so that they travel while the current tile
 // runs.  Batches of several waves skip it: there the prefetches thrashed L2
 // (measured 11% slower on 2048 decode rows of 8192-wide projections).
+// first (may be null): filled with each segment's first tile (see find_tile).
 template <bool SPEC, int NT, int MODE, int RMAX, int TM>
 __device__ int scan_tiles(const TileParams &p, const uint32_t *slot_gen, int want, int want2,
-                          const ProjView &v2, SharedCtl &ctl, bool reporter)
+                          const ProjView &v2, SharedCtl &ctl, bool reporter, int *first = nullptr)
 {
     constexpr int kThreads = NT, kWarps = NT / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -257,6 +272,7 @@ __device__ int scan_tiles(const TileParams &p, const uint32_t *slot_gen, int wan
         }
         incl += before;
         const int lo = running + incl - cnt;
+        if (!SPEC && first != nullptr && g < p.n_segments && g < kSegTable) first[g] = lo;
         if (cnt > 0 && want >= lo && want < running + incl) {
             ctl.tile[0] = g;
             ctl.tile[1] = p0 + (want - lo) * TM;
@@ -276,6 +292,48 @@ __device__ int scan_tiles(const TileParams &p, const uint32_t *slot_gen, int wan
         __syncthreads();   // ctl.scan is rewritten by the next chunk
     }
     return running;
+}
+
+// Tile `want` (< the launch's tile count) after a full scan_tiles of the same
+// metadata by this CTA (at most kSegTable segments): its segment is the last one whose
+// first tile is <= want (segments without tiles of this kernel share the next one's
+// first tile, so the last such index is a segment with tiles), found by binary search
+// in first; the rest as scan_tiles leaves it in ctl.  want2 (-1: none, else a
+// valid tile) as in scan_tiles.
+template <int MODE, int RMAX, int TM>
+__device__ void find_tile(const TileParams &p, const uint32_t *slot_gen, int want, int want2, const ProjView &v2,
+                          SharedCtl &ctl, const int *first)
+{
+    const int tid = threadIdx.x;
+    auto segment_of = [&](int t) {
+        int lo = 0, hi = p.n_segments - 1;   // ctl.first[lo] <= t
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (first[mid] <= t) lo = mid;
+            else hi = mid - 1;
+        }
+        return lo;
+    };
+    if (tid == 0) {
+        const int g = segment_of(want);
+        const int a = p.slots[g];
+        ctl.tile[0] = g;
+        ctl.tile[1] = p.offsets[g] + (want - first[g]) * TM;
+        ctl.tile[2] = p.offsets[g + 1];
+        ctl.tile[3] = a;
+        ctl.tile[4] = p.ranks ? p.ranks[g] : -1;
+        ctl.seg_scale = p.scales ? p.scales[g] : 0.f;
+        ctl.stale = p.generations && slot_gen[a] != p.generations[g];
+    }
+    if constexpr (RMAX <= 16) {   // as in scan_tiles
+        if (tid == 32 && p.early && want2 >= 0 && p.ranks != nullptr) {
+            const int g2 = segment_of(want2);
+            const int R2 = rank_bucket(p.ranks[g2]);
+            const int a2 = p.slots[g2];
+            if (R2 > 0 && R2 <= RMAX && a2 >= 0 && a2 < p.n_slots) prefetch_slices_one<MODE>(p, v2, a2, R2, cluster_rank());
+        }
+    }
+    __syncthreads();
 }
 
 // Geometry of this CTA's part of a tile.
@@ -802,6 +860,8 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT, TM>::MIN_BLOCKS))
 {
     extern __shared__ __align__(16) float smem_f[];
     __shared__ SharedCtl ctl;
+    constexpr bool kTable = NT == 128;
+    __shared__ SegTable<kTable> segtab;
     const int tid = threadIdx.x;
     const uint32_t crank = cluster_rank();
     const uint32_t csize = cluster_size();
@@ -829,7 +889,8 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT, TM>::MIN_BLOCKS))
     griddep_wait();
     const int item2 = item + n_clusters;   // this cluster's next work item
     const int total = scan_tiles<false, NT, MODE, RMAX, TM>(p, p.proj[k].slot_gen, tile, item2 / np,
-                                                        p.proj[FUSED ? item2 % np : 0], ctl, reporter) *
+                                                        p.proj[FUSED ? item2 % np : 0], ctl, reporter,
+                                                        kTable ? segtab.first : nullptr) *
                       np;
     uint32_t nt = 0;   // tiles done by this CTA (parity of the exchange buffers and barriers)
     for (; item < total; item += n_clusters, ++nt) {
@@ -842,8 +903,13 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT, TM>::MIN_BLOCKS))
         const ProjView &v = p.proj[k];
         if (item != (int)cluster_index()) {
             const int next = item + n_clusters;
-            scan_tiles<false, NT, MODE, RMAX, TM>(p, v.slot_gen, tile, next / np, p.proj[FUSED ? next % np : 0],
-                                              ctl, false);
+            // later tiles: a binary search in the first scan's table, else another scan
+            if (kTable && p.n_segments <= kSegTable)
+                find_tile<MODE, RMAX, TM>(p, v.slot_gen, tile, next < total ? next / np : -1,
+                                          p.proj[FUSED ? next % np : 0], ctl, segtab.first);
+            else
+                scan_tiles<false, NT, MODE, RMAX, TM>(p, v.slot_gen, tile, next / np, p.proj[FUSED ? next % np : 0],
+                                                  ctl, false);
         }
         // every CTA of the cluster reads the same metadata and reaches the same tile
         Tile tl;
