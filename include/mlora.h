@@ -323,8 +323,8 @@ mlora_status mlora_apply_multi(mlora_pool *const *pools, int32_t n_proj,
  *     lazy module loading is what brings it onto the device), so the first
  *     mlora_apply_noalloc call finds it in place; every GPU that has held a pool keeps
  *     it until the process exits.
- *   - Only batches that take the long-segment kernels use it: n_tokens >= 128, d_in a
- *     multiple of 64, and segs->max_segment_rows either 0 (unknown) or >= 128.  Such
+ *   - Only batches that take the long-segment kernels use it: n_tokens >= 128 and
+ *     segs->max_segment_rows either 0 (unknown) or >= 128.  Such
  *     a batch needs n_tokens * max(16, bucket(r_max)) * 4 bytes (up to 16384 grouped
  *     rows for a rank-64 pool, 65536 for r_max <= 16); a larger one returns
  *     MLORA_ERR_UNSUPPORTED with nothing launched.  Other batches have no size limit.

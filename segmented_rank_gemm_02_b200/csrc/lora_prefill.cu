@@ -255,7 +255,9 @@ __device__ __forceinline__ const __nv_bfloat16 *proj_slot_a(const TileParams &p,
     return j == 0 ? p.pool + (int64_t)slot * p.slot_stride : p.proj[j].pool + (int64_t)slot * p.proj[j].slot_stride;
 }
 
-template <int RMAX, int R, int NP>
+// RAGGED: d_in is not a multiple of 64 (its last block is partial); a separate
+// instantiation, so that the common case runs the same instructions as without it.
+template <int RMAX, int R, int NP, bool RAGGED>
 __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, uint8_t *zero,
                             uint32_t tmem, uint32_t &gb, uint32_t &tc, uint32_t crank, uint32_t csize,
                             int nvalid, int rank, bool ok)
@@ -268,9 +270,9 @@ __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, ui
     const int k0 = min(p.d_in, (int)crank * p.k_part);
     const int k1 = min(p.d_in, k0 + p.k_part);
     const int nkb = (k1 - k0 + KB - 1) / KB;            // 64-column blocks
+    constexpr bool ragged = RAGGED;
     constexpr int NBOX = C::NBOX;
     const int nst = (nkb + NBOX - 1) / NBOX;             // stages
-    constexpr uint32_t A_BYTES = 8 * R * 16;             // one block of A
 
     if (warp == 0) {
         // ---- copies: X block (tile or gathers) + one A block per projection per stage
@@ -292,16 +294,30 @@ __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, ui
             uint8_t *as = xs + C::X_STAGE;
             const int kb0 = k0 + b * NBOX * KB;
             const int nb = min(NBOX, nkb - b * NBOX);   // blocks in this stage
+            // A bytes of the stage: fewer than nb blocks' only in the last block of a d_in
+            // that is not a multiple of 64 (the X copies read zeros past d_in)
+            uint32_t a_bytes = (uint32_t)nb * R * 128;
+            const int valid = ragged ? min(k1, kb0 + nb * KB) - kb0 : nb * KB;
+            if (ragged) a_bytes = (uint32_t)(valid / 8) * R * 16;
+            if (ragged && valid % 16 != 0) {
+                // the last K=16 step reads one 8-column group past d_in: zero it (X is
+                // zero there too, and stale shared memory may hold any bits)
+                for (int j = 0; j < NP; ++j)
+                    for (int o = lane * 16; o < R * 16; o += 32 * 16)
+                        *reinterpret_cast<uint4 *>(as + j * C::A_STAGE + a_bytes + o) = make_uint4(0, 0, 0, 0);
+                fence_proxy_async_smem();   // read by the tensor core
+                __syncwarp();
+            }
             if (lane == 0) {
-                mbar_arrive_expect_tx(&ctl.full[s], (uint32_t)nb * (C::X_BOX + NP * A_BYTES));
+                mbar_arrive_expect_tx(&ctl.full[s], (uint32_t)nb * C::X_BOX + NP * a_bytes);
                 // the blocks of a stage go out back to back
                 if (contiguous)
                     for (int i = 0; i < nb; ++i)
                         tma_load_2d(xs + i * C::X_BOX, &p.x_tile, kb0 + i * KB, ctl.rows[0], &ctl.full[s]);
 #pragma unroll
                 for (int j = 0; j < NP; ++j)
-                    bulk_load(as + j * C::A_STAGE, proj_slot_a(p, j, slot) + (int64_t)(kb0 / 8) * R * 8,
-                              (uint32_t)nb * A_BYTES, &ctl.full[s]);
+                    bulk_load(as + j * C::A_STAGE, proj_slot_a(p, j, slot) + (int64_t)(kb0 / 8) * R * 8, a_bytes,
+                              &ctl.full[s]);
             }
             __syncwarp();
             if (!contiguous)
@@ -320,19 +336,27 @@ __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, ui
             const uint32_t xs = smem_addr(ring + s * C::S_STAGE);
             const uint32_t as = xs + C::X_STAGE;
             const int nb = min(NBOX, nkb - b * NBOX);
-            for (int i = 0; i < nb; ++i) {
+            const int valid = ragged ? min(k1, k0 + b * NBOX * KB + nb * KB) - (k0 + b * NBOX * KB) : nb * KB;
+            // one K=16 step of block i for every projection
+            auto step = [&](int i, int st) {
+                const uint64_t ad = umma_desc_sw128(xs + i * C::X_BOX + st * 32);
 #pragma unroll
-                for (int st = 0; st < KB / 16; ++st) {
-                    const uint64_t ad = umma_desc_sw128(xs + i * C::X_BOX + st * 32);
-#pragma unroll
-                    for (int j = 0; j < NP; ++j) {
-                        const uint32_t a0 = as + j * C::A_STAGE + (i * (KB / 16) + st) * 2 * R * 16;
-                        // adapter rows 8 .. 15 of bucket 8 come from the zero block
-                        const uint32_t sbo = (R == 8) ? smem_addr(zero) - a0 : 128;
-                        const uint64_t bd = umma_desc_kmajor(a0, R * 16, sbo);
-                        umma_bf16(tmem + (uint32_t)(j * RK), ad, bd, idesc, (b > 0 || i > 0 || st > 0) ? 1u : 0u);
-                    }
+                for (int j = 0; j < NP; ++j) {
+                    const uint32_t a0 = as + j * C::A_STAGE + (i * (KB / 16) + st) * 2 * R * 16;
+                    // adapter rows 8 .. 15 of bucket 8 come from the zero block
+                    const uint32_t sbo = (R == 8) ? smem_addr(zero) - a0 : 128;
+                    const uint64_t bd = umma_desc_kmajor(a0, R * 16, sbo);
+                    umma_bf16(tmem + (uint32_t)(j * RK), ad, bd, idesc, (b > 0 || i > 0 || st > 0) ? 1u : 0u);
                 }
+            };
+            if (valid == nb * KB) {
+                for (int i = 0; i < nb; ++i) {
+#pragma unroll
+                    for (int st = 0; st < KB / 16; ++st) step(i, st);
+                }
+            } else {   // the last block of d_in: steps up to d_in only
+                for (int i = 0; i < nb; ++i)
+                    for (int st = 0; st < KB / 16 && i * KB + st * 16 < valid; ++st) step(i, st);
             }
             umma_commit(&ctl.bar[s]);   // stage s is free once these MMAs end
         }
@@ -440,7 +464,7 @@ __device__ void shrink_tile(const TileParams &p, LongCtl &ctl, uint8_t *ring, ui
     tc_fence_after();
 }
 
-template <int RMAX, int NP>
+template <int RMAX, int NP, bool RAGGED>
 __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__ TileParams p)
 {
     using C = ShrinkCfg<RMAX, NP>;
@@ -483,15 +507,15 @@ __global__ void __launch_bounds__(PT) long_shrink_kernel(const __grid_constant__
         int rank;
         const int R = tile_setup(p, ctl, nvalid, crank == 0, ok, rank);
         if (R == 8) {
-            shrink_tile<RMAX, 8, NP>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
+            shrink_tile<RMAX, 8, NP, RAGGED>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
         } else if (R == 16) {
-            shrink_tile<RMAX, 16, NP>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
+            shrink_tile<RMAX, 16, NP, RAGGED>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
         } else if (R == 32) {
             if constexpr (RMAX >= 32)
-                shrink_tile<RMAX, 32, NP>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
+                shrink_tile<RMAX, 32, NP, RAGGED>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
         } else if (R == 64) {
             if constexpr (RMAX >= 64)
-                shrink_tile<RMAX, 64, NP>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
+                shrink_tile<RMAX, 64, NP, RAGGED>(p, ctl, ring, zero, tmem, gb, tc, crank, csize, nvalid, rank, ok);
         }
         __syncthreads();
     }
@@ -1051,7 +1075,7 @@ cudaError_t shrink_active(int cluster, int &active)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaOccupancyMaxActiveClusters(&active, long_shrink_kernel<RMAX, NP>, &cfg);
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&active, long_shrink_kernel<RMAX, NP, false>, &cfg);
     if (e != cudaSuccess) return e;
     if (active <= 0) return cudaErrorInvalidConfiguration;
     int sms = 0;
@@ -1088,7 +1112,8 @@ cudaError_t shrink_rmax(const TileParams &p, int64_t max_tiles, cudaStream_t str
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, long_shrink_kernel<RMAX, NP>, p);
+    return (p.d_in % KB) ? cudaLaunchKernelEx(&cfg, long_shrink_kernel<RMAX, NP, true>, p)
+                         : cudaLaunchKernelEx(&cfg, long_shrink_kernel<RMAX, NP, false>, p);
 }
 
 template <int RMAX, int MODE>
@@ -1133,8 +1158,11 @@ template <int RMAX, int NP>
 cudaError_t set_shrink_attrs()
 {
     cudaError_t e;
-    if ((e = set_smem(long_shrink_kernel<RMAX, NP>, ShrinkCfg<RMAX, NP>::S_SMEM)) != cudaSuccess) return e;
-    return cudaFuncSetAttribute(long_shrink_kernel<RMAX, NP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    for (auto k : {long_shrink_kernel<RMAX, NP, false>, long_shrink_kernel<RMAX, NP, true>}) {
+        if ((e = set_smem(k, ShrinkCfg<RMAX, NP>::S_SMEM)) != cudaSuccess) return e;
+        if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 template <int RMAX>

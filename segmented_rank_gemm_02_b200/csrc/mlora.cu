@@ -235,7 +235,7 @@ mlora_status ensure_workspace(mlora_pool *pool, size_t bytes, cudaStream_t strea
 // segment may reach kLongRows (the host's hint, when given, rules them out).
 bool long_path(const mlora_pool *pool, const mlora_segments *s)
 {
-    return s->n_tokens >= kLongRows && pool->d_in % 64 == 0 &&
+    return s->n_tokens >= kLongRows &&
            (s->max_segment_rows <= 0 || s->max_segment_rows >= kLongRows) && pool->b_maps_ok;
 }
 

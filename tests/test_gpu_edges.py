@@ -392,3 +392,20 @@ def test_host_rejects_bad_arguments():
     Ynarrow = torch.zeros(16, 56, dtype=torch.bfloat16, device=DEVICE)   # row stride < d_out
     with pytest.raises(mlora.MloraError):
         mlora.apply(pool, st["segs"], st["X"], Ynarrow)
+
+
+@pytest.mark.parametrize("d_in,ranks", [(200, (8, 64)), (4000, (16, 32)), (136, (64,))])
+def test_long_segments_with_d_in_not_a_multiple_of_64(d_in, ranks):
+    # prefill segments whose d_in ends inside a 64-column block: 200 = 3 x 64 + 8 (the
+    # last tensor-core step half past d_in), 4000 = 62 x 64 + 32, 136 = 2 x 64 + 8; the
+    # long-segment kernels take them, with rank buckets 8 to 64
+    W = wl.random_case(90 + d_in, 900, d_in, 384, 4, ranks, base_frac=0.0, shuffle=False)
+    proj = W.projection(0)
+    meta = _meta_from_oracle(W)
+    assert int(np.diff(meta["offsets"]).max()) >= 128
+    Y, flags, _ = run_apply(W, proj, meta=meta)
+    assert flags == 0
+    ref, f = _ref(W, proj, meta)
+    assert f == 0
+    assert_close(Y, ref, f"d_in {d_in}")
+    free()
