@@ -134,6 +134,8 @@ struct ExpandOps<R, 2> {
 // its later tiles are found by a binary search instead of another scan.  Only the
 // 128-thread kernels keep the table: they run the batches of several waves of tiles;
 // the 256-thread ones run about one wave, where a cluster rarely has a second tile.
+// Of those, the fused and rank > 16 ones (measured): in the single-projection rank-16
+// kernel the table's registers cost more than the scans it saves.
 constexpr int kSegTable = 256;
 template <bool KEEP>
 struct SegTable {
@@ -860,7 +862,7 @@ __global__ void __launch_bounds__(NT, (DecodeCfg<RMAX, NT, TM>::MIN_BLOCKS))
 {
     extern __shared__ __align__(16) float smem_f[];
     __shared__ SharedCtl ctl;
-    constexpr bool kTable = NT == 128;
+    constexpr bool kTable = NT == 128 && (FUSED || RMAX > 16);
     __shared__ SegTable<kTable> segtab;
     const int tid = threadIdx.x;
     const uint32_t crank = cluster_rank();
