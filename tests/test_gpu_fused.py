@@ -241,3 +241,14 @@ def test_fused_full_size_block_attention_sampled():
     for p, Y in zip(projs, Ys):
         assert_untouched(Y, p.Y0, base, "base rows")
     free()
+
+
+def test_fused_long_shrink_with_d_in_not_a_multiple_of_64():
+    # one shrink launch for three projections whose d_in (200 = 3 x 64 + 8) ends inside a
+    # 64-column block: each projection's A copy is cut at d_in, with a zeroed group after
+    W, projs = fused_case(49, 900, 200, (256, 128, 384), 4, (8, 16, 64), base_frac=0.0, shuffle=False)
+    assert mlora.build_segments(W.row_slot)["max_segment_rows"] >= 128
+    Ys, flags, _ = run_fused(W, projs)
+    assert flags == [0] * len(projs)
+    check_all(W, projs, Ys, "long, d_in 200, 3 projections")
+    free()
