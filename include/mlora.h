@@ -292,9 +292,12 @@ mlora_status mlora_base_gemm_apply(mlora_pool *pool, const mlora_segments *segs,
  * [n_rows, d_in], shared; Y[k]: device bf16 [n_rows, d_out of pools[k]] with row
  * stride ldy[k], distinct, non-overlapping buffers.  1 <= n_proj <= MLORA_MAX_FUSED.
  * Short segments run in one launch whose work items are (tile, projection) with a
- * tile's projections side by side, so its X rows are read from HBM once; long
- * segments run the long-segment kernels once per projection, each with its pool's
- * workspace (grown as in mlora_apply, all before anything is launched).
+ * tile's projections side by side, so its X rows are read from HBM once.  Long
+ * segments: when all pools have the same rank bucket and hold every slot at the same
+ * rank, one shrink launch computes H for every projection (X's rows read once), each
+ * into its pool's workspace; otherwise each projection runs its own shrink; then each
+ * projection's expand (workspaces grown as in mlora_apply, all before anything is
+ * launched).
  * Errors: host-side as mlora_apply (plus a repeated pool or output, different
  * d_in / n_slots / device: MLORA_ERR_INVALID_ARG).  Device-side: metadata problems
  * found while scanning the segments (bad offsets or slots) go to pools[0]'s status
